@@ -1,0 +1,309 @@
+// dsa_lib.cu -- the C ABI of libdsa.so (declared in include/dsa.h): host-side argument
+// checks, launch configuration and the chunked forward orchestration.  All arithmetic
+// of the path runs in the kernels included below.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "../../include/dsa.h"
+#include "dsa_common.cuh"
+#include "indexer.cuh"
+#include "indexer_tc.cuh"
+#include "sparse_mla.cuh"
+#include "topk.cuh"
+
+namespace {
+
+using dsa::Problem;
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+dsa_status_t check_problem(const dsa_problem_t *p) {
+    if (p == nullptr) return DSA_ERR_INVALID_ARG;
+    if (p->batch < 1 || p->total_q < 0 || p->total_k < 0 || p->max_len_q < 0 || p->max_len_k < 0)
+        return DSA_ERR_INVALID_ARG;
+    if ((p->cu_q == nullptr) != (p->cu_k == nullptr)) return DSA_ERR_INVALID_ARG;
+    if (p->cu_q == nullptr) {
+        if (p->batch != 1 || p->total_q > p->total_k) return DSA_ERR_INVALID_ARG;
+        if (p->max_len_k < p->total_k || p->max_len_q < p->total_q) return DSA_ERR_INVALID_ARG;
+    }
+    if (p->max_len_q > p->max_len_k && p->cu_q == nullptr) return DSA_ERR_INVALID_ARG;
+    if (p->topk < 1) return DSA_ERR_INVALID_ARG;
+    if (p->n_idx_heads != 64 || p->idx_dim != 128 || p->n_heads != 128 || p->d_qk != 576 || p->d_v != 512)
+        return DSA_ERR_UNSUPPORTED;
+    if (p->topk > 2048) return DSA_ERR_UNSUPPORTED;
+    if (p->idx_dtype != DSA_BF16 && p->idx_dtype != DSA_E4M3) return DSA_ERR_UNSUPPORTED;
+    if (!(p->sm_scale > 0.0f)) return DSA_ERR_INVALID_ARG;
+    return DSA_OK;
+}
+
+Problem to_dev(const dsa_problem_t *p) {
+    Problem P;
+    P.batch = p->batch;
+    P.cu_q = p->cu_q;
+    P.cu_k = p->cu_k;
+    P.total_q = p->total_q;
+    P.total_k = p->total_k;
+    P.max_len_q = p->max_len_q;
+    P.max_len_k = p->max_len_k;
+    P.topk = p->topk;
+    P.sm_scale = p->sm_scale;
+    return P;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda needed).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (fn == nullptr) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// 2-D row-major tensor map with a 128-byte-swizzled box of `box_rows` rows x 128 bytes.
+bool make_tmap_rows(CUtensorMap *m, const void *base, bool fp8, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+    auto enc = tensor_map_encoder();
+    if (enc == nullptr) return false;
+    const uint32_t eb = fp8 ? 1 : 2;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * eb};
+    cuuint32_t box[2] = {128 / eb, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                     const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+inline dsa_status_t launch_status() {
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+// One-time per-process opt-in to large dynamic shared memory for each kernel.
+dsa_status_t set_smem_attrs() {
+    static bool done = false;
+    if (done) return DSA_OK;
+    cudaError_t e = cudaSuccess;
+    e = cudaFuncSetAttribute(dsa::indexer::indexer_cuda_core_kernel<false>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, dsa::indexer::CUDA_CORE_SMEM);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(dsa::indexer::indexer_cuda_core_kernel<true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, dsa::indexer::CUDA_CORE_SMEM);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(dsa::mla::sparse_mla_cuda_core_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 dsa::mla::CUDA_CORE_SMEM);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(dsa::topk::topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 200 * 1024);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(dsa::indexer::indexer_tc_kernel<8, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 dsa::indexer::TcCfg<8, false>::SMEM);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(dsa::indexer::indexer_tc_kernel<8, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 dsa::indexer::TcCfg<8, true>::SMEM);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(dsa::indexer::indexer_tc_kernel<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 dsa::indexer::TcCfg<1, false>::SMEM);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(dsa::indexer::indexer_tc_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 dsa::indexer::TcCfg<1, true>::SMEM);
+    if (e != cudaSuccess) return DSA_ERR_CUDA;
+    done = true;
+    return DSA_OK;
+}
+
+template <int QG, bool FP8>
+dsa_status_t indexer_tc_launch(const dsa_problem_t *p, const void *q_idx, const float *q_scale, const void *k_idx,
+                               const float *k_scale, const float *w, float *scores, int64_t ld, int row_begin,
+                               int row_count, cudaStream_t stream) {
+    using C = dsa::indexer::TcCfg<QG, FP8>;
+    CUtensorMap tq, tk;
+    if (!make_tmap_rows(&tq, q_idx, FP8, 128, (uint64_t)p->total_q * 64, 64)) return DSA_ERR_CUDA;
+    if (!make_tmap_rows(&tk, k_idx, FP8, 128, (uint64_t)p->total_k, 128)) return DSA_ERR_CUDA;
+    Problem P = to_dev(p);
+    int nsplit = 1;
+    unsigned grid;
+    if (QG > 1) {
+        grid = (unsigned)((row_count + QG - 1) / QG);
+    } else {
+        nsplit = (p->max_len_k + C::SPLIT_KEYS - 1) / C::SPLIT_KEYS;
+        grid = (unsigned)row_count * (unsigned)nsplit;
+    }
+    dsa::indexer::indexer_tc_kernel<QG, FP8><<<grid, C::THREADS, C::SMEM, stream>>>(
+        tq, tk, P, q_scale, k_scale, w, scores, ld, row_begin, row_count, nsplit);
+    return launch_status();
+}
+
+dsa_status_t indexer_launch(const dsa_problem_t *p, const void *q_idx, const float *q_scale, const void *k_idx,
+                            const float *k_scale, const float *w, float *scores, int64_t ld, int row_begin,
+                            int row_count, cudaStream_t stream) {
+    if (row_count == 0 || p->max_len_k == 0 || p->total_k == 0) return DSA_OK;
+    const bool fp8 = p->idx_dtype == DSA_E4M3;
+    // One sequence: groups of 8 consecutive queries share each key tile.  Ragged batches
+    // (decode): one query per CTA, its key range split across CTAs.
+    if (p->cu_q == nullptr)
+        return fp8 ? indexer_tc_launch<8, true>(p, q_idx, q_scale, k_idx, k_scale, w, scores, ld, row_begin,
+                                                row_count, stream)
+                   : indexer_tc_launch<8, false>(p, q_idx, q_scale, k_idx, k_scale, w, scores, ld, row_begin,
+                                                 row_count, stream);
+    return fp8 ? indexer_tc_launch<1, true>(p, q_idx, q_scale, k_idx, k_scale, w, scores, ld, row_begin, row_count,
+                                            stream)
+               : indexer_tc_launch<1, false>(p, q_idx, q_scale, k_idx, k_scale, w, scores, ld, row_begin, row_count,
+                                             stream);
+}
+
+dsa_status_t topk_launch(const dsa_problem_t *p, const float *scores, int64_t ld, int row_begin, int row_count,
+                         int32_t *idx, cudaStream_t stream) {
+    if (row_count == 0) return DSA_OK;
+    Problem P = to_dev(p);
+    int row_cap = 0;
+    const int max_row_cap = (200 * 1024 - dsa::topk::FIXED_SMEM) / 4;
+    if (p->max_len_k <= max_row_cap) row_cap = p->max_len_k;
+    size_t smem = dsa::topk::FIXED_SMEM + (size_t)row_cap * 4;
+    dsa::topk::topk_rows_kernel<<<row_count, dsa::topk::THREADS, smem, stream>>>(P, scores, ld, row_begin, idx,
+                                                                                  row_cap);
+    return launch_status();
+}
+
+dsa_status_t mla_launch(const dsa_problem_t *p, const void *q, const void *kv, const int32_t *idx, void *out,
+                        float *lse, cudaStream_t stream) {
+    if (p->total_q == 0) return DSA_OK;
+    Problem P = to_dev(p);
+    dim3 grid(p->total_q, dsa::mla::H / dsa::mla::CC_HG);
+    dsa::mla::sparse_mla_cuda_core_kernel<<<grid, 256, dsa::mla::CUDA_CORE_SMEM, stream>>>(
+        P, reinterpret_cast<const __nv_bfloat16 *>(q), reinterpret_cast<const __nv_bfloat16 *>(kv), idx,
+        reinterpret_cast<__nv_bfloat16 *>(out), lse);
+    return launch_status();
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int64_t scores_ld(const dsa_problem_t *p) { return (int64_t)align_up((size_t)(p->max_len_k > 0 ? p->max_len_k : 1), 4); }
+
+int effective_chunk(const dsa_problem_t *p, int32_t chunk_q) {
+    int T = p->total_q > 0 ? p->total_q : 1;
+    if (chunk_q <= 0 || chunk_q > T) return T;
+    return chunk_q;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *dsa_status_string(dsa_status_t s) {
+    switch (s) {
+        case DSA_OK: return "success";
+        case DSA_ERR_INVALID_ARG: return "invalid argument (null or misaligned pointer, or inconsistent size)";
+        case DSA_ERR_UNSUPPORTED: return "unsupported problem shape for this build";
+        case DSA_ERR_WORKSPACE: return "workspace missing or too small";
+        case DSA_ERR_CUDA: return "CUDA launch or runtime error";
+        case DSA_ERR_DEVICE_TIMEOUT: return "a device-side bounded wait gave up";
+    }
+    return "unknown status";
+}
+
+int32_t dsa_abi_version(void) { return DSA_ABI_VERSION; }
+
+dsa_status_t dsa_indexer_scores(const dsa_problem_t *p, const void *q_idx, const float *q_scale, const void *k_idx,
+                                const float *k_scale, const float *w, float *scores, int64_t ld_scores,
+                                int32_t row_begin, int32_t row_count, dsa_stream_t stream) {
+    dsa_status_t st = check_problem(p);
+    if (st != DSA_OK) return st;
+    if (row_begin < 0 || row_count < 0 || (int64_t)row_begin + row_count > p->total_q) return DSA_ERR_INVALID_ARG;
+    if (ld_scores < p->max_len_k || (ld_scores & 3) != 0) return DSA_ERR_INVALID_ARG;
+    if (row_count > 0) {
+        if (!q_idx || !k_idx || !w || !scores) return DSA_ERR_INVALID_ARG;
+        if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(w) || !aligned16(scores)) return DSA_ERR_INVALID_ARG;
+        if (p->idx_dtype == DSA_E4M3 && (!q_scale || !k_scale)) return DSA_ERR_INVALID_ARG;
+    }
+    if ((st = set_smem_attrs()) != DSA_OK) return st;
+    return indexer_launch(p, q_idx, q_scale, k_idx, k_scale, w, scores, ld_scores, row_begin, row_count,
+                          (cudaStream_t)stream);
+}
+
+dsa_status_t dsa_topk(const dsa_problem_t *p, const float *scores, int64_t ld_scores, int32_t row_begin,
+                      int32_t row_count, int32_t *idx, dsa_stream_t stream) {
+    dsa_status_t st = check_problem(p);
+    if (st != DSA_OK) return st;
+    if (row_begin < 0 || row_count < 0 || (int64_t)row_begin + row_count > p->total_q) return DSA_ERR_INVALID_ARG;
+    if (ld_scores < p->max_len_k || (ld_scores & 3) != 0) return DSA_ERR_INVALID_ARG;
+    if (row_count > 0) {
+        if (!scores || !idx || !aligned16(scores) || !aligned16(idx)) return DSA_ERR_INVALID_ARG;
+    }
+    if ((st = set_smem_attrs()) != DSA_OK) return st;
+    return topk_launch(p, scores, ld_scores, row_begin, row_count, idx, (cudaStream_t)stream);
+}
+
+dsa_status_t dsa_sparse_mla_fwd(const dsa_problem_t *p, const void *q, const void *kv, const int32_t *idx, void *out,
+                                float *lse, dsa_stream_t stream) {
+    dsa_status_t st = check_problem(p);
+    if (st != DSA_OK) return st;
+    if (p->total_q > 0) {
+        if (!q || !kv || !idx || !out || !lse) return DSA_ERR_INVALID_ARG;
+        if (!aligned16(q) || !aligned16(kv) || !aligned16(idx) || !aligned16(out) || !aligned16(lse))
+            return DSA_ERR_INVALID_ARG;
+    }
+    if ((st = set_smem_attrs()) != DSA_OK) return st;
+    return mla_launch(p, q, kv, idx, out, lse, (cudaStream_t)stream);
+}
+
+size_t dsa_forward_workspace_size(const dsa_problem_t *p, int32_t chunk_q) {
+    if (check_problem(p) != DSA_OK) return 0;
+    size_t chunk = (size_t)effective_chunk(p, chunk_q);
+    size_t scores = align_up(chunk * (size_t)scores_ld(p) * sizeof(float), 256);
+    size_t idx = align_up((size_t)(p->total_q > 0 ? p->total_q : 1) * (size_t)p->topk * sizeof(int32_t), 256);
+    return scores + idx;
+}
+
+dsa_status_t dsa_forward(const dsa_problem_t *p, const void *q_idx, const float *q_scale, const void *k_idx,
+                         const float *k_scale, const float *w, const void *q, const void *kv, int32_t chunk_q,
+                         int32_t *idx_out, void *out, float *lse, void *workspace, size_t workspace_bytes,
+                         dsa_stream_t stream) {
+    dsa_status_t st = check_problem(p);
+    if (st != DSA_OK) return st;
+    if (chunk_q < 0) return DSA_ERR_INVALID_ARG;
+    if (p->total_q == 0) return DSA_OK;
+    if (!q_idx || !k_idx || !w || !q || !kv || !out || !lse) return DSA_ERR_INVALID_ARG;
+    if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(w) || !aligned16(q) || !aligned16(kv) ||
+        !aligned16(out) || !aligned16(lse) || (idx_out && !aligned16(idx_out)))
+        return DSA_ERR_INVALID_ARG;
+    if (p->idx_dtype == DSA_E4M3 && (!q_scale || !k_scale)) return DSA_ERR_INVALID_ARG;
+    const size_t need = dsa_forward_workspace_size(p, chunk_q);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return DSA_ERR_WORKSPACE;
+    if ((st = set_smem_attrs()) != DSA_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int chunk = effective_chunk(p, chunk_q);
+    const int64_t ld = scores_ld(p);
+    float *scores = reinterpret_cast<float *>(workspace);
+    int32_t *idx = idx_out;
+    if (!idx) {
+        size_t off = align_up((size_t)chunk * (size_t)ld * sizeof(float), 256);
+        idx = reinterpret_cast<int32_t *>(reinterpret_cast<unsigned char *>(workspace) + off);
+    }
+    for (int r0 = 0; r0 < p->total_q; r0 += chunk) {
+        const int rc = p->total_q - r0 < chunk ? p->total_q - r0 : chunk;
+        st = indexer_launch(p, q_idx, q_scale, k_idx, k_scale, w, scores, ld, r0, rc, s);
+        if (st != DSA_OK) return st;
+        st = topk_launch(p, scores, ld, r0, rc, idx + (int64_t)r0 * p->topk, s);
+        if (st != DSA_OK) return st;
+    }
+    return mla_launch(p, q, kv, idx, out, lse, s);
+}
+
+dsa_status_t dsa_check_device_errors(dsa_stream_t stream) {
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return DSA_ERR_CUDA;
+    unsigned int flag = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&flag, dsa::g_error_flag, sizeof(flag)) != cudaSuccess) return DSA_ERR_CUDA;
+    if (flag != 0 && cudaMemcpyToSymbol(dsa::g_error_flag, &zero, sizeof(zero)) != cudaSuccess) return DSA_ERR_CUDA;
+    return flag ? DSA_ERR_DEVICE_TIMEOUT : DSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,251 @@
+// indexer_tc.cuh -- lightning indexer on the 5th-generation tensor cores (tcgen05).
+//
+// "DeepSeek-V3.2 tech report summary", §1 DSA, ① Lightning Indexer:
+//     I[t,s] = sum_{j<64} w[t,j] * ReLU(q_I[t,j] . k_I[s]),  s <= pos(t),  d_I = 128,
+// bf16 or FP8 (e4m3 with per-token scales).
+//
+// GEMM view: D[key, (query, head)] = k_I[key] . q_I[query, head], K = d_I = 128.
+//  * keys sit on the MMA M axis (128 per tile, one TMEM lane each) and (query, head)
+//    pairs on N (4 queries x 64 heads = 256 columns per MMA); a CTA keeps the q_I rows of
+//    QG consecutive queries resident in shared memory and streams the key tiles of their
+//    causal range through a TMA ring;
+//  * accumulators live in TMEM, double-buffered: while the tensor core fills one buffer,
+//    an epilogue warpgroup reads the other (tcgen05.ld), so each thread owns one key row
+//    and sums w[t,j] * ReLU(.) over the 64 heads of a query in registers -- no shuffles;
+//  * the fp32 score row is written coalesced (128 consecutive keys per query); keys past
+//    pos(t) are never written, tiles past the group's last position are never loaded.
+// FP8: kind::f8f6f4 MMA on e4m3 codes; since the per-token scales are positive,
+// ReLU(a*b*x) = a*b*ReLU(x) and the scales multiply the finished sum.
+//
+// Warp roles (12 warps): 0 TMA producer, 1 MMA issuer, 2 TMEM allocator, 3 idle,
+// 4-7 epilogue for accumulator buffer 0, 8-11 epilogue for buffer 1.
+#pragma once
+
+#include "dsa_common.cuh"
+#include "sm100.cuh"
+
+namespace dsa {
+namespace indexer {
+
+template <int QG, bool FP8>
+struct TcCfg {
+    static constexpr int BM = 128;                          // keys per tile = MMA M
+    static constexpr int EB = FP8 ? 1 : 2;                  // bytes per element
+    static constexpr int ROWB = 128 * EB;                   // bytes per key / query-head row
+    static constexpr int ATOMS = ROWB / 128;                // 128-byte swizzle atoms per row
+    static constexpr int KSTEP = FP8 ? 32 : 16;             // K of one MMA instruction
+    static constexpr int NKS = 128 / KSTEP;                 // MMAs per item
+    static constexpr int KS_PER_ATOM = 128 / (KSTEP * EB);  // MMAs per swizzle atom
+    static constexpr int QROWS = QG * 64;                   // B rows
+    static constexpr int N = QROWS < 256 ? QROWS : 256;     // MMA N
+    static constexpr int NSUB = QROWS / N;                  // items (MMA groups) per tile
+    static constexpr int QPI = N / 64;                      // queries per item
+    static constexpr int STAGES = (!FP8) ? 3 : 4;
+    static constexpr int KTILE_BYTES = BM * ROWB;
+    static constexpr int KATOM_BYTES = BM * 128;
+    static constexpr int Q_BYTES = QROWS * ROWB;
+    static constexpr int QATOM_BYTES = QROWS * 128;
+    static constexpr int QBOX_BYTES = 64 * 128;             // one TMA box: 64 rows x 128 bytes
+    static constexpr int TMEM_COLS = 2 * N < 32 ? 32 : 2 * N;
+    static constexpr int OFF_K = Q_BYTES;
+    static constexpr int OFF_W = OFF_K + STAGES * KTILE_BYTES;
+    static constexpr int OFF_BAR = OFF_W + QROWS * 4;
+    static constexpr int NBARS = 1 + 2 * STAGES + 4;
+    static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
+    static constexpr int SMEM = OFF_MISC + 16;
+    static constexpr int THREADS = 384;
+    static constexpr int SPLIT_KEYS = 4096;                 // key range of one CTA when QG == 1
+    static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+template <int QG, bool FP8>
+__global__ void __launch_bounds__(384, 1)
+indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k, Problem P,
+                  const float *__restrict__ q_scale, const float *__restrict__ k_scale, const float *__restrict__ w,
+                  float *__restrict__ scores, int64_t ld, int row_begin, int row_count, int nsplit) {
+    using C = TcCfg<QG, FP8>;
+    using namespace sm100;
+    extern __shared__ __align__(1024) unsigned char smem[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    // ---- which query rows and which key range this CTA owns
+    int t0, qcount, kbase, key0, nkeys_total;
+    int pos0;   // position of query t0 (queries of a group are consecutive positions)
+    if (QG > 1) {
+        const int ngroups = (row_count + QG - 1) / QG;
+        const int g = ngroups - 1 - (int)blockIdx.x;          // heaviest (latest) groups first
+        t0 = row_begin + g * QG;
+        qcount = min(QG, row_begin + row_count - t0);
+        const RowInfo ri = row_info(P, t0);                   // single sequence (cu arrays absent)
+        kbase = ri.kbase;
+        pos0 = ri.pos;
+        key0 = 0;
+        nkeys_total = min(ri.pos + qcount, ri.len_k);          // visible keys of the last query
+    } else {
+        const int r = (int)blockIdx.x / nsplit, split = (int)blockIdx.x % nsplit;
+        t0 = row_begin + r;
+        qcount = 1;
+        const RowInfo ri = row_info(P, t0);
+        kbase = ri.kbase;
+        pos0 = ri.pos;
+        key0 = split * C::SPLIT_KEYS;
+        nkeys_total = min(visible_keys(ri), key0 + C::SPLIT_KEYS);
+    }
+    if (nkeys_total <= key0) return;                          // uniform for the whole CTA
+    const int ntiles = (nkeys_total - key0 + C::BM - 1) / C::BM;
+    const int nitems = ntiles * C::NSUB;
+
+    const uint32_t sbase = smem_u32(smem);
+    if (sbase & 1023u) {                                      // SW128 operands need 1 KB alignment
+        if (tid == 0) raise_error(ERR_SMEM_ALIGN);
+        return;
+    }
+    const uint32_t q_s = sbase;
+    const uint32_t k_s = sbase + C::OFF_K;
+    float *w_s = reinterpret_cast<float *>(smem + C::OFF_W);
+    const uint32_t bar0 = sbase + C::OFF_BAR;
+    const uint32_t q_full = bar0;
+    auto k_full = [&](int s) { return bar0 + 8u * (1 + s); };
+    auto k_empty = [&](int s) { return bar0 + 8u * (1 + C::STAGES + s); };
+    auto acc_full = [&](int b) { return bar0 + 8u * (1 + 2 * C::STAGES + b); };
+    auto acc_empty = [&](int b) { return bar0 + 8u * (1 + 2 * C::STAGES + 2 + b); };
+    volatile uint32_t *misc = reinterpret_cast<volatile uint32_t *>(smem + C::OFF_MISC);  // [0] tmem base, [1] abort
+
+    if (tid == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(k_full(s), 1);
+            mbar_init(k_empty(s), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(acc_full(b), 1);
+            mbar_init(acc_empty(b), 4);
+        }
+        misc[1] = 0;
+        fence_barrier_init();
+    }
+    if (warp == 2) tmem_alloc(sbase + C::OFF_MISC, C::TMEM_COLS);
+    for (int i = tid; i < C::QROWS; i += C::THREADS) {
+        const int q = i / 64;
+        w_s[i] = q < qcount ? __ldg(w + (int64_t)(t0 + q) * 64 + (i % 64)) : 0.f;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = misc[0];
+
+    if (warp == 0 && lane == 0) {
+        // ------------------------------------------------ TMA producer
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        mbar_expect_tx(q_full, (uint32_t)(qcount * 64 * C::ROWB));
+        for (int a = 0; a < C::ATOMS; ++a)
+            for (int q = 0; q < qcount; ++q)
+                tma_load_2d(q_s + a * C::QATOM_BYTES + q * C::QBOX_BYTES, &tm_q, q_full, a * 128 / C::EB,
+                            (t0 + q) * 64);
+        for (int j = 0; j < ntiles; ++j) {
+            const int s = j % C::STAGES;
+            if (j >= C::STAGES && !mbar_wait(k_empty(s), ((j / C::STAGES) - 1) & 1)) { misc[1] = 1; break; }
+            if (misc[1]) break;
+            mbar_expect_tx(k_full(s), C::KTILE_BYTES);
+            for (int a = 0; a < C::ATOMS; ++a)
+                tma_load_2d(k_s + s * C::KTILE_BYTES + a * C::KATOM_BYTES, &tm_k, k_full(s), a * 128 / C::EB,
+                            kbase + key0 + j * C::BM);
+        }
+        // drain: the last commits on k_empty must land before the CTA may exit
+        for (int j = max(0, ntiles - C::STAGES); j < ntiles && !misc[1]; ++j)
+            if (!mbar_wait(k_empty(j % C::STAGES), (j / C::STAGES) & 1)) misc[1] = 1;
+    } else if (warp == 1 && lane == 0) {
+        // ------------------------------------------------ MMA issuer
+        const uint32_t idesc = FP8 ? idesc_e4m3(C::BM, C::N) : idesc_bf16(C::BM, C::N);
+        bool ok = mbar_wait(q_full, 0);
+        tc_fence_after();
+        int it = 0;
+        for (int j = 0; ok && j < ntiles && !misc[1]; ++j) {
+            const int s = j % C::STAGES;
+            if (!mbar_wait(k_full(s), (j / C::STAGES) & 1)) { ok = false; break; }
+            tc_fence_after();
+            for (int h = 0; h < C::NSUB; ++h, ++it) {
+                const int b = it & 1;
+                const int use = it >> 1;
+                if (use > 0 && !mbar_wait(acc_empty(b), (use - 1) & 1)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d = tmem + (uint32_t)(b * C::N);
+#pragma unroll
+                for (int kk = 0; kk < C::NKS; ++kk) {
+                    const uint32_t a_addr = k_s + s * C::KTILE_BYTES + (kk / C::KS_PER_ATOM) * C::KATOM_BYTES +
+                                            (kk % C::KS_PER_ATOM) * 32;
+                    const uint32_t b_addr = q_s + (kk / C::KS_PER_ATOM) * C::QATOM_BYTES + h * C::N * 128 +
+                                            (kk % C::KS_PER_ATOM) * 32;
+                    if (FP8)
+                        mma_f8(d, desc_sw128(a_addr), desc_sw128(b_addr), idesc, kk > 0 ? 1u : 0u);
+                    else
+                        mma_f16(d, desc_sw128(a_addr), desc_sw128(b_addr), idesc, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(acc_full(b));
+            }
+            if (!ok) break;
+            mma_commit(k_empty(s));
+        }
+        if (!ok) misc[1] = 1;
+    } else if (warp >= 4) {
+        // ------------------------------------------------ epilogue warpgroups
+        const int g = (warp - 4) >> 2;            // accumulator buffer handled by this warpgroup
+        const int quarter = warp & 3;             // TMEM lane quarter this warp may access
+        const int row = quarter * 32 + lane;      // key row inside the tile
+        const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
+        for (int it = g; it < nitems; it += 2) {
+            const int use = it >> 1;
+            if (misc[1] || !mbar_wait(acc_full(g), use & 1)) { misc[1] = 1; break; }
+            tc_fence_after();
+            const int j = it / C::NSUB, h = it % C::NSUB;
+            float res[C::QPI];
+#pragma unroll
+            for (int qi = 0; qi < C::QPI; ++qi) {
+                uint32_t v0[32], v1[32];
+                const uint32_t col = (uint32_t)(g * C::N + qi * 64);
+                tmem_ld32(t_lane + col, v0);
+                tmem_ld32(t_lane + col + 32, v1);
+                tmem_wait_ld();
+                const float *wq = w_s + (h * C::QPI + qi) * 64;
+                float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+                for (int c = 0; c < 32; c += 2) {
+                    acc0 = fmaf(wq[c], fmaxf(__uint_as_float(v0[c]), 0.f), acc0);
+                    acc1 = fmaf(wq[c + 1], fmaxf(__uint_as_float(v0[c + 1]), 0.f), acc1);
+                }
+#pragma unroll
+                for (int c = 0; c < 32; c += 2) {
+                    acc0 = fmaf(wq[32 + c], fmaxf(__uint_as_float(v1[c]), 0.f), acc0);
+                    acc1 = fmaf(wq[32 + c + 1], fmaxf(__uint_as_float(v1[c + 1]), 0.f), acc1);
+                }
+                res[qi] = acc0 + acc1;
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acc_empty(g));
+            const int key = key0 + j * C::BM + row;
+            float ks = 1.f;
+            if (FP8 && key < nkeys_total) ks = __ldg(k_scale + kbase + key);
+#pragma unroll
+            for (int qi = 0; qi < C::QPI; ++qi) {
+                const int q = h * C::QPI + qi;
+                if (q < qcount && key <= pos0 + q && key < nkeys_total) {
+                    const int t = t0 + q;
+                    float v = res[qi];
+                    if (FP8) v *= __ldg(q_scale + t) * ks;
+                    scores[(int64_t)(t - row_begin) * ld + key] = v;
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+}  // namespace indexer
+}  // namespace dsa

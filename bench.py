@@ -1,0 +1,490 @@
+#!/usr/bin/env python
+"""Benchmark of the DSA forward hot path (lightning indexer -> top-k -> sparse MLA) on B200.
+
+One step = one ``dsa_forward`` call over the whole workload (all query rows: chunked
+indexer + top-k, then the sparse MLA), inputs resident in HBM.  Default workload: one
+32K-token prefill (topk 2048).  Prints ONE JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+N > 1 (launched by torchrun) runs N independent replicas, one per GPU: the path has no
+exchange step on one problem, so there is no collective on the data path; the timing is
+the max over ranks and ``value`` counts the tokens all ranks processed.
+
+``--impl reference`` times the fp64 CPU oracle on the host cores (bounded row samples of
+the same workload); it is the slow reference arm, not a GPU implementation.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import dsa_synth  # noqa: E402
+
+METRIC = "DSA fwd tokens/s at 32K prefill (indexer+topk+sparse MLA); decode µs/step"
+L2_BYTES = 126 * 1024 * 1024
+FLOP_PER_PAIR_INDEXER = 64 * 128 * 2            # per causal (query, key) pair
+FLOP_PER_PAIR_MLA = 128 * (576 + 512) * 2       # per (query, selected key) pair, 128 heads
+
+# ncu DRAM traffic (read + write bytes per launch) of each kernel, recorded against the
+# sha256 of the source file it was captured from; reported only while the source is
+# unchanged.  Filled from the committed summaries under profiles/.
+TRAFFIC = {}
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=d["hbm_gbs"], bf16=d["bf16_tflops"], bf16_sus=d.get("bf16_tflops_sustained"),
+                    src="measured")
+    except Exception:
+        return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+def _src_sha(name: str) -> str:
+    p = os.path.join(ROOT, "attention_lightning_indexer_b200", "csrc", name)
+    try:
+        return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return ""
+
+
+# ----------------------------------------------------------------- distributed
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def _init_pg(ws, local, backend="nccl"):
+    if ws <= 1:
+        return None
+    import datetime
+
+    import torch.distributed as dist
+
+    if backend == "nccl":
+        torch.cuda.set_device(local)
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def _barrier(dist):
+    if dist is not None:
+        if dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[torch.cuda.current_device()])
+        else:
+            dist.barrier()
+
+
+def _max_over_ranks(dist, x: float) -> float:
+    if dist is None:
+        return x
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        self.path = None
+        self.uuid = None
+        try:
+            self.uuid = str(torch.cuda.get_device_properties(device).uuid)
+            if not self.uuid.startswith("GPU-"):
+                self.uuid = "GPU-" + self.uuid
+        except Exception:
+            self.uuid = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200"]
+            if self.uuid:
+                cmd.insert(1, f"--id={self.uuid}")
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
+                                 hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        load = [r for r in rows if r["power"] > 200.0] or rows
+        reasons = set()
+        for r in load:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
+                              ("pcap", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in load), "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows), "samples_under_load": len(load)}
+
+
+# ----------------------------------------------------------------- workload facts
+
+def _pairs(inp):
+    """(causal indexer pairs, selected MLA pairs, top-k algorithmic bytes) of a workload."""
+    cu_q = inp["cu_q"].cpu().numpy().astype(np.int64)
+    cu_k = inp["cu_k"].cpu().numpy().astype(np.int64)
+    k = inp["topk"]
+    idx_pairs = mla_pairs = topk_bytes = 0
+    for b in range(len(cu_q) - 1):
+        lq, lk = cu_q[b + 1] - cu_q[b], cu_k[b + 1] - cu_k[b]
+        n = np.arange(lk - lq, lk, dtype=np.int64) + 1          # visible keys per query row
+        idx_pairs += int(n.sum())
+        mla_pairs += int(np.minimum(n, k).sum())
+        topk_bytes += int((4 * n * (n > k)).sum()) + 4 * k * int(lq)
+    return idx_pairs, mla_pairs, topk_bytes
+
+
+def _tokens(inp):
+    return int(inp["total_q"])
+
+
+# ----------------------------------------------------------------- our arm
+
+def _forward_args(inp):
+    fp8 = "q_idx8" in inp
+    return dict(q_idx=inp["q_idx8"] if fp8 else inp["q_idx"], k_idx=inp["k_idx8"] if fp8 else inp["k_idx"],
+                q_scale=inp.get("q_scale"), k_scale=inp.get("k_scale"))
+
+
+def run_ours(args, ws, rank, local, dist):
+    import attention_lightning_indexer_b200 as dsa
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wl = dsa_synth.WORKLOADS[args.workload]
+    inp = dsa_synth.make_workload(args.workload, seed=args.seed, device=dev)
+    chunk = args.chunk if args.chunk is not None else wl.chunk
+    p = dsa.problem_from_inputs(inp)
+    fa = _forward_args(inp)
+    T = inp["total_q"]
+    out = torch.empty((T, 128, 512), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((T, 128), dtype=torch.float32, device=dev)
+    wsb = torch.empty(dsa.dsa_forward_workspace_size(p, chunk), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(o=out, l=lse, q=inp["q"], kv=inp["kv"], qi=fa["q_idx"], ki=fa["k_idx"], w=inp["w"]):
+        dsa.dsa_forward(p, qi, ki, w, q, kv, o, l, wsb, chunk_q=chunk, q_scale=fa["q_scale"],
+                        k_scale=fa["k_scale"], stream=stream)
+
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    dsa.dsa_check_device_errors()
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    _barrier(dist)
+    torch.cuda.synchronize(dev)
+    for i in range(args.steps):
+        flush.zero_()                      # evict L2 between timed steps (outside the events)
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize(dev)
+    _barrier(dist)
+    clk = clocks.stop()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = _max_over_ranks(dist, sum(step_ms))
+    dsa.dsa_check_device_errors()
+
+    tokens = _tokens(inp)
+    n_chunks = (T + (chunk or T) - 1) // (chunk or T)
+    launches_per_step = 2 * n_chunks + 1
+    res = {
+        "metric": METRIC,
+        "value": ws * tokens * args.steps / (total_ms / 1e3),
+        "unit": "tokens/s",
+        "n_gpus": ws,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": total_ms / args.steps,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if "q_idx8" not in inp else "e4m3 indexer + bf16 attention",
+        "data": "synthetic (seeded; shapes and distributions of the workload recipe)",
+        "config": {"workload": args.workload, "global_batch": ws * inp["batch"], "seq_len": int(inp["max_len_k"]),
+                   "topk": inp["topk"], "chunk_q": chunk, "parallelism": f"replicas x{ws}",
+                   "l2": "flushed between timed steps (2 x 126 MB write) and inputs > L2"},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
+
+    if rank == 0 and not args.no_breakdown:
+        res["roofline"], res["kernels"] = _breakdown(dsa, p, inp, fa, chunk, dev, stream, flush)
+    if not args.no_e2e:
+        res["e2e"] = _e2e(dsa, p, inp, fa, chunk, dev, stream, args, ws, dist)
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = _cpu_baseline(inp, args.cpu_rows, args.seed)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+def _breakdown(dsa, p, inp, fa, chunk, dev, stream, flush, reps=2):
+    """Average device time of each kernel of the step, timed with CUDA events on the launch stream."""
+    T = inp["total_q"]
+    chunk = chunk or T
+    ld = dsa.scores_ld(inp["max_len_k"])
+    scores = torch.empty((chunk, ld), dtype=torch.float32, device=dev)
+    idx = torch.empty((T, inp["topk"]), dtype=torch.int32, device=dev)
+    out = torch.empty((T, 128, 512), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((T, 128), dtype=torch.float32, device=dev)
+    t_idx = t_topk = t_mla = 0.0
+    n_idx = n_topk = n_mla = 0
+
+    def timed(fn):
+        flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        b.synchronize()
+        return a.elapsed_time(b)
+
+    for _ in range(reps):
+        for r0 in range(0, T, chunk):
+            rc = min(chunk, T - r0)
+            t_idx += timed(lambda: dsa.dsa_indexer_scores(p, fa["q_idx"], fa["k_idx"], inp["w"], scores, row_begin=r0,
+                                                          row_count=rc, q_scale=fa["q_scale"], k_scale=fa["k_scale"],
+                                                          stream=stream))
+            t_topk += timed(lambda: dsa.dsa_topk(p, scores, idx[r0:r0 + rc], row_begin=r0, row_count=rc,
+                                                 stream=stream))
+            n_idx += 1
+            n_topk += 1
+        t_mla += timed(lambda: dsa.dsa_sparse_mla_fwd(p, inp["q"], inp["kv"], idx, out, lse, stream=stream))
+        n_mla += 1
+    idx_pairs, mla_pairs, topk_bytes = _pairs(inp)
+    pk = _peaks()
+    fp8 = "q_idx8" in inp
+    idx_peak = pk["bf16"] * (2.0 if fp8 else 1.0)
+    kernels = {
+        "indexer": {"ms_per_launch": t_idx / n_idx, "launches_per_step": n_idx // reps,
+                    "ms_per_step": t_idx / reps, "tflops": idx_pairs * FLOP_PER_PAIR_INDEXER / (t_idx / reps) / 1e9,
+                    "peak_tflops": idx_peak},
+        "topk": {"ms_per_launch": t_topk / n_topk, "launches_per_step": n_topk // reps, "ms_per_step": t_topk / reps,
+                 "gbs": topk_bytes / (t_topk / reps) / 1e6, "peak_gbs": pk["hbm_gbs"]},
+        "sparse_mla": {"ms_per_launch": t_mla / n_mla, "launches_per_step": 1, "ms_per_step": t_mla / reps,
+                       "tflops": mla_pairs * FLOP_PER_PAIR_MLA / (t_mla / reps) / 1e9, "peak_tflops": pk["bf16"]},
+    }
+    dom = max(kernels, key=lambda k: kernels[k]["ms_per_step"])
+    kd = kernels[dom]
+    src = {"indexer": "indexer.cuh", "topk": "topk.cuh", "sparse_mla": "sparse_mla.cuh"}[dom]
+    tr = TRAFFIC.get(dom)
+    traffic = tr["bytes_per_launch"] if tr and tr.get("src_sha") == _src_sha(src) else None
+    if dom == "topk":
+        roof = {"bound": "hbm", "achieved": kd["gbs"], "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": kd["gbs"] / pk["hbm_gbs"], "traffic": traffic}
+    else:
+        roof = {"bound": "tensor", "achieved": kd["tflops"], "peak": kd["peak_tflops"], "unit": "TFLOP/s",
+                "frac": kd["tflops"] / kd["peak_tflops"], "traffic": traffic}
+    roof.update({"kernel": dom, "peak_source": pk["src"] + " (MEASURED_PEAKS burst figure)"
+                 if pk["src"] == "measured" else "fallback"})
+    return roof, kernels
+
+
+def _e2e(dsa, p, inp, fa, chunk, dev, stream, args, ws, dist):
+    """Same metric through the public call with host buffers: H2D of the step's inputs from
+    pinned memory, dsa_forward, D2H of the result (out + lse), all inside the timed region."""
+    names = [n for n in ("q_idx", "q_idx8", "q_scale", "k_idx", "k_idx8", "k_scale", "w", "q", "kv") if n in inp]
+    host = {n: inp[n].cpu().pin_memory() for n in names}
+    devb = {n: torch.empty_like(inp[n]) for n in names}
+    T = inp["total_q"]
+    out = torch.empty((T, 128, 512), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((T, 128), dtype=torch.float32, device=dev)
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    wsb = torch.empty(dsa.dsa_forward_workspace_size(p, chunk), dtype=torch.uint8, device=dev)
+    fp8 = "q_idx8" in inp
+
+    def step():
+        for n in names:
+            devb[n].copy_(host[n], non_blocking=True)
+        dsa.dsa_forward(p, devb["q_idx8" if fp8 else "q_idx"], devb["k_idx8" if fp8 else "k_idx"], devb["w"],
+                        devb["q"], devb["kv"], out, lse, wsb, chunk_q=chunk, q_scale=devb.get("q_scale"),
+                        k_scale=devb.get("k_scale"), stream=stream)
+        out_h.copy_(out, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize(dev)
+    steps = max(1, min(args.steps, 3))
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    _barrier(dist)
+    torch.cuda.synchronize(dev)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    _barrier(dist)
+    ms = _max_over_ranks(dist, a.elapsed_time(b)) / steps
+    h2d = sum(host[n].numel() * host[n].element_size() for n in names)
+    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * lse_h.element_size()
+    return {"value": ws * _tokens(inp) / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps}
+
+
+# ----------------------------------------------------------------- oracle (CPU) arms
+
+def _oracle_inputs_host(inp):
+    """Host copies the oracle reads: full key-side tensors, query-side tensors stay on device."""
+    keys = {n: inp[n].cpu() for n in ("k_idx", "k_idx8", "k_scale", "kv") if n in inp}
+    return keys
+
+
+def _oracle_forward_rows(inp, keys, rows):
+    import oracle
+
+    rt = torch.from_numpy(rows)
+    cu_q = inp["cu_q"].cpu().numpy()
+    cu_k = inp["cu_k"].cpu().numpy()
+    dev_rows = rt.to(inp["w"].device)
+    w = inp["w"][dev_rows].cpu()
+    q = inp["q"][dev_rows].cpu()
+    if "q_idx8" in inp:
+        sc = oracle.indexer_fp8(inp["q_idx8"][dev_rows].cpu(), inp["q_scale"][dev_rows].cpu(), w, keys["k_idx8"],
+                                keys["k_scale"], rows=rows, cu_q=cu_q, cu_k=cu_k, ld=inp["max_len_k"])
+    else:
+        sc = oracle.indexer(inp["q_idx"][dev_rows].cpu(), w, keys["k_idx"], rows=rows, cu_q=cu_q, cu_k=cu_k,
+                            ld=inp["max_len_k"])
+    ix = oracle.topk(sc, inp["topk"], rows=rows, cu_q=cu_q, cu_k=cu_k)
+    oracle.sparse_mla(q, keys["kv"], ix, dsa_synth.SM_SCALE, rows=rows, cu_q=cu_q, cu_k=cu_k)
+
+
+def _cpu_baseline(inp, n_rows, seed):
+    import oracle
+
+    keys = _oracle_inputs_host(inp)
+    rng = np.random.default_rng(seed + 1234)
+    rows = np.sort(rng.choice(inp["total_q"], size=min(n_rows, inp["total_q"]), replace=False)).astype(np.int64)
+    t0 = time.perf_counter()
+    _oracle_forward_rows(inp, keys, rows)
+    dt = time.perf_counter() - t0
+    return {"value": len(rows) / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{len(rows)} uniformly drawn query rows of the same workload (full indexer row, top-k, "
+                      f"sparse MLA per row), fp64, {dt:.1f} s"}
+
+
+def run_reference(args, ws, rank, local):
+    if rank != 0:
+        return
+    import oracle
+
+    dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
+    inp = dsa_synth.make_workload(args.workload, seed=args.seed, device=dev)
+    keys = _oracle_inputs_host(inp)
+    rng = np.random.default_rng(args.seed + 99)
+    per_step = min(args.cpu_rows, inp["total_q"])
+
+    def step():
+        rows = np.sort(rng.choice(inp["total_q"], size=per_step, replace=False)).astype(np.int64)
+        _oracle_forward_rows(inp, keys, rows)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = per_step * args.steps / dt
+    wl = dsa_synth.WORKLOADS[args.workload]
+    res = {
+        "impl": "reference",
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded; same recipe)",
+        "config": {"workload": args.workload, "global_batch": inp["batch"], "seq_len": int(inp["max_len_k"]),
+                   "topk": inp["topk"], "chunk_q": wl.chunk, "parallelism": "host cores (rank 0 only)"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": f"{per_step} uniformly drawn query rows per step of the same workload, fp64"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="prefill_32k", choices=sorted(dsa_synth.WORKLOADS))
+    ap.add_argument("--chunk", type=int, default=None, help="query rows per indexer/top-k chunk (0 = all)")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cpu-rows", type=int, default=48, help="oracle rows per CPU sample")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-breakdown", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    ws, rank, local = _dist()
+    if args.impl == "reference":
+        run_reference(args, ws, rank, local)
+        return
+    dist = _init_pg(ws, local)
+    try:
+        run_ours(args, ws, rank, local, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

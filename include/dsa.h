@@ -1,0 +1,172 @@
+/*
+ * dsa.h -- C ABI of libdsa.so: the DeepSeek Sparse Attention (DSA) forward hot path
+ * on one NVIDIA B200 (sm_100a).
+ *
+ * The path (definitions from "DeepSeek-V3.2 tech report summary", section 1
+ * "DeepSeek Sparse Attention (DSA)"; shapes from "DeepSeek-V3.2" (miles docs) §1):
+ *   1. lightning indexer   I[t,s] = sum_{j<H_I} w[t,j] * ReLU(q_I[t,j] . k_I[s]),  s <= pos(t)
+ *   2. top-k selection     the k_eff = min(topk, pos(t)+1) largest I[t,.] per query
+ *   3. sparse MLA (MQA)    softmax attention of 128 heads over only the selected latent
+ *                          rows; each 576-d latent row (512 KV-LoRA + 64 RoPE) is shared
+ *                          by all heads, the value is its first 512 dims, scale 1/sqrt(192)
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Ownership: every data pointer is caller-owned DEVICE memory (except the
+ *    dsa_problem_t itself, which is host memory read during the call).  The library
+ *    never allocates, frees or synchronises; work is enqueued on `stream` and runs
+ *    asynchronously in stream order.
+ *  - Layout: dense row-major, last dimension innermost, every base pointer 16-byte
+ *    aligned.  bf16 is IEEE bfloat16; e4m3 is OCP FP8 E4M3 ("fn": no infinities).
+ *  - Ragged batches: sequence b owns query rows [cu_q[b], cu_q[b+1]) and key rows
+ *    [cu_k[b], cu_k[b+1]).  Its queries are its LAST len_q(b) tokens, so the query in
+ *    global row t of sequence b sits at position
+ *        pos(t) = len_k(b) - len_q(b) + (t - cu_q[b])
+ *    and sees keys 0..pos(t) of its own sequence ("preceding tokens", the token
+ *    itself included).  Key indices are positions within the sequence.
+ *  - Errors: argument, shape and alignment checks run on the host before anything
+ *    is launched and return DSA_ERR_INVALID_ARG / DSA_ERR_UNSUPPORTED without side
+ *    effects.  A failed launch returns DSA_ERR_CUDA.  Device-side bounded waits that
+ *    give up set a sticky device flag, reported by dsa_check_device_errors().
+ *    Nothing traps, nothing aborts, and no C++ exception crosses this ABI.
+ */
+#ifndef DSA_H_
+#define DSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DSA_ABI_VERSION 1
+
+/* Same object as cudaStream_t; NULL = the legacy default stream. */
+typedef struct CUstream_st *dsa_stream_t;
+
+typedef enum dsa_status {
+    DSA_OK = 0,
+    DSA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, negative or inconsistent size */
+    DSA_ERR_UNSUPPORTED = 2,   /* a shape this build does not implement (see below) */
+    DSA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than dsa_forward_workspace_size */
+    DSA_ERR_CUDA = 4,          /* a CUDA launch or query failed */
+    DSA_ERR_DEVICE_TIMEOUT = 5 /* a device-side bounded wait gave up (from dsa_check_device_errors) */
+} dsa_status_t;
+
+typedef enum dsa_dtype {
+    DSA_BF16 = 0,
+    DSA_E4M3 = 1
+} dsa_dtype_t;
+
+/*
+ * One DSA problem.  Sizes this build implements: n_idx_heads = 64, idx_dim = 128,
+ * n_heads = 128, d_qk = 576, d_v = 512 (the DeepSeek-V3.2 shapes), 1 <= topk <= 2048.
+ * Other values return DSA_ERR_UNSUPPORTED.
+ */
+typedef struct dsa_problem {
+    int32_t batch;          /* B >= 1 */
+    const int32_t *cu_q;    /* device [B+1] query-row offsets, cu_q[0] = 0; NULL only if B == 1 */
+    const int32_t *cu_k;    /* device [B+1] key-row offsets, cu_k[0] = 0;   NULL only if B == 1 */
+    int32_t total_q;        /* T  = cu_q[B] */
+    int32_t total_k;        /* S  = cu_k[B] */
+    int32_t max_len_q;      /* >= every len_q(b) */
+    int32_t max_len_k;      /* >= every len_k(b); every len_q(b) <= len_k(b) */
+    int32_t n_idx_heads;    /* H_I = 64 */
+    int32_t idx_dim;        /* d_I = 128 */
+    int32_t n_heads;        /* H = 128 */
+    int32_t d_qk;           /* 576 = 512 latent + 64 RoPE */
+    int32_t d_v;            /* 512 */
+    int32_t topk;           /* index_topk, e.g. 2048 */
+    dsa_dtype_t idx_dtype;  /* indexer inputs: DSA_BF16 or DSA_E4M3 (per-token scales) */
+    float sm_scale;         /* attention softmax scale, 1/sqrt(192) for DeepSeek-V3.2 */
+} dsa_problem_t;
+
+/*
+ * Lightning indexer ("DeepSeek-V3.2 tech report summary", §1 DSA, ① Lightning
+ * Indexer; heads/dims from "Model techniques map -- DeepSeek-V3.2", indexer wq_b/wk):
+ *     scores[r, s] = sum_j w[t,j] * ReLU( sum_d q_idx[t,j,d] * k_idx[kbase(b)+s, d] )
+ * for query rows t = row_begin + r, 0 <= r < row_count, and 0 <= s <= pos(t).
+ * Entries with s > pos(t) are left unspecified (callers must not read them).
+ *   q_idx   : [T, H_I, d_I]  bf16, or e4m3 codes when idx_dtype == DSA_E4M3
+ *   q_scale : [T]  fp32 per-query-token scale (e4m3 only; NULL for bf16)
+ *   k_idx   : [S, d_I]       bf16 or e4m3 codes
+ *   k_scale : [S]  fp32 per-key-token scale (e4m3 only; NULL for bf16)
+ *   w       : [T, H_I] fp32
+ *   scores  : [row_count, ld_scores] fp32, ld_scores >= max_len_k, ld_scores % 4 == 0
+ * Accumulation is fp32 (tensor cores); the e4m3 scales are applied in fp32.
+ */
+dsa_status_t dsa_indexer_scores(const dsa_problem_t *p, const void *q_idx, const float *q_scale,
+                                const void *k_idx, const float *k_scale, const float *w,
+                                float *scores, int64_t ld_scores, int32_t row_begin,
+                                int32_t row_count, dsa_stream_t stream);
+
+/*
+ * Top-k token selection ("DeepSeek-V3.2 tech report summary", §1 DSA, ② fine-grained
+ * token selection; "Model techniques map -- DeepSeek-V3.2", Indexer-selected sparse
+ * attention: topk = min(index_topk, len), int32 indices):
+ * for each query row t = row_begin + r, idx[r, :] receives the k_eff = min(topk, pos(t)+1)
+ * positions s <= pos(t) with the largest scores[r, s], ranked by (score desc, s asc)
+ * with -0.0 == +0.0; slots k_eff..topk-1 are -1.  The order of the selected indices
+ * within a row is unspecified.  Exact: no approximation, deterministic.
+ *   scores : [row_count, ld_scores] fp32 (NaN-free in columns 0..pos(t))
+ *   idx    : [row_count, topk] int32
+ */
+dsa_status_t dsa_topk(const dsa_problem_t *p, const float *scores, int64_t ld_scores,
+                      int32_t row_begin, int32_t row_count, int32_t *idx, dsa_stream_t stream);
+
+/*
+ * Sparse MLA forward in MQA mode ("DeepSeek-V3.2 tech report summary", §1 DSA,
+ * MLA-based implementation: each latent KV entry is shared by all query heads;
+ * latent = 512 KV-LoRA + 64 RoPE per "Model techniques map -- DeepSeek-V3.2",
+ * Multi-head latent attention):
+ *   z[t,h,i] = sm_scale * q[t,h,:] . kv[kbase(b)+idx[t,i], :]        (576 dims)
+ *   out[t,h,:] = sum_i softmax_i(z) * kv[kbase(b)+idx[t,i], 0:512]
+ *   lse[t,h]   = log(sum_i exp(z[t,h,i]))                              (natural log)
+ * over the slots i whose index satisfies 0 <= idx <= pos(t); every other slot (-1,
+ * future or out-of-range positions) is masked, so causality holds for any input.
+ * A row with no valid slot gets out = 0 and lse = -inf.  A repeated index counts once
+ * per occurrence.
+ *   q   : [T, 128, 576] bf16     kv  : [S, 576] bf16     idx : [T, topk] int32
+ *   out : [T, 128, 512] bf16 (round-to-nearest-even from fp32)   lse : [T, 128] fp32
+ */
+dsa_status_t dsa_sparse_mla_fwd(const dsa_problem_t *p, const void *q, const void *kv,
+                                const int32_t *idx, void *out, float *lse, dsa_stream_t stream);
+
+/*
+ * Bytes of workspace dsa_forward needs for this problem when it processes the
+ * queries in chunks of `chunk_q` rows (0 = one chunk of max(T, 1) rows).
+ */
+size_t dsa_forward_workspace_size(const dsa_problem_t *p, int32_t chunk_q);
+
+/*
+ * The whole path: for each chunk of chunk_q query rows, indexer scores into the
+ * workspace, top-k into idx_out (or the workspace when idx_out is NULL), then the
+ * sparse MLA for all rows.  Same tensors and rules as the three calls above; the
+ * full T x S score matrix is never materialised (at most chunk_q x max_len_k).
+ *   idx_out   : [T, topk] int32 or NULL
+ *   workspace : device, >= dsa_forward_workspace_size(p, chunk_q) bytes, 256-byte aligned
+ */
+dsa_status_t dsa_forward(const dsa_problem_t *p, const void *q_idx, const float *q_scale,
+                         const void *k_idx, const float *k_scale, const float *w, const void *q,
+                         const void *kv, int32_t chunk_q, int32_t *idx_out, void *out, float *lse,
+                         void *workspace, size_t workspace_bytes, dsa_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the device-side error flag of the
+ * current device (set by a kernel whose bounded wait gave up).  Returns DSA_OK,
+ * DSA_ERR_DEVICE_TIMEOUT, or DSA_ERR_CUDA if the synchronisation itself failed.
+ */
+dsa_status_t dsa_check_device_errors(dsa_stream_t stream);
+
+/* Static English description of a status code (never NULL). */
+const char *dsa_status_string(dsa_status_t s);
+
+/* DSA_ABI_VERSION of the loaded library. */
+int32_t dsa_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H_ */

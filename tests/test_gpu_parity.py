@@ -1,0 +1,304 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the same
+seeded inputs.  Tolerances are defined in gpu_utils.py and restated there.
+
+Small sizes compare every element and span several tiles plus a ragged tail; the
+full-size workloads compare sampled rows in the launch configuration bench.py times.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import attention_lightning_indexer_b200 as dsa
+import dsa_synth
+import oracle
+from gpu_utils import (LSE_ATOL, O_ATOL, RECALL_MIN, assert_scores_close, fp8_to_f64, recall_excluding_near_ties,
+                       sample_rows, score_bound_row, sorted_rows)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+SCALE = dsa_synth.SM_SCALE
+
+
+def _scores_buffer(rows: int, max_len_k: int, fill=float("nan")):
+    return torch.full((rows, dsa.scores_ld(max_len_k)), fill, dtype=torch.float32, device=DEV)
+
+
+def _cu(lens_q, lens_k):
+    cu_q = np.concatenate([[0], np.cumsum(lens_q)]).astype(np.int32)
+    cu_k = np.concatenate([[0], np.cumsum(lens_k)]).astype(np.int32)
+    return cu_q, cu_k
+
+
+# ------------------------------------------------------------------------- top-k
+
+def _tie_heavy_scores(rows, cols, seed):
+    g = torch.Generator().manual_seed(seed)
+    sc = torch.randn(rows, cols, generator=g).mul_(4).round_().div_(4)
+    sc[torch.rand(rows, cols, generator=g) < 0.02] = -0.0
+    sc[torch.rand(rows, cols, generator=g) < 0.02] = 0.0
+    return sc
+
+
+@pytest.mark.parametrize("L,k", [(256, 64), (700, 128), (5000, 2048), (3000, 1), (2100, 2048)])
+def test_topk_bit_exact_on_identical_scores(L, k):
+    sc = _tie_heavy_scores(L, L, seed=L + k)
+    above = torch.triu(torch.ones(L, L, dtype=torch.bool), 1)
+    sc = sc.masked_fill(above, 1e30)          # future entries: never read by either side
+    sc_gpu = _scores_buffer(L, L)
+    sc_gpu[:, :L] = sc.to(DEV)
+    p = dsa.make_problem(1, L, L, L, L, k)
+    idx = torch.full((L, k), -7, dtype=torch.int32, device=DEV)
+    dsa.dsa_topk(p, sc_gpu, idx)
+    ref = oracle.topk(sc_gpu[:, :L].cpu(), k)
+    np.testing.assert_array_equal(sorted_rows(idx.cpu().numpy()), sorted_rows(ref))
+
+
+def test_topk_long_rows_from_global_memory_and_ragged_batch():
+    # Sequence 0 is longer than the shared-memory staging capacity; sequence 1 is short.
+    lens_k = [60000, 1000]
+    lens_q = [3, 3]
+    cu_q, cu_k = _cu(lens_q, lens_k)
+    k = 2048
+    sc = _tie_heavy_scores(6, 60000, seed=5)
+    sc_gpu = _scores_buffer(6, 60000, fill=0.0)
+    sc_gpu[:, :60000] = sc.to(DEV)
+    p = dsa.make_problem(2, 6, sum(lens_k), 3, 60000, k, cu_q=torch.from_numpy(cu_q).to(DEV),
+                         cu_k=torch.from_numpy(cu_k).to(DEV))
+    idx = torch.empty((6, k), dtype=torch.int32, device=DEV)
+    dsa.dsa_topk(p, sc_gpu, idx)
+    ref = oracle.topk(sc_gpu.cpu()[:, :60000], k, rows=np.arange(6), cu_q=cu_q, cu_k=cu_k)
+    np.testing.assert_array_equal(sorted_rows(idx.cpu().numpy()), sorted_rows(ref))
+
+
+def test_topk_row_subrange_and_empty_rows():
+    L, k = 300, 32
+    sc = _tie_heavy_scores(L, L, seed=9)
+    sc_gpu = _scores_buffer(100, L, fill=0.0)
+    sc_gpu[:, :L] = sc[150:250].to(DEV)
+    p = dsa.make_problem(1, L, L, L, L, k)
+    idx = torch.empty((100, k), dtype=torch.int32, device=DEV)
+    dsa.dsa_topk(p, sc_gpu, idx, row_begin=150, row_count=100)
+    ref = oracle.topk(sc_gpu.cpu()[:, :L], k, rows=np.arange(150, 250), cu_q=[0, L], cu_k=[0, L])
+    np.testing.assert_array_equal(sorted_rows(idx.cpu().numpy()), sorted_rows(ref))
+    dsa.dsa_topk(p, sc_gpu, idx, row_begin=0, row_count=0)   # empty launch is a no-op
+
+
+# ----------------------------------------------------------------------- indexer
+
+def _oracle_scores(inp, rows):
+    rows_t = torch.from_numpy(rows)
+    cu_q = inp["cu_q"].cpu().numpy()
+    cu_k = inp["cu_k"].cpu().numpy()
+    if "q_idx8" in inp:
+        qr = inp["q_idx8"].cpu()[rows_t]
+        qs = inp["q_scale"].cpu()[rows_t]
+        ref = oracle.indexer_fp8(qr, qs, inp["w"].cpu()[rows_t], inp["k_idx8"].cpu(), inp["k_scale"].cpu(),
+                                 rows=rows, cu_q=cu_q, cu_k=cu_k, ld=inp["max_len_k"])
+        return ref
+    return oracle.indexer(inp["q_idx"].cpu()[rows_t], inp["w"].cpu()[rows_t], inp["k_idx"].cpu(), rows=rows,
+                          cu_q=cu_q, cu_k=cu_k, ld=inp["max_len_k"])
+
+
+def _bound_rows(inp, rows):
+    """Per listed row, the score tolerance scale of its visible keys 0..pos(t)."""
+    pos = _positions(inp, rows)
+    kb = _kbase(inp, rows)
+    if "q_idx8" in inp:
+        q_all = inp["q_idx8"].cpu()
+        k_all = fp8_to_f64(inp["k_idx8"].cpu()) * inp["k_scale"].cpu().double()[:, None]
+    else:
+        q_all = inp["q_idx"].cpu()
+        k_all = inp["k_idx"].cpu()
+    w_all = inp["w"].cpu()
+    out = []
+    for i, t in enumerate(rows):
+        if "q_idx8" in inp:
+            qr = fp8_to_f64(q_all[int(t)]) * float(inp["q_scale"][int(t)])
+        else:
+            qr = q_all[int(t)]
+        n = int(pos[i]) + 1
+        out.append(score_bound_row(qr, w_all[int(t)], k_all[int(kb[i]):int(kb[i]) + n]))
+    return out
+
+
+def _positions(inp, rows):
+    return oracle.positions(rows, inp["cu_q"].cpu().numpy(), inp["cu_k"].cpu().numpy())
+
+
+def _kbase(inp, rows):
+    cu_q = inp["cu_q"].cpu().numpy()
+    cu_k = inp["cu_k"].cpu().numpy()
+    return np.array([cu_k[np.searchsorted(cu_q, t, side="right") - 1] for t in rows])
+
+
+def _gpu_scores(inp, p):
+    T = inp["total_q"]
+    sc = _scores_buffer(T, inp["max_len_k"])
+    if "q_idx8" in inp:
+        dsa.dsa_indexer_scores(p, inp["q_idx8"], inp["k_idx8"], inp["w"], sc, q_scale=inp["q_scale"],
+                               k_scale=inp["k_scale"])
+    else:
+        dsa.dsa_indexer_scores(p, inp["q_idx"], inp["k_idx"], inp["w"], sc)
+    return sc
+
+
+def _check_indexer(inp, rows):
+    p = dsa.problem_from_inputs(inp)
+    sc = _gpu_scores(inp, p).cpu().numpy()[rows]
+    ref = _oracle_scores(inp, rows)
+    pos = _positions(inp, rows)
+    assert_scores_close(sc, ref, _bound_rows(inp, rows), pos)
+
+
+@pytest.mark.parametrize("L,seed", [(256, 0), (700, 1), (1000, 2)])
+def test_indexer_bf16_all_rows(L, seed):
+    inp = dsa_synth.make_prefill(L, topk=64, seed=seed, device=DEV)
+    _check_indexer(inp, np.arange(L))
+
+
+def test_indexer_fp8_all_rows():
+    inp = dsa_synth.make_prefill(700, topk=64, seed=3, device=DEV, fp8_indexer=True)
+    _check_indexer(inp, np.arange(700))
+
+
+def test_indexer_ragged_batch_several_queries_per_sequence():
+    inp = dsa_synth.make_decode(5, 150, 900, topk=64, seed=4, device=DEV, q_per_seq=3)
+    _check_indexer(inp, np.arange(inp["total_q"]))
+
+
+# ---------------------------------------------------------------- sparse MLA
+
+def _random_idx(inp, k, seed, sprinkle_invalid=True):
+    rng = np.random.default_rng(seed)
+    T = inp["total_q"]
+    pos = _positions(inp, np.arange(T))
+    idx = np.full((T, k), -1, dtype=np.int32)
+    for t in range(T):
+        n = min(k, int(pos[t]) + 1)
+        idx[t, :n] = rng.choice(int(pos[t]) + 1, n, replace=False)
+        if sprinkle_invalid and n < k:
+            idx[t, n] = int(pos[t]) + 1 + rng.integers(0, 5)   # future key: masked
+            if n + 1 < k:
+                idx[t, n + 1] = -3
+        rng.shuffle(idx[t])
+    return idx
+
+
+def _check_mla(inp, idx_np, rows=None):
+    T = inp["total_q"]
+    p = dsa.problem_from_inputs(inp)
+    idx = torch.from_numpy(idx_np).to(DEV)
+    out = torch.empty((T, 128, 512), dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty((T, 128), dtype=torch.float32, device=DEV)
+    dsa.dsa_sparse_mla_fwd(p, inp["q"], inp["kv"], idx, out, lse)
+    rows = np.arange(T) if rows is None else rows
+    rt = torch.from_numpy(rows)
+    o_ref, lse_ref = oracle.sparse_mla(inp["q"].cpu()[rt], inp["kv"].cpu(), idx_np[rows], SCALE, rows=rows,
+                                       cu_q=inp["cu_q"].cpu().numpy(), cu_k=inp["cu_k"].cpu().numpy())
+    o = out.cpu()[rt].double().numpy()
+    ls = lse.cpu()[rt].double().numpy()
+    assert np.max(np.abs(o - o_ref)) <= O_ATOL
+    fin = np.isfinite(lse_ref)
+    assert np.array_equal(fin, np.isfinite(ls))
+    assert np.max(np.abs(ls[fin] - lse_ref[fin]), initial=0.0) <= LSE_ATOL
+    return out, lse
+
+
+@pytest.mark.parametrize("L,k,std", [(256, 64, 1 / 24), (700, 128, 1.0), (300, 512, 1.0)])
+def test_sparse_mla_same_index_set(L, k, std):
+    inp = dsa_synth.make_prefill(L, topk=k, seed=L, device=DEV, latent_std=std)
+    _check_mla(inp, _random_idx(inp, k, seed=L))
+
+
+def test_sparse_mla_rows_without_valid_keys():
+    inp = dsa_synth.make_prefill(64, topk=16, seed=11, device=DEV)
+    idx = _random_idx(inp, 16, seed=11)
+    idx[5] = -1
+    idx[9] = 60       # all future for row 9 (pos 9) -> masked
+    out, lse = _check_mla(inp, idx)
+    assert torch.all(out[5] == 0) and torch.all(torch.isneginf(lse[5]))
+    assert torch.all(out[9] == 0) and torch.all(torch.isneginf(lse[9]))
+
+
+def test_sparse_mla_decode_ragged():
+    inp = dsa_synth.make_decode(6, 300, 3000, topk=256, seed=12, device=DEV)
+    _check_mla(inp, _random_idx(inp, 256, seed=12))
+
+
+# ---------------------------------------------------------------- fused forward
+
+def _run_forward(inp, chunk=0, want_idx=True):
+    T = inp["total_q"]
+    p = dsa.problem_from_inputs(inp)
+    ws = torch.empty(dsa.dsa_forward_workspace_size(p, chunk), dtype=torch.uint8, device=DEV)
+    out = torch.empty((T, 128, 512), dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty((T, 128), dtype=torch.float32, device=DEV)
+    idx = torch.empty((T, inp["topk"]), dtype=torch.int32, device=DEV) if want_idx else None
+    fp8 = "q_idx8" in inp
+    dsa.dsa_forward(p, inp["q_idx8"] if fp8 else inp["q_idx"], inp["k_idx8"] if fp8 else inp["k_idx"], inp["w"],
+                    inp["q"], inp["kv"], out, lse, ws, chunk_q=chunk, idx_out=idx,
+                    q_scale=inp.get("q_scale"), k_scale=inp.get("k_scale"))
+    return idx, out, lse
+
+
+def _check_forward_rows(inp, rows, chunk=0):
+    idx, out, lse = _run_forward(inp, chunk)
+    k = inp["topk"]
+    pos = _positions(inp, rows)
+    ref_sc = _oracle_scores(inp, rows)
+    bound = _bound_rows(inp, rows)
+    gidx = idx.cpu().numpy()[rows]
+    recall, wrong = recall_excluding_near_ties(gidx, ref_sc, bound, pos, k)
+    assert recall >= RECALL_MIN and wrong == 0, (recall, wrong)
+    rt = torch.from_numpy(rows)
+    o_ref, lse_ref = oracle.sparse_mla(inp["q"].cpu()[rt], inp["kv"].cpu(), gidx, SCALE, rows=rows,
+                                       cu_q=inp["cu_q"].cpu().numpy(), cu_k=inp["cu_k"].cpu().numpy())
+    assert np.max(np.abs(out.cpu()[rt].double().numpy() - o_ref)) <= O_ATOL
+    assert np.max(np.abs(lse.cpu()[rt].double().numpy() - lse_ref)) <= LSE_ATOL
+    return idx, out, lse
+
+
+def test_forward_pr_reference_config_all_rows():
+    inp = dsa_synth.make_workload("pr_ref_256", seed=0, device=DEV)
+    _check_forward_rows(inp, np.arange(256))
+
+
+def test_forward_chunking_is_bit_identical():
+    inp = dsa_synth.make_prefill(1000, topk=128, seed=21, device=DEV)
+    a = _run_forward(inp, chunk=0)
+    b = _run_forward(inp, chunk=96)
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+    c = _run_forward(inp, chunk=0, want_idx=False)
+    assert torch.equal(a[1], c[1]) and torch.equal(a[2], c[2])
+
+
+def test_forward_fp8_indexer_small():
+    inp = dsa_synth.make_prefill(1200, topk=256, seed=22, device=DEV, fp8_indexer=True)
+    _check_forward_rows(inp, sample_rows(1200, 256, n_rand=48, seed=22), chunk=512)
+
+
+def test_forward_decode_small_ragged():
+    inp = dsa_synth.make_decode(6, 500, 5000, topk=512, seed=23, device=DEV)
+    _check_forward_rows(inp, np.arange(6))
+
+
+# ------------------------------------------- full-size workloads, sampled rows
+
+def test_prefill_4k_full_size_sampled():
+    inp = dsa_synth.make_workload("prefill_4k", seed=0, device=DEV)
+    rows = sample_rows(4096, 2048, n_rand=24, seed=1, edge=8)
+    _check_forward_rows(inp, rows, chunk=4096)
+
+
+def test_prefill_32k_full_size_sampled_bench_config():
+    inp = dsa_synth.make_workload("prefill_32k", seed=0, device=DEV)
+    rows = sample_rows(32768, 2048, n_rand=12, seed=2, edge=4)
+    _check_forward_rows(inp, rows, chunk=dsa_synth.WORKLOADS["prefill_32k"].chunk)
+
+
+def test_decode_b64_full_size_sampled():
+    inp = dsa_synth.make_workload("decode_b64", seed=0, device=DEV)
+    _check_forward_rows(inp, np.array([0, 7, 31, 63]))
