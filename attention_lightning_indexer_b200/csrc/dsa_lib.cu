@@ -9,7 +9,6 @@
 
 #include "../../include/dsa.h"
 #include "dsa_common.cuh"
-#include "indexer.cuh"
 #include "indexer_tc.cuh"
 #include "sparse_mla.cuh"
 #include "topk.cuh"
@@ -91,13 +90,7 @@ dsa_status_t set_smem_attrs() {
     static bool done = false;
     if (done) return DSA_OK;
     cudaError_t e = cudaSuccess;
-    e = cudaFuncSetAttribute(dsa::indexer::indexer_cuda_core_kernel<false>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, dsa::indexer::CUDA_CORE_SMEM);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(dsa::indexer::indexer_cuda_core_kernel<true>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, dsa::indexer::CUDA_CORE_SMEM);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(dsa::mla::sparse_mla_cuda_core_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(dsa::mla::sparse_mla_cuda_core_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  dsa::mla::CUDA_CORE_SMEM);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(dsa::topk::topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
