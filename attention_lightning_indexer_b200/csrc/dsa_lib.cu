@@ -10,7 +10,7 @@
 #include "../../include/dsa.h"
 #include "dsa_common.cuh"
 #include "indexer_tc.cuh"
-#include "sparse_mla.cuh"
+#include "sparse_mla_tc.cuh"
 #include "topk.cuh"
 
 namespace {
@@ -65,7 +65,8 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-// 2-D row-major tensor map with a 128-byte-swizzled box of `box_rows` rows x 128 bytes.
+// 2-D row-major tensor map (`cols` x `rows`, 1- or 2-byte elements) whose box is
+// `box_rows` rows x 128 bytes, loaded with the 128-byte swizzle.
 bool make_tmap_rows(CUtensorMap *m, const void *base, bool fp8, uint64_t cols, uint64_t rows, uint32_t box_rows) {
     auto enc = tensor_map_encoder();
     if (enc == nullptr) return false;
@@ -90,11 +91,8 @@ dsa_status_t set_smem_attrs() {
     static bool done = false;
     if (done) return DSA_OK;
     cudaError_t e = cudaSuccess;
-    e = cudaFuncSetAttribute(dsa::mla::sparse_mla_cuda_core_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 dsa::mla::CUDA_CORE_SMEM);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(dsa::topk::topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 200 * 1024);
+    e = cudaFuncSetAttribute(dsa::mla::sparse_mla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             dsa::mla::TcCfg::SMEM);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(dsa::indexer::indexer_tc_kernel<8, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  dsa::indexer::TcCfg<8, false>::SMEM);
@@ -156,12 +154,7 @@ dsa_status_t topk_launch(const dsa_problem_t *p, const float *scores, int64_t ld
                          int32_t *idx, cudaStream_t stream) {
     if (row_count == 0) return DSA_OK;
     Problem P = to_dev(p);
-    int row_cap = 0;
-    const int max_row_cap = (200 * 1024 - dsa::topk::FIXED_SMEM) / 4;
-    if (p->max_len_k <= max_row_cap) row_cap = p->max_len_k;
-    size_t smem = dsa::topk::FIXED_SMEM + (size_t)row_cap * 4;
-    dsa::topk::topk_rows_kernel<<<row_count, dsa::topk::THREADS, smem, stream>>>(P, scores, ld, row_begin, idx,
-                                                                                  row_cap);
+    dsa::topk::topk_rows_kernel<<<row_count, dsa::topk::THREADS, 0, stream>>>(P, scores, ld, row_begin, idx);
     return launch_status();
 }
 
@@ -169,10 +162,13 @@ dsa_status_t mla_launch(const dsa_problem_t *p, const void *q, const void *kv, c
                         float *lse, cudaStream_t stream) {
     if (p->total_q == 0) return DSA_OK;
     Problem P = to_dev(p);
-    dim3 grid(p->total_q, dsa::mla::H / dsa::mla::CC_HG);
-    dsa::mla::sparse_mla_cuda_core_kernel<<<grid, 256, dsa::mla::CUDA_CORE_SMEM, stream>>>(
-        P, reinterpret_cast<const __nv_bfloat16 *>(q), reinterpret_cast<const __nv_bfloat16 *>(kv), idx,
-        reinterpret_cast<__nv_bfloat16 *>(out), lse);
+    CUtensorMap tq, tkv;
+    // q: [T*128 rows, 576] read as 128-row boxes; kv: [S, 576] read 4 gathered rows at a time
+    if (!make_tmap_rows(&tq, q, false, 576, (uint64_t)p->total_q * 128, 128)) return DSA_ERR_CUDA;
+    if (!make_tmap_rows(&tkv, kv, false, 576, (uint64_t)(p->total_k > 0 ? p->total_k : 1), 1)) return DSA_ERR_CUDA;
+    dsa::mla::sparse_mla_tc_kernel<<<2u * (unsigned)p->total_q, dsa::mla::TcCfg::THREADS, dsa::mla::TcCfg::SMEM,
+                                     stream>>>(tq, tkv, P, reinterpret_cast<const __nv_bfloat16 *>(q), idx,
+                                               reinterpret_cast<__nv_bfloat16 *>(out), lse);
     return launch_status();
 }
 

@@ -4,19 +4,23 @@
 // top-k index scores of each query; "Model techniques map -- DeepSeek-V3.2",
 // Indexer-selected sparse attention: k_eff = min(index_topk, #candidates), int32 out.
 //
-// Design (one CTA per query row, HBM-bound):
-//   * scores are mapped to order-preserving 32-bit keys (-0.0 folded onto +0.0), so
-//     comparing keys as unsigned integers compares the floats as values;
-//   * an 11/11/10-bit MSB-first radix select finds the exact k-th largest key `thr`
-//     and how many keys equal to `thr` are taken (the smallest indices win ties);
-//   * after the first digit only the keys that share the selected digit are kept as
-//     candidates (compacted in shared memory), so the later digits touch a few % of
-//     the row;
-//   * a final ordered pass writes keys > thr and the first `need_eq` keys == thr
-//     using warp ballots, so the output is deterministic (ascending index within each
-//     class) and independent of the launch shape.
-// The row is staged once in shared memory when it fits; longer rows are re-read from
-// global memory (L2) on each pass.
+// Design (one 256-thread CTA per query row; HBM-bound, several CTAs per SM):
+//   * scores map to order-preserving 32-bit keys (-0.0 folded onto +0.0), so comparing
+//     keys as unsigned integers compares the floats as values;
+//   * pass 1 (the only HBM read of the row): histogram of the top 11 key bits, 4 float4
+//     loads in flight per thread, warp-aggregated shared atomics (match.any);
+//   * the bin holding the k-th largest key is found; pass 2 (an L2 re-read) counts, per
+//     warp range, the keys in higher bins (certainly selected) and compacts the indices
+//     of the keys in that bin (the candidates) into shared memory;
+//   * digits 2 (bits 20..10) and 3 (bits 9..0) are resolved on the candidates only,
+//     giving the exact k-th largest key `thr` and the number `need_eq` of keys equal to
+//     it that are taken (smallest indices first);
+//   * pass 3 (an L2 re-read) writes, in ascending index order, every key > thr followed
+//     by the first need_eq keys == thr, from per-warp offsets and in-warp prefix sums:
+//     the output is deterministic and independent of the launch shape.
+// When the candidates overflow the shared buffer (e.g. a row of identical scores) the
+// later digits and the per-warp counts are taken from the row itself instead (slower,
+// same result).
 #pragma once
 
 #include "dsa_common.cuh"
@@ -24,14 +28,11 @@
 namespace dsa {
 namespace topk {
 
-constexpr int THREADS = 512;
+constexpr int THREADS = 256;
 constexpr int WARPS = THREADS / 32;
 constexpr int BINS = 2048;        // 11-bit digits
-constexpr int CAND_CAP = 8192;    // candidates kept after the first digit
+constexpr int CAND_CAP = 6144;    // candidates kept after the first digit
 constexpr unsigned FULL = 0xffffffffu;
-
-// Shared-memory bytes besides the staged row.
-constexpr int FIXED_SMEM = BINS * 4 + CAND_CAP * 4 + 64 * 4;
 
 __device__ __forceinline__ uint32_t order_key(float f) {
     uint32_t u = __float_as_uint(f);
@@ -40,33 +41,39 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 }
 
 struct Smem {
-    uint32_t *hist;      // [BINS]
-    int *cand;           // [CAND_CAP]
-    int *scal;           // small scalars
-    uint32_t *row;       // [row_cap] staged keys (may be unused)
+    uint32_t hist[BINS];
+    int cand[CAND_CAP];
+    int warp_gt0[WARPS];   // keys whose first digit is above the threshold bin, per warp range
+    int warp_gt[WARPS];    // candidates above thr, per warp range
+    int warp_eq[WARPS];    // candidates equal to thr, per warp range
+    int scal[8];           // [0] bin  [1] above  [2] ncand
 };
 
-// Finds the digit bin holding the `remaining`-th largest key of the histogram.
-// Writes bin and the count of keys in strictly higher bins to scal[0], scal[1].
+// Warp-aggregated histogram increment; d == BINS means "no key" (lane still participates).
+__device__ __forceinline__ void hist_add(uint32_t *hist, uint32_t d, int lane) {
+    const unsigned peers = __match_any_sync(FULL, d);
+    if (d < (uint32_t)BINS && lane == __ffs(peers) - 1) atomicAdd(&hist[d], (uint32_t)__popc(peers));
+}
+
+// Warp 0: the bin holding the `remaining`-th largest key; writes bin and the count of
+// keys in strictly higher bins to scal[0], scal[1].
 __device__ __forceinline__ void select_bin(const uint32_t *hist, int nbins, int remaining, int *scal) {
     const int lane = threadIdx.x & 31;
-    const int per = nbins / 32;                // bins per lane (64 or 32)
-    // lane 0 owns the highest bins
-    const int top = nbins - 1 - lane * per;
+    const int per = nbins / 32;
+    const int top = nbins - 1 - lane * per;   // lane 0 owns the highest bins
     uint32_t mine = 0;
     for (int i = 0; i < per; ++i) mine += hist[top - i];
     uint32_t incl = mine;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-        uint32_t v = __shfl_up_sync(FULL, incl, off);
+        const uint32_t v = __shfl_up_sync(FULL, incl, off);
         if (lane >= off) incl += v;
     }
-    uint32_t above = incl - mine;              // keys in bins of lanes before mine
-    bool here = (above < (uint32_t)remaining) && ((uint32_t)remaining <= incl);
-    if (here) {
+    const uint32_t above = incl - mine;
+    if (above < (uint32_t)remaining && (uint32_t)remaining <= incl) {
         uint32_t acc = above;
         for (int i = 0; i < per; ++i) {
-            uint32_t h = hist[top - i];
+            const uint32_t h = hist[top - i];
             if (acc + h >= (uint32_t)remaining) {
                 scal[0] = top - i;
                 scal[1] = (int)acc;
@@ -77,48 +84,128 @@ __device__ __forceinline__ void select_bin(const uint32_t *hist, int nbins, int 
     }
 }
 
-template <bool STAGED>
-__device__ __forceinline__ uint32_t key_at(const Smem &sm, const float *src, int i) {
-    if (STAGED) return sm.row[i];
-    return order_key(__ldg(src + i));
+__device__ __forceinline__ int warp_sum(int v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(FULL, v, off);
+    return v;
 }
 
-template <bool STAGED>
-__device__ void select_row(const Smem &sm, const float *src, int n, int K, int32_t *out) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    int *scal = sm.scal;
-    // scal: [0] bin, [1] above, [2] ncand, [3..3+WARPS) gt counts, [3+WARPS..3+2W) eq counts
-
-    // ---- digit 0: bits 31..21 over the whole row
-    for (int i = tid; i < BINS; i += THREADS) sm.hist[i] = 0;
-    if (tid == 0) scal[2] = 0;
-    __syncthreads();
-    const int n_pad = (n + 31) & ~31;
-    for (int i = tid; i < n_pad; i += THREADS) {
-        uint32_t d = i < n ? (key_at<STAGED>(sm, src, i) >> 21) : (uint32_t)BINS;
-        unsigned peers = __match_any_sync(FULL, d);
-        if (d < (uint32_t)BINS && lane == __ffs(peers) - 1) atomicAdd(&sm.hist[d], (uint32_t)__popc(peers));
+__device__ __forceinline__ int warp_excl_scan(int v, int lane, int &total) {
+    int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int x = __shfl_up_sync(FULL, incl, off);
+        if (lane >= off) incl += x;
     }
-    __syncthreads();
-    if (warp == 0) select_bin(sm.hist, BINS, K, scal);
-    __syncthreads();
-    int remaining = K - scal[1];
-    uint32_t prefix = (uint32_t)scal[0] << 21;
-    uint32_t mask = 0xFFE00000u;
-    __syncthreads();
+    total = __shfl_sync(FULL, incl, 31);
+    return incl - v;
+}
 
-    // ---- compact candidates that share digit 0
-    for (int i = tid; i < n; i += THREADS) {
-        if ((key_at<STAGED>(sm, src, i) & mask) == prefix) {
-            int slot = atomicAdd(&scal[2], 1);
-            if (slot < CAND_CAP) sm.cand[slot] = i;
+// The lane's 4 consecutive keys i0..i0+3 of the warp range [.., we); invalid ones get 0.
+__device__ __forceinline__ int load4(const float *src, int i0, int we, uint32_t (&k)[4]) {
+    if (i0 + 3 < we) {
+        const float4 v = __ldg(reinterpret_cast<const float4 *>(src + i0));
+        k[0] = order_key(v.x);
+        k[1] = order_key(v.y);
+        k[2] = order_key(v.z);
+        k[3] = order_key(v.w);
+        return 4;
+    }
+    int nv = 0;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        k[c] = 0u;
+        if (i0 + c < we) {
+            k[c] = order_key(__ldg(src + i0 + c));
+            ++nv;
         }
     }
+    return nv;
+}
+
+__global__ void __launch_bounds__(THREADS) topk_rows_kernel(Problem P, const float *__restrict__ scores, int64_t ld,
+                                                            int row_begin, int32_t *__restrict__ idx) {
+    __shared__ Smem sm;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int r = blockIdx.x;
+    const int K = P.topk;
+    int32_t *out = idx + (int64_t)r * K;
+    const RowInfo ri = row_info(P, row_begin + r);
+    const int n = visible_keys(ri);
+    if (n <= K) {   // select every visible key
+        for (int j = tid; j < K; j += THREADS) out[j] = j < n ? j : -1;
+        return;
+    }
+    const float *src = scores + (int64_t)r * ld;
+
+    for (int i = tid; i < BINS; i += THREADS) sm.hist[i] = 0;
+    if (tid < WARPS) {
+        sm.warp_gt[tid] = 0;
+        sm.warp_eq[tid] = 0;
+    }
+    if (tid == 0) sm.scal[2] = 0;
     __syncthreads();
-    const int ncand = scal[2];
+
+    // ---- pass 1: histogram of bits 31..21
+    {
+        const float4 *s4 = reinterpret_cast<const float4 *>(src);
+        const int n4 = n >> 2;
+        for (int base = 0; base < n4; base += THREADS * 4) {
+            float4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = base + u * THREADS + tid;
+                v[u] = i < n4 ? __ldg(s4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const bool ok = base + u * THREADS + tid < n4;
+                hist_add(sm.hist, ok ? order_key(v[u].x) >> 21 : (uint32_t)BINS, lane);
+                hist_add(sm.hist, ok ? order_key(v[u].y) >> 21 : (uint32_t)BINS, lane);
+                hist_add(sm.hist, ok ? order_key(v[u].z) >> 21 : (uint32_t)BINS, lane);
+                hist_add(sm.hist, ok ? order_key(v[u].w) >> 21 : (uint32_t)BINS, lane);
+            }
+        }
+        const int tail = n - (n4 << 2);
+        if (tid < tail) atomicAdd(&sm.hist[order_key(__ldg(src + (n4 << 2) + tid)) >> 21], 1u);
+    }
+    __syncthreads();
+    if (warp == 0) select_bin(sm.hist, BINS, K, sm.scal);
+    __syncthreads();
+    const uint32_t b0 = (uint32_t)sm.scal[0];
+    int remaining = K - sm.scal[1];
+
+    // ---- pass 2: per-warp count of keys above bin b0, compaction of the keys in b0
+    const int R = ((n + WARPS * 128 - 1) / (WARPS * 128)) * 128;   // warp range, multiple of 128
+    const int wb = warp * R;
+    const int we = min(n, wb + R);
+    {
+        int g0 = 0;
+        for (int base = wb; base < we; base += 128) {
+            const int i0 = base + lane * 4;
+            uint32_t k[4];
+            load4(src, i0, we, k);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                if (i0 + c >= we) continue;
+                const uint32_t d = k[c] >> 21;
+                if (d > b0) {
+                    ++g0;
+                } else if (d == b0) {
+                    const int slot = atomicAdd(&sm.scal[2], 1);
+                    if (slot < CAND_CAP) sm.cand[slot] = i0 + c;
+                }
+            }
+        }
+        g0 = warp_sum(g0);
+        if (lane == 0) sm.warp_gt0[warp] = g0;
+    }
+    __syncthreads();
+    const int ncand = sm.scal[2];
     const bool use_cand = ncand <= CAND_CAP;
 
-    // ---- digits 1 (bits 20..10) and 2 (bits 9..0)
+    // ---- digits 2 and 3 on the candidates (or on the whole row after an overflow)
+    uint32_t prefix = b0 << 21, mask = 0xFFE00000u;
     for (int pass = 1; pass <= 2; ++pass) {
         const int shift = pass == 1 ? 10 : 0;
         const int nb = pass == 1 ? 2048 : 1024;
@@ -129,18 +216,16 @@ __device__ void select_row(const Smem &sm, const float *src, int n, int K, int32
         for (int j = tid; j < m_pad; j += THREADS) {
             uint32_t d = (uint32_t)BINS;
             if (j < m) {
-                int i = use_cand ? sm.cand[j] : j;
-                uint32_t key = key_at<STAGED>(sm, src, i);
+                const uint32_t key = order_key(__ldg(src + (use_cand ? sm.cand[j] : j)));
                 if ((key & mask) == prefix) d = (key >> shift) & (uint32_t)(nb - 1);
             }
-            unsigned peers = __match_any_sync(FULL, d);
-            if (d < (uint32_t)BINS && lane == __ffs(peers) - 1) atomicAdd(&sm.hist[d], (uint32_t)__popc(peers));
+            hist_add(sm.hist, d, lane);
         }
         __syncthreads();
-        if (warp == 0) select_bin(sm.hist, nb, remaining, scal);
+        if (warp == 0) select_bin(sm.hist, nb, remaining, sm.scal);
         __syncthreads();
-        remaining -= scal[1];
-        prefix |= (uint32_t)scal[0] << shift;
+        remaining -= sm.scal[1];
+        prefix |= (uint32_t)sm.scal[0] << shift;
         mask |= (uint32_t)(nb - 1) << shift;
         __syncthreads();
     }
@@ -148,85 +233,69 @@ __device__ void select_row(const Smem &sm, const float *src, int n, int K, int32
     const int need_eq = remaining;       // >= 1
     const int count_gt = K - need_eq;
 
-    // ---- ordered output: warp w owns the index range [w*R, min(n, (w+1)*R))
-    const int R = ((n + WARPS * 32 - 1) / (WARPS * 32)) * 32;
-    const int wb = warp * R;
-    const int we = min(n, wb + R);
-    int gt = 0, eq = 0;
-    for (int base = wb; base < we; base += 32) {
-        int i = base + lane;
-        uint32_t key = i < we ? key_at<STAGED>(sm, src, i) : 0u;
-        gt += __popc(__ballot_sync(FULL, i < we && key > thr));
-        eq += __popc(__ballot_sync(FULL, i < we && key == thr));
-    }
-    if (lane == 0) {
-        scal[3 + warp] = gt;
-        scal[3 + WARPS + warp] = eq;
+    // ---- per-warp counts of the keys > thr and == thr inside bin b0
+    if (use_cand) {
+        for (int j = tid; j < ncand; j += THREADS) {
+            const int i = sm.cand[j];
+            const uint32_t key = order_key(__ldg(src + i));
+            if (key > thr) atomicAdd(&sm.warp_gt[i / R], 1);
+            else if (key == thr) atomicAdd(&sm.warp_eq[i / R], 1);
+        }
+    } else {
+        int cg = 0, ce = 0;
+        for (int base = wb; base < we; base += 128) {
+            const int i0 = base + lane * 4;
+            uint32_t k[4];
+            load4(src, i0, we, k);
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                if (i0 + c >= we || (k[c] >> 21) != b0) continue;
+                cg += k[c] > thr;
+                ce += k[c] == thr;
+            }
+        }
+        cg = warp_sum(cg);
+        ce = warp_sum(ce);
+        if (lane == 0) {
+            sm.warp_gt[warp] = cg;
+            sm.warp_eq[warp] = ce;
+        }
     }
     __syncthreads();
+
+    // ---- pass 3: ordered output
     int gt_off = 0, eq_off = 0;
     for (int w2 = 0; w2 < warp; ++w2) {
-        gt_off += scal[3 + w2];
-        eq_off += scal[3 + WARPS + w2];
+        gt_off += sm.warp_gt0[w2] + sm.warp_gt[w2];
+        eq_off += sm.warp_eq[w2];
     }
-    const unsigned lt_mask = (1u << lane) - 1u;
-    for (int base = wb; base < we; base += 32) {
-        int i = base + lane;
-        uint32_t key = i < we ? key_at<STAGED>(sm, src, i) : 0u;
-        unsigned bg = __ballot_sync(FULL, i < we && key > thr);
-        unsigned be = __ballot_sync(FULL, i < we && key == thr);
-        if (i < we && key > thr) {
-            int slot = gt_off + __popc(bg & lt_mask);
-            if (slot < count_gt) out[slot] = i;      // always true when the counts agree
+    for (int base = wb; base < we; base += 128) {
+        const int i0 = base + lane * 4;
+        uint32_t k[4];
+        load4(src, i0, we, k);
+        int cg = 0, ce = 0;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const bool v = i0 + c < we;
+            cg += v && k[c] > thr;
+            ce += v && k[c] == thr;
         }
-        if (i < we && key == thr) {
-            int rank = eq_off + __popc(be & lt_mask);
-            if (rank < need_eq && count_gt + rank < K) out[count_gt + rank] = i;
+        int tg, te;
+        int og = warp_excl_scan(cg, lane, tg) + gt_off;
+        int oe = warp_excl_scan(ce, lane, te) + eq_off;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            if (i0 + c >= we) continue;
+            if (k[c] > thr) {
+                if (og < count_gt) out[og] = i0 + c;
+                ++og;
+            } else if (k[c] == thr) {
+                if (oe < need_eq && count_gt + oe < K) out[count_gt + oe] = i0 + c;
+                ++oe;
+            }
         }
-        gt_off += __popc(bg);
-        eq_off += __popc(be);
-    }
-}
-
-// grid = row_count CTAs of THREADS threads; dynamic smem = FIXED_SMEM + row_cap*4.
-__global__ void __launch_bounds__(THREADS) topk_rows_kernel(Problem P, const float *__restrict__ scores,
-                                                            int64_t ld, int row_begin, int32_t *__restrict__ idx,
-                                                            int row_cap) {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    Smem sm;
-    sm.hist = reinterpret_cast<uint32_t *>(smem_raw);
-    sm.cand = reinterpret_cast<int *>(smem_raw + BINS * 4);
-    sm.scal = reinterpret_cast<int *>(smem_raw + BINS * 4 + CAND_CAP * 4);
-    sm.row = reinterpret_cast<uint32_t *>(smem_raw + FIXED_SMEM);
-
-    const int r = blockIdx.x;
-    const int t = row_begin + r;
-    const int K = P.topk;
-    int32_t *out = idx + (int64_t)r * K;
-    const RowInfo ri = row_info(P, t);
-    const int n = visible_keys(ri);
-    if (n <= K) {   // select all visible keys
-        for (int j = threadIdx.x; j < K; j += THREADS) out[j] = j < n ? j : -1;
-        return;
-    }
-    const float *src = scores + (int64_t)r * ld;
-    if (n <= row_cap) {
-        const int n4 = n >> 2;
-        const float4 *s4 = reinterpret_cast<const float4 *>(src);
-        for (int i = threadIdx.x; i < n4; i += THREADS) {
-            float4 v = __ldg(s4 + i);
-            uint4 k;
-            k.x = order_key(v.x);
-            k.y = order_key(v.y);
-            k.z = order_key(v.z);
-            k.w = order_key(v.w);
-            reinterpret_cast<uint4 *>(sm.row)[i] = k;
-        }
-        for (int i = (n4 << 2) + threadIdx.x; i < n; i += THREADS) sm.row[i] = order_key(__ldg(src + i));
-        __syncthreads();
-        select_row<true>(sm, src, n, K, out);
-    } else {
-        select_row<false>(sm, src, n, K, out);
+        gt_off += tg;
+        eq_off += te;
     }
 }
 

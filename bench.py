@@ -458,6 +458,68 @@ def run_reference(args, ws, rank, local):
     print(json.dumps(res), flush=True)
 
 
+def run_kernel(args, local):
+    """One kernel entry point on a bounded slice of the workload, for profilers: the
+    indexer or top-k on the last (heaviest) chunk of query rows, or the sparse MLA on
+    `--rows` query rows (the last ones).  Prints one JSON line with the mean device time."""
+    import attention_lightning_indexer_b200 as dsa
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wl = dsa_synth.WORKLOADS[args.workload]
+    need_latent = args.kernel == "sparse_mla"
+    inp = dsa_synth.make_workload(args.workload, seed=args.seed, device=dev, with_latent=need_latent)
+    p = dsa.problem_from_inputs(inp)
+    fa = _forward_args(inp)
+    T = inp["total_q"]
+    rows = min(T, args.rows or (args.chunk or wl.chunk or T))
+    r0 = T - rows
+    ld = dsa.scores_ld(inp["max_len_k"])
+    stream = torch.cuda.current_stream(dev)
+    if args.kernel in ("indexer", "topk"):
+        scores = torch.empty((rows, ld), dtype=torch.float32, device=dev)
+        idx = torch.empty((rows, inp["topk"]), dtype=torch.int32, device=dev)
+        dsa.dsa_indexer_scores(p, fa["q_idx"], fa["k_idx"], inp["w"], scores, row_begin=r0, row_count=rows,
+                               q_scale=fa["q_scale"], k_scale=fa["k_scale"], stream=stream)
+        if args.kernel == "indexer":
+            fn = lambda: dsa.dsa_indexer_scores(p, fa["q_idx"], fa["k_idx"], inp["w"], scores, row_begin=r0,
+                                                row_count=rows, q_scale=fa["q_scale"], k_scale=fa["k_scale"],
+                                                stream=stream)
+        else:
+            fn = lambda: dsa.dsa_topk(p, scores, idx, row_begin=r0, row_count=rows, stream=stream)
+    else:
+        # index set: the GPU top-k of the GPU scores, chunk by chunk, for the last `rows` rows
+        idx = torch.empty((T, inp["topk"]), dtype=torch.int32, device=dev)
+        ch = args.chunk or wl.chunk or T
+        scores = torch.empty((min(ch, rows), ld), dtype=torch.float32, device=dev)
+        for c0 in range(r0, T, ch):
+            rc = min(ch, T - c0)
+            dsa.dsa_indexer_scores(p, fa["q_idx"], fa["k_idx"], inp["w"], scores, row_begin=c0, row_count=rc,
+                                   q_scale=fa["q_scale"], k_scale=fa["k_scale"], stream=stream)
+            dsa.dsa_topk(p, scores, idx[c0:c0 + rc], row_begin=c0, row_count=rc, stream=stream)
+        del scores
+        sub = dsa.make_problem(1, rows, inp["total_k"], rows, inp["max_len_k"], inp["topk"]) if p.cu_q is None else p
+        q = inp["q"][r0:]
+        out = torch.empty((rows, 128, 512), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((rows, 128), dtype=torch.float32, device=dev)
+        ix = idx[r0:]
+        fn = lambda: dsa.dsa_sparse_mla_fwd(sub, q, inp["kv"], ix, out, lse, stream=stream)
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize(dev)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    dsa.dsa_check_device_errors()
+    ms = a.elapsed_time(b) / args.steps
+    print(json.dumps({"kernel": args.kernel, "workload": args.workload, "rows": rows, "row_begin": r0,
+                      "ms_per_launch": ms}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -471,10 +533,16 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-breakdown", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel", choices=("indexer", "topk", "sparse_mla"), default=None,
+                    help="time one kernel on a bounded slice (for profilers) instead of the full step")
+    ap.add_argument("--rows", type=int, default=0, help="query rows for --kernel (default: one chunk)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     ws, rank, local = _dist()
+    if args.kernel is not None:
+        run_kernel(args, local)
+        return
     if args.impl == "reference":
         run_reference(args, ws, rank, local)
         return

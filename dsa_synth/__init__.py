@@ -90,8 +90,12 @@ def quantize_e4m3_per_token(x: torch.Tensor):
 
 
 def make_prefill(L: int, topk: int = 2048, seed: int = 0, device="cpu", structured_keys: bool = True,
-                 latent_std: float = 1.0, fp8_indexer: bool = False, T: Optional[int] = None):
-    """One sequence of L tokens.  T (default L) queries are the last T tokens."""
+                 latent_std: float = 1.0, fp8_indexer: bool = False, T: Optional[int] = None,
+                 with_latent: bool = True):
+    """One sequence of L tokens.  T (default L) queries are the last T tokens.
+
+    ``with_latent=False`` skips the last draws (q, kv) and leaves the indexer inputs
+    unchanged, for runs that only need the indexer side."""
     T = L if T is None else T
     g = _gen(seed, device)
     q_idx = _randn(g, (T, N_IDX_HEADS, IDX_DIM), device)
@@ -101,9 +105,11 @@ def make_prefill(L: int, topk: int = 2048, seed: int = 0, device="cpu", structur
         B = _randn(g, (16, IDX_DIM), device, std=0.25)
         k_idx += Z @ B
     w = _randn(g, (T, N_IDX_HEADS), device, std=0.125)
-    q = _randn(g, (T, N_HEADS, D_QK), device, std=latent_std).to(torch.bfloat16)
-    kv = _randn(g, (L, D_QK), device, std=latent_std).to(torch.bfloat16)
-    out = dict(w=w.contiguous(), q=q.contiguous(), kv=kv.contiguous(), topk=topk,
+    out = {}
+    if with_latent:
+        out["q"] = _randn(g, (T, N_HEADS, D_QK), device, std=latent_std).to(torch.bfloat16).contiguous()
+        out["kv"] = _randn(g, (L, D_QK), device, std=latent_std).to(torch.bfloat16).contiguous()
+    out.update(w=w.contiguous(), topk=topk,
                cu_q=torch.tensor([0, T], dtype=torch.int32, device=device),
                cu_k=torch.tensor([0, L], dtype=torch.int32, device=device),
                total_q=T, total_k=L, max_len_q=T, max_len_k=L, batch=1)
@@ -142,7 +148,7 @@ def make_decode(batch: int, ctx_min: int, ctx_max: int, topk: int = 2048, seed: 
                 total_q=T, total_k=S, max_len_q=q_per_seq, max_len_k=int(lens_cpu.max()), batch=batch)
 
 
-def make_workload(name: str, seed: int = 0, device="cpu", **overrides):
+def make_workload(name: str, seed: int = 0, device="cpu", with_latent: bool = True, **overrides):
     wl = WORKLOADS[name]
     if wl.kind == "decode":
         return make_decode(wl.batch, overrides.get("ctx_min", wl.ctx_min), overrides.get("ctx_max", wl.ctx_max),
@@ -150,4 +156,4 @@ def make_workload(name: str, seed: int = 0, device="cpu", **overrides):
                            latent_std=wl.latent_std)
     return make_prefill(overrides.get("L", wl.seq_len), topk=wl.topk, seed=seed, device=device,
                         structured_keys=wl.structured_keys, latent_std=wl.latent_std,
-                        fp8_indexer=wl.fp8_indexer)
+                        fp8_indexer=wl.fp8_indexer, with_latent=with_latent)
