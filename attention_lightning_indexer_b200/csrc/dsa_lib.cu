@@ -162,12 +162,12 @@ dsa_status_t mla_launch(const dsa_problem_t *p, const void *q, const void *kv, c
                         float *lse, cudaStream_t stream) {
     if (p->total_q == 0) return DSA_OK;
     Problem P = to_dev(p);
-    CUtensorMap tq, tkv;
-    // q: [T*128 rows, 576] read as 128-row boxes; kv: [S, 576] read 4 gathered rows at a time
+    CUtensorMap tq;
+    // q: [T*128 rows, 576] read as 128-row boxes of 64 dims (the latent rows are gathered with cp.async)
     if (!make_tmap_rows(&tq, q, false, 576, (uint64_t)p->total_q * 128, 128)) return DSA_ERR_CUDA;
-    if (!make_tmap_rows(&tkv, kv, false, 576, (uint64_t)(p->total_k > 0 ? p->total_k : 1), 1)) return DSA_ERR_CUDA;
     dsa::mla::sparse_mla_tc_kernel<<<2u * (unsigned)p->total_q, dsa::mla::TcCfg::THREADS, dsa::mla::TcCfg::SMEM,
-                                     stream>>>(tq, tkv, P, reinterpret_cast<const __nv_bfloat16 *>(q), idx,
+                                     stream>>>(tq, P, reinterpret_cast<const __nv_bfloat16 *>(q),
+                                               reinterpret_cast<const __nv_bfloat16 *>(kv), idx,
                                                reinterpret_cast<__nv_bfloat16 *>(out), lse);
     return launch_status();
 }

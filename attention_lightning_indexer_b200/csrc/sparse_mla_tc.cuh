@@ -16,14 +16,16 @@
 // one slot per 64-dim atom of the current block's 128 gathered latent rows (144 KB);
 // slot a always holds atom a, so the 4 atoms of this CTA's value half are 4
 // consecutive slots and serve directly as the MN-major B operand of the PV product.
-// Rows are gathered with TMA tile::gather4 (4 rows x 128 bytes per instruction).
-// The selected indices are compacted on the fly (invalid slots -- -1, future or
-// out-of-range positions -- are skipped); the tail of the last block is padded with a
-// duplicate row and masked in the softmax.
+// Rows are gathered by three producer warps with 16-byte cp.async (each warp
+// instruction moves 4 rows x 128 bytes of one atom; the 128-byte swizzle is applied in
+// the shared-memory address).  Small TMA gathers were issue-bound here; the LSU path
+// keeps the gather off the critical path.  The selected indices are compacted on the
+// fly (invalid slots -- -1, future or out-of-range positions -- are skipped); the tail
+// of the last block is padded with a duplicate row and masked in the softmax.
 //
 // Warp roles (12 warps): 0 index compaction + gathers + q TMA, 1 MMA issuer, 2 TMEM
-// allocator, 3 idle, 4-11 softmax/epilogue: warp w owns TMEM lane quarter w % 4 (32
-// heads) and key/column half c = (w - 4) / 4.
+// allocator then gathers, 3 gathers, 4-11 softmax/epilogue: warp w owns TMEM lane
+// quarter w % 4 (32 heads) and key/column half c = (w - 4) / 4.
 #pragma once
 
 #include "dsa_common.cuh"
@@ -40,8 +42,8 @@ struct TcCfg {
     static constexpr int OFF_QHI = 0;
     static constexpr int OFF_KV = QHI_ATOMS * ATOM_BYTES;            // 81920
     static constexpr int OFF_RED = OFF_KV + NATOM * ATOM_BYTES;      // 229376
-    static constexpr int OFF_STAGE = OFF_RED + 2 * 2 * 128 * 4;      // row-max / sum exchange
-    static constexpr int STAGE_CAP = 160;
+    static constexpr int OFF_STAGE = OFF_RED + 2 * 128 * 4;          // row-max / sum exchange
+    static constexpr int STAGE_CAP = 256;                            // compacted indices
     static constexpr int OFF_BAR = OFF_STAGE + STAGE_CAP * 4;
     static constexpr int NBARS = 2 * NATOM + 5;
     static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
@@ -53,8 +55,8 @@ struct TcCfg {
 };
 
 __global__ void __launch_bounds__(384, 1)
-sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv, Problem P,
-                     const __nv_bfloat16 *__restrict__ q, const int32_t *__restrict__ idx,
+sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, Problem P, const __nv_bfloat16 *__restrict__ q,
+                     const __nv_bfloat16 *__restrict__ kv, const int32_t *__restrict__ idx,
                      __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
     using C = TcCfg;
     using namespace sm100;
@@ -73,7 +75,7 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     }
     const uint32_t qhi_s = sbase + C::OFF_QHI;
     const uint32_t kv_s = sbase + C::OFF_KV;
-    float *red = reinterpret_cast<float *>(smem + C::OFF_RED);      // [2 parity][2 halves][128]
+    float *red = reinterpret_cast<float *>(smem + C::OFF_RED);      // [2 halves][128]
     int *stage = reinterpret_cast<int *>(smem + C::OFF_STAGE);
     const uint32_t bar0 = sbase + C::OFF_BAR;
     auto kv_full = [&](int a) { return bar0 + 8u * a; };
@@ -88,7 +90,7 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     // ---- setup
     if (tid == 0) {
         for (int a = 0; a < C::NATOM; ++a) {
-            mbar_init(kv_full(a), 1);
+            mbar_init(kv_full(a), 32);   // one arrival per lane of the producing warp
             mbar_init(kv_empty(a), 1);
         }
         mbar_init(q_full, 1);
@@ -120,60 +122,124 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     // QK atom order: the 5 atoms outside this CTA's value half first, then its 4 value atoms
     auto atom_of = [&](int ai) { return ai < 5 ? (ai + 4 * (1 - v) + (ai >= 4 ? 4 * v : 0)) % 9 : ai - 5 + 4 * v; };
 
-    if (warp == 0) {
-        // ------------------------------------------------ compaction, gathers, q TMA
-        if (lane == 0 && nblocks > 0) {
+    if (warp == 0 || warp == 2 || warp == 3) {
+        // ------------------------------------------------ index compaction, gathers, q TMA
+        const int pw = warp == 0 ? 0 : warp - 1;            // producer 0, 1, 2
+        if (warp == 0 && lane == 0 && nblocks > 0) {
             prefetch_tmap(&tm_q);
-            prefetch_tmap(&tm_kv);
             mbar_expect_tx(q_full, C::QHI_ATOMS * C::ATOM_BYTES);
             for (int a = 0; a < C::QHI_ATOMS; ++a)
                 tma_load_2d(qhi_s + a * C::ATOM_BYTES, &tm_q, q_full, 256 + 64 * a, t * 128);
         }
         const int32_t *irow = idx + (int64_t)t * K;
-        int rd = 0, cnt = 0;   // idx entries consumed, entries queued in `stage`
-        bool ok_run = true;
-        for (int j = 0; j < nblocks && ok_run; ++j) {
-            while (cnt < C::BK && rd < K) {
-                const int i = rd + lane;
-                const int s = i < K ? __ldg(irow + i) : -1;
-                const bool ok = s >= 0 && s <= ri.pos && s < ri.len_k;
-                const unsigned bal = __ballot_sync(0xffffffffu, ok);
-                if (ok) stage[cnt + __popc(bal & ((1u << lane) - 1u))] = ri.kbase + s;
-                cnt += __popc(bal);
-                rd += 32;
-            }
-            __syncwarp();
-            const int nb = min(cnt, C::BK);
-            const int base_row = stage[0];
-            int r[4];
+        const bool vec4 = (K & 3) == 0;                      // rows of idx are 16-byte aligned
+        auto load_chunk = [&](int rd, int (&e)[4]) {         // entries rd + 4*lane .. +3
+            const int i = rd + 4 * lane;
+            if (vec4 && i + 3 < K) {
+                const int4 x = __ldg(reinterpret_cast<const int4 *>(irow + i));
+                e[0] = x.x; e[1] = x.y; e[2] = x.z; e[3] = x.w;
+            } else {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int k = lane * 4 + e;
-                r[e] = k < nb ? stage[k] : base_row;
+                for (int u = 0; u < 4; ++u) e[u] = i + u < K ? __ldg(irow + i + u) : -1;
             }
-            __syncwarp();
-            // keep the entries beyond this block for the next one
-            const int left = cnt - nb;
-            int carry = lane < left ? stage[C::BK + lane] : 0;
-            __syncwarp();
-            if (lane < left) stage[lane] = carry;
-            cnt = left;
-            __syncwarp();
-            for (int ai = 0; ai < C::NATOM; ++ai) {
-                const int a = atom_of(ai);
-                if (j > 0) {
-                    bool okw = true;
-                    if (lane == 0) okw = mbar_wait(kv_empty(a), (j - 1) & 1);
-                    okw = __shfl_sync(0xffffffffu, okw, 0);
-                    if (!okw || misc[2]) { misc[2] = 1; ok_run = false; break; }
+        };
+        int rd = 0, cnt = 0;
+        int nxt[4] = {-1, -1, -1, -1};
+        if (warp == 0 && nblocks > 0) load_chunk(0, nxt);
+        const char *kv_bytes = reinterpret_cast<const char *>(kv);
+        bool ok_run = true;
+        for (int j = 0; j < nblocks; ++j) {
+            // the three producer warps leave together when any of them gave up
+            if (named_bar_or(2, 96, !ok_run || misc[2] != 0)) { ok_run = false; break; }
+            if (warp == 0) {
+                while (cnt < C::BK && rd < K) {
+                    int cur[4] = {nxt[0], nxt[1], nxt[2], nxt[3]};
+                    rd += 128;
+                    if (rd < K) load_chunk(rd, nxt);            // prefetch the next chunk
+                    int vc = 0;
+                    bool okv[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        okv[u] = cur[u] >= 0 && cur[u] <= ri.pos && cur[u] < ri.len_k;
+                        vc += okv[u];
+                    }
+                    int incl = vc;                            // in-warp prefix of valid entries
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const int x = __shfl_up_sync(0xffffffffu, incl, o);
+                        if (lane >= o) incl += x;
+                    }
+                    const int tot = __shfl_sync(0xffffffffu, incl, 31);
+                    int off = cnt + incl - vc;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        if (okv[u]) stage[off++] = ri.kbase + cur[u];
+                    cnt += tot;
                 }
-                if (lane == 0) mbar_expect_tx(kv_full(a), C::ATOM_BYTES);
+                if (lane == 0) misc[3] = (uint32_t)min(cnt, C::BK);
+            }
+            named_bar(2, 96);                                 // stage holds this block's rows
+            const int nb = (int)misc[3];
+            const int base_row = stage[0];
+            int rows[32];
+#pragma unroll
+            for (int g = 0; g < 32; ++g) {
+                const int k = 4 * g + (lane >> 3);
+                rows[g] = k < nb ? stage[k] : base_row;
+            }
+            named_bar(2, 96);                                 // all rows read: stage may be rewritten
+            if (warp == 0) {                                  // keep the entries beyond this block
+                const int left = cnt - nb;                    // < 128
+                int keep[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) keep[u] = lane + 32 * u < left ? stage[C::BK + lane + 32 * u] : 0;
                 __syncwarp();
-                tma_gather4(kv_s + a * C::ATOM_BYTES + lane * 512, &tm_kv, kv_full(a), 64 * a, r[0], r[1], r[2], r[3]);
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    if (lane + 32 * u < left) stage[lane + 32 * u] = keep[u];
+                __syncwarp();
+                cnt = left;
+            }
+            // phase 1: atoms outside this CTA's value half (free once QK of the previous
+            // block consumed them); phase 2: the value atoms (free after the previous PV)
+            for (int phase = 0; phase < 2 && ok_run; ++phase) {
+                // this warp's atoms in QK order: ai = first + pw, first + pw + 3 (when in range)
+                const int first = phase == 0 ? 0 : 5, last = phase == 0 ? 5 : 9;
+                const int nmine = (first + pw < last) + (first + pw + 3 < last);
+                for (int q = 0; q < nmine; ++q) {
+                    const int a = atom_of(first + pw + 3 * q);
+                    if (j > 0) {
+                        bool okw = true;
+                        if (lane == 0) okw = mbar_wait(kv_empty(a), (j - 1) & 1);
+                        okw = __shfl_sync(0xffffffffu, okw, 0);
+                        if (!okw || misc[2]) { misc[2] = 1; ok_run = false; break; }
+                    }
+                    const uint32_t slot = kv_s + a * C::ATOM_BYTES;
+                    const int ch = lane & 7;
+#pragma unroll
+                    for (int g = 0; g < 32; ++g) {
+                        const int r = 4 * g + (lane >> 3);
+                        cp_async16(slot + r * 128 + ((ch ^ (r & 7)) << 4),
+                                   kv_bytes + (int64_t)rows[g] * 1152 + a * 128 + ch * 16);
+                    }
+                    cp_async_commit();
+                }
+                if (!ok_run) break;
+                // signal each atom once its copies have landed
+                if (nmine == 2) {
+                    cp_async_wait<1>();
+                    fence_proxy_async_smem();
+                    mbar_arrive(kv_full(atom_of(first + pw)));
+                }
+                if (nmine >= 1) {
+                    cp_async_wait<0>();
+                    fence_proxy_async_smem();
+                    mbar_arrive(kv_full(atom_of(first + pw + 3 * (nmine - 1))));
+                }
             }
         }
         // drain: the MMA commits on the value atoms of the last block must land before exit
-        if (lane == 0 && ok_run && nblocks > 0)
+        if (warp == 0 && lane == 0 && ok_run && nblocks > 0)
             for (int ai = 5; ai < C::NATOM; ++ai)
                 if (!mbar_wait(kv_empty(atom_of(ai)), (nblocks - 1) & 1)) { misc[2] = 1; break; }
     } else if (warp == 1 && lane == 0 && nblocks > 0) {
@@ -258,10 +324,11 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                 if (kbase_c + i < nb) mx = fmaxf(mx, __uint_as_float(s0[i]));
                 if (kbase_c + 32 + i < nb) mx = fmaxf(mx, __uint_as_float(s1[i]));
             }
-            float *rj = red + (j & 1) * 256;
-            rj[c * 128 + h] = mx;
+            // red is single-buffered: every thread passed this block's opening barrier
+            // only after reading the previous block's values
+            red[c * 128 + h] = mx;
             named_bar(1, 256);
-            const float m_blk = fmaxf(rj[h], rj[128 + h]) * sl2;
+            const float m_blk = fmaxf(red[h], red[128 + h]) * sl2;
             // Lazy rescale: a row moves its reference max only when the block max exceeds it
             // by more than TAU.  The TMEM load/store is warp-collective, so the whole warp
             // takes that path when any of its rows needs it (factor 1 for the others).
@@ -315,10 +382,11 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         } else {
             bool okw = mbar_wait(pv_done, (nblocks - 1) & 1);
             tc_fence_after();
-            float *rl = red + ((nblocks) & 1) * 256;   // the parity slot not used by the last block
-            rl[c * 128 + h] = l_part;
+            // the last block's max was read before its p_full arrival, which the last PV
+            // (hence pv_done) waited for: red may be reused
+            red[c * 128 + h] = l_part;
             named_bar(1, 256);
-            const float l = rl[h] + rl[128 + h];
+            const float l = red[h] + red[128 + h];
             const float inv = (l > 0.f && okw) ? 1.0f / l : 0.f;
 #pragma unroll
             for (int ch = 0; ch < 4; ++ch) {
