@@ -102,22 +102,35 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, Problem P, const 
         fence_barrier_init();
     }
     if (warp == 2) tmem_alloc(sbase + C::OFF_MISC, 512);
-    if (warp == 0) {   // number of valid selected indices of this row
+    if (warp == 0 || warp == 3) {   // number of valid selected indices of this row (2 warps)
         int cnt = 0;
         const int32_t *irow = idx + (int64_t)t * K;
-        for (int i0 = 0; i0 < K; i0 += 32) {
-            const int i = i0 + lane;
-            int s = i < K ? __ldg(irow + i) : -1;
-            const bool ok = s >= 0 && s <= ri.pos && s < ri.len_k;
-            cnt += __popc(__ballot_sync(0xffffffffu, ok));
+        const int half = (warp == 0) ? 0 : 1;
+        if ((K & 3) == 0) {
+            // 16-byte loads, all issued before use
+            const int n4 = K >> 2;
+#pragma unroll 4
+            for (int i4 = half * 32 + lane; i4 < n4; i4 += 64) {
+                const int4 x = __ldg(reinterpret_cast<const int4 *>(irow) + i4);
+                cnt += (x.x >= 0 && x.x <= ri.pos && x.x < ri.len_k) + (x.y >= 0 && x.y <= ri.pos && x.y < ri.len_k) +
+                       (x.z >= 0 && x.z <= ri.pos && x.z < ri.len_k) + (x.w >= 0 && x.w <= ri.pos && x.w < ri.len_k);
+            }
+        } else {
+            for (int i = half * 32 + lane; i < K; i += 64) {
+                const int s = __ldg(irow + i);
+                cnt += s >= 0 && s <= ri.pos && s < ri.len_k;
+            }
         }
-        if (lane == 0) misc[1] = (uint32_t)cnt;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+        if (lane == 0) red[half] = (float)cnt;   // exact for counts <= 2^24
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = misc[0];
-    const int nvalid = (int)misc[1];
+    const int nvalid = (int)red[0] + (int)red[1];
+    __syncthreads();   // red is reused by the softmax warps
     const int nblocks = (nvalid + C::BK - 1) / C::BK;
     // QK atom order: the 5 atoms outside this CTA's value half first, then its 4 value atoms
     auto atom_of = [&](int ai) { return ai < 5 ? (ai + 4 * (1 - v) + (ai >= 4 ? 4 * v : 0)) % 9 : ai - 5 + 4 * v; };
@@ -251,8 +264,9 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, Problem P, const 
         for (int j = 0; ok && j < nblocks; ++j) {
             for (int ai = 0; ai < C::NATOM; ++ai) {
                 const int a = atom_of(ai);
+                // shared-memory operands only: the mbarrier (after the producers' proxy fence)
+                // orders them; no tcgen05 fence is needed here
                 if (!mbar_wait(kv_full(a), j & 1)) { ok = false; break; }
-                tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk) {
                     const uint64_t bdesc = desc_sw128(kv_s + a * C::ATOM_BYTES + kk * 32);
@@ -353,16 +367,16 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, Problem P, const 
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const int k0 = kbase_c + 2 * i;
-                const float p0 = k0 < nb ? exp2f(fmaf(__uint_as_float(s0[2 * i]), sl2, -m_run)) : 0.f;
-                const float p1 = k0 + 1 < nb ? exp2f(fmaf(__uint_as_float(s0[2 * i + 1]), sl2, -m_run)) : 0.f;
+                const float p0 = k0 < nb ? ex2_approx(fmaf(__uint_as_float(s0[2 * i]), sl2, -m_run)) : 0.f;
+                const float p1 = k0 + 1 < nb ? ex2_approx(fmaf(__uint_as_float(s0[2 * i + 1]), sl2, -m_run)) : 0.f;
                 ls += p0 + p1;
                 pk[i] = pack_bf16x2(p0, p1);
             }
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const int k0 = kbase_c + 32 + 2 * i;
-                const float p0 = k0 < nb ? exp2f(fmaf(__uint_as_float(s1[2 * i]), sl2, -m_run)) : 0.f;
-                const float p1 = k0 + 1 < nb ? exp2f(fmaf(__uint_as_float(s1[2 * i + 1]), sl2, -m_run)) : 0.f;
+                const float p0 = k0 < nb ? ex2_approx(fmaf(__uint_as_float(s1[2 * i]), sl2, -m_run)) : 0.f;
+                const float p1 = k0 + 1 < nb ? ex2_approx(fmaf(__uint_as_float(s1[2 * i + 1]), sl2, -m_run)) : 0.f;
                 ls += p0 + p1;
                 pk[16 + i] = pack_bf16x2(p0, p1);
             }

@@ -123,6 +123,41 @@ __device__ __forceinline__ int load4(const float *src, int i0, int we, uint32_t 
     return nv;
 }
 
+// Pass 3: warp w writes, in ascending index order, the keys of its range [wb, we) that
+// are > thr (from slot gt_off on) and those == thr whose rank among equal keys is below
+// need_eq (from slot count_gt + eq_off on).
+__device__ __forceinline__ void ordered_output(const float *src, int wb, int we, int lane, uint32_t thr, int need_eq,
+                                               int count_gt, int K, int gt_off, int eq_off, int32_t *out) {
+    for (int base = wb; base < we; base += 128) {
+        const int i0 = base + lane * 4;
+        uint32_t k[4];
+        load4(src, i0, we, k);
+        int cg = 0, ce = 0;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const bool v = i0 + c < we;
+            cg += v && k[c] > thr;
+            ce += v && k[c] == thr;
+        }
+        int tg, te;
+        int og = warp_excl_scan(cg, lane, tg) + gt_off;
+        int oe = warp_excl_scan(ce, lane, te) + eq_off;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            if (i0 + c >= we) continue;
+            if (k[c] > thr) {
+                if (og < count_gt) out[og] = i0 + c;
+                ++og;
+            } else if (k[c] == thr) {
+                if (oe < need_eq && count_gt + oe < K) out[count_gt + oe] = i0 + c;
+                ++oe;
+            }
+        }
+        gt_off += tg;
+        eq_off += te;
+    }
+}
+
 __global__ void __launch_bounds__(THREADS) topk_rows_kernel(Problem P, const float *__restrict__ scores, int64_t ld,
                                                             int row_begin, int32_t *__restrict__ idx) {
     __shared__ Smem sm;
@@ -137,7 +172,134 @@ __global__ void __launch_bounds__(THREADS) topk_rows_kernel(Problem P, const flo
         return;
     }
     const float *src = scores + (int64_t)r * ld;
+    const float4 *s4 = reinterpret_cast<const float4 *>(src);
+    const int n4 = n >> 2;
+    const int R = ((n + WARPS * 128 - 1) / (WARPS * 128)) * 128;   // warp range, multiple of 128
+    const int wb = warp * R;
+    const int we = min(n, wb + R);
 
+    // ---- fast path: a sample fixes a lower digit bound; only keys at or above it are counted
+    for (int i = tid; i < BINS; i += THREADS) sm.hist[i] = 0;
+    if (tid < WARPS) {
+        sm.warp_gt[tid] = 0;
+        sm.warp_eq[tid] = 0;
+    }
+    if (tid < 8) sm.scal[tid] = 0;
+    __syncthreads();
+    int ns = 0;                                            // sampled keys (every 16th float4)
+    for (int m = tid; 16 * m < n4; m += THREADS) {
+        const float4 v = __ldg(s4 + 16 * m);
+        atomicAdd(&sm.hist[order_key(v.x) >> 21], 1u);
+        atomicAdd(&sm.hist[order_key(v.y) >> 21], 1u);
+        atomicAdd(&sm.hist[order_key(v.z) >> 21], 1u);
+        atomicAdd(&sm.hist[order_key(v.w) >> 21], 1u);
+    }
+    ns = 4 * ((n4 + 15) / 16);
+    __syncthreads();
+    if (warp == 0) {
+        // lowest bin b_lo whose sampled tail covers ~1.5 K keys of the full row (+ margin)
+        const uint32_t target = (uint32_t)((1.5 * K * (double)ns) / (double)n) + 16u;
+        select_bin(sm.hist, BINS, (int)min(target, (uint32_t)ns), sm.scal);   // scal[0] = b_lo
+    }
+    __syncthreads();
+    const uint32_t b_lo = (uint32_t)sm.scal[0];
+    __syncthreads();
+    for (int i = tid; i < BINS; i += THREADS) sm.hist[i] = 0;
+    if (tid == 0) sm.scal[2] = 0;
+    __syncthreads();
+    {
+        for (int base = 0; base < n4; base += THREADS * 4) {
+            float4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = base + u * THREADS + tid;
+                v[u] = i < n4 ? __ldg(s4 + i) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i4 = base + u * THREADS + tid;
+                const float e[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint32_t key = order_key(e[c]);
+                    const bool is = i4 < n4 && (key >> 21) >= b_lo;
+                    const unsigned bal = __ballot_sync(FULL, is);
+                    if (bal) {
+                        int slot0 = 0;
+                        if (lane == __ffs(bal) - 1) slot0 = atomicAdd(&sm.scal[2], __popc(bal));
+                        slot0 = __shfl_sync(FULL, slot0, __ffs(bal) - 1);
+                        if (is) {
+                            const int slot = slot0 + __popc(bal & ((1u << lane) - 1u));
+                            if (slot < CAND_CAP) sm.cand[slot] = 4 * i4 + c;
+                            atomicAdd(&sm.hist[key >> 21], 1u);
+                        }
+                    }
+                }
+            }
+        }
+        const int tail = n - (n4 << 2);
+        if (tid < tail) {
+            const int i = (n4 << 2) + tid;
+            const uint32_t key = order_key(__ldg(src + i));
+            if ((key >> 21) >= b_lo) {
+                const int slot = atomicAdd(&sm.scal[2], 1);
+                if (slot < CAND_CAP) sm.cand[slot] = i;
+                atomicAdd(&sm.hist[key >> 21], 1u);
+            }
+        }
+    }
+    __syncthreads();
+    const int ncand_fast = sm.scal[2];
+    const bool fast = ncand_fast >= K && ncand_fast <= CAND_CAP;
+    if (fast) {
+        // exact digits 1..3 on the candidates (bins below b_lo hold no count)
+        if (warp == 0) select_bin(sm.hist, BINS, K, sm.scal);
+        __syncthreads();
+        int remaining = K - sm.scal[1];
+        uint32_t prefix = (uint32_t)sm.scal[0] << 21, mask = 0xFFE00000u;
+        __syncthreads();
+        for (int pass = 1; pass <= 2; ++pass) {
+            const int shift = pass == 1 ? 10 : 0;
+            const int nb = pass == 1 ? 2048 : 1024;
+            for (int i = tid; i < nb; i += THREADS) sm.hist[i] = 0;
+            __syncthreads();
+            const int m_pad = (ncand_fast + 31) & ~31;
+            for (int j = tid; j < m_pad; j += THREADS) {
+                uint32_t d = (uint32_t)BINS;
+                if (j < ncand_fast) {
+                    const uint32_t key = order_key(__ldg(src + sm.cand[j]));
+                    if ((key & mask) == prefix) d = (key >> shift) & (uint32_t)(nb - 1);
+                }
+                hist_add(sm.hist, d, lane);
+            }
+            __syncthreads();
+            if (warp == 0) select_bin(sm.hist, nb, remaining, sm.scal);
+            __syncthreads();
+            remaining -= sm.scal[1];
+            prefix |= (uint32_t)sm.scal[0] << shift;
+            mask |= (uint32_t)(nb - 1) << shift;
+            __syncthreads();
+        }
+        const uint32_t thr = prefix;
+        const int need_eq = remaining;
+        const int count_gt = K - need_eq;
+        // every key > thr is a candidate: per-warp-range counts from the candidate list
+        for (int j = tid; j < ncand_fast; j += THREADS) {
+            const int i = sm.cand[j];
+            const uint32_t key = order_key(__ldg(src + i));
+            if (key > thr) atomicAdd(&sm.warp_gt[i / R], 1);
+            else if (key == thr) atomicAdd(&sm.warp_eq[i / R], 1);
+        }
+        __syncthreads();
+        int gt_off = 0, eq_off = 0;
+        for (int w2 = 0; w2 < warp; ++w2) {
+            gt_off += sm.warp_gt[w2];
+            eq_off += sm.warp_eq[w2];
+        }
+        ordered_output(src, wb, we, lane, thr, need_eq, count_gt, K, gt_off, eq_off, out);
+        return;
+    }
+    // ---- general path (the sample was not representative): full radix selection
     for (int i = tid; i < BINS; i += THREADS) sm.hist[i] = 0;
     if (tid < WARPS) {
         sm.warp_gt[tid] = 0;
@@ -148,8 +310,6 @@ __global__ void __launch_bounds__(THREADS) topk_rows_kernel(Problem P, const flo
 
     // ---- pass 1: histogram of bits 31..21
     {
-        const float4 *s4 = reinterpret_cast<const float4 *>(src);
-        const int n4 = n >> 2;
         for (int base = 0; base < n4; base += THREADS * 4) {
             float4 v[4];
 #pragma unroll
@@ -176,9 +336,6 @@ __global__ void __launch_bounds__(THREADS) topk_rows_kernel(Problem P, const flo
     int remaining = K - sm.scal[1];
 
     // ---- pass 2: per-warp count of keys above bin b0, compaction of the keys in b0
-    const int R = ((n + WARPS * 128 - 1) / (WARPS * 128)) * 128;   // warp range, multiple of 128
-    const int wb = warp * R;
-    const int we = min(n, wb + R);
     {
         int g0 = 0;
         for (int base = wb; base < we; base += 128) {
@@ -262,41 +419,12 @@ __global__ void __launch_bounds__(THREADS) topk_rows_kernel(Problem P, const flo
         }
     }
     __syncthreads();
-
-    // ---- pass 3: ordered output
-    int gt_off = 0, eq_off = 0;
+    int gt_off0 = 0, eq_off0 = 0;
     for (int w2 = 0; w2 < warp; ++w2) {
-        gt_off += sm.warp_gt0[w2] + sm.warp_gt[w2];
-        eq_off += sm.warp_eq[w2];
+        gt_off0 += sm.warp_gt0[w2] + sm.warp_gt[w2];
+        eq_off0 += sm.warp_eq[w2];
     }
-    for (int base = wb; base < we; base += 128) {
-        const int i0 = base + lane * 4;
-        uint32_t k[4];
-        load4(src, i0, we, k);
-        int cg = 0, ce = 0;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const bool v = i0 + c < we;
-            cg += v && k[c] > thr;
-            ce += v && k[c] == thr;
-        }
-        int tg, te;
-        int og = warp_excl_scan(cg, lane, tg) + gt_off;
-        int oe = warp_excl_scan(ce, lane, te) + eq_off;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            if (i0 + c >= we) continue;
-            if (k[c] > thr) {
-                if (og < count_gt) out[og] = i0 + c;
-                ++og;
-            } else if (k[c] == thr) {
-                if (oe < need_eq && count_gt + oe < K) out[count_gt + oe] = i0 + c;
-                ++oe;
-            }
-        }
-        gt_off += tg;
-        eq_off += te;
-    }
+    ordered_output(src, wb, we, lane, thr, need_eq, count_gt, K, gt_off0, eq_off0, out);
 }
 
 }  // namespace topk
