@@ -13,6 +13,8 @@ from ._native import (  # noqa: F401
     DsaProblem,
     dsa_check_device_errors,
     dsa_forward,
+    dsa_forward_noalloc,
+    dsa_forward_noalloc_scratch_bytes,
     dsa_forward_workspace_size,
     dsa_indexer_scores,
     dsa_sparse_mla_fwd,
@@ -26,6 +28,7 @@ from ._native import (  # noqa: F401
 
 __all__ = [
     "DSA_BF16", "DSA_E4M3", "DsaError", "DsaProblem", "dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_fwd",
-    "dsa_forward_workspace_size", "dsa_forward", "dsa_check_device_errors", "make_problem",
+    "dsa_forward_workspace_size", "dsa_forward", "dsa_forward_noalloc", "dsa_forward_noalloc_scratch_bytes",
+    "dsa_check_device_errors", "make_problem",
     "problem_from_inputs", "scores_ld", "load", "library_path",
 ]

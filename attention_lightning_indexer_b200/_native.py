@@ -33,6 +33,8 @@ EXPORTED = (
     "dsa_sparse_mla_fwd",
     "dsa_forward_workspace_size",
     "dsa_forward",
+    "dsa_forward_noalloc",
+    "dsa_forward_noalloc_scratch_bytes",
     "dsa_check_device_errors",
     "dsa_status_string",
     "dsa_abi_version",
@@ -92,11 +94,15 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.dsa_forward_workspace_size.argtypes = [pp, i32]
     lib.dsa_forward_workspace_size.restype = sz
     lib.dsa_forward.argtypes = [pp, P, P, P, P, P, P, P, i32, P, P, P, P, sz, P]
+    lib.dsa_forward_noalloc.argtypes = [pp, P, P, P, P, P, P, P, P, P, P, P]
+    lib.dsa_forward_noalloc_scratch_bytes.argtypes = []
+    lib.dsa_forward_noalloc_scratch_bytes.restype = sz
     lib.dsa_check_device_errors.argtypes = [P]
     lib.dsa_status_string.argtypes = [ctypes.c_int]
     lib.dsa_status_string.restype = ctypes.c_char_p
     lib.dsa_abi_version.restype = i32
-    for name in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_forward", "dsa_check_device_errors"):
+    for name in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_forward", "dsa_forward_noalloc",
+                 "dsa_check_device_errors"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -184,6 +190,20 @@ def dsa_forward(p: DsaProblem, q_idx, k_idx, w, q, kv, out, lse, workspace, chun
     _check(lib.dsa_forward(ctypes.byref(p), _ptr(q_idx), _ptr(q_scale), _ptr(k_idx), _ptr(k_scale), _ptr(w), _ptr(q),
                            _ptr(kv), chunk_q, _ptr(idx_out), _ptr(out), _ptr(lse), _ptr(workspace),
                            workspace.numel() * workspace.element_size(), _stream(stream)), "dsa_forward")
+
+
+def dsa_forward_noalloc(p: DsaProblem, q_idx, k_idx, w, q, kv, idx_out, out, lse, q_scale=None, k_scale=None,
+                        stream=None) -> None:
+    """dsa_forward with the library's fixed scratch array instead of a caller workspace (no
+    device allocation by the call; see include/dsa.h for the size limit and sharing rules)."""
+    lib = load()
+    _check(lib.dsa_forward_noalloc(ctypes.byref(p), _ptr(q_idx), _ptr(q_scale), _ptr(k_idx), _ptr(k_scale), _ptr(w),
+                                   _ptr(q), _ptr(kv), _ptr(idx_out), _ptr(out), _ptr(lse), _stream(stream)),
+           "dsa_forward_noalloc")
+
+
+def dsa_forward_noalloc_scratch_bytes() -> int:
+    return int(load().dsa_forward_noalloc_scratch_bytes())
 
 
 def dsa_check_device_errors(stream=None) -> None:

@@ -296,3 +296,80 @@ dsa_status_t dsa_check_device_errors(dsa_stream_t stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------
+// Allocation-free variant of dsa_forward.
+//
+// Some callers cannot allocate device memory at the point where they run the path: code
+// that runs inside a host callback or a custom allocator, runtimes that own all device
+// memory up front and hand out nothing else, or deployments where a cudaMalloc in the
+// serving loop would stall other streams.  dsa_forward_noalloc serves them: its only
+// scratch (the fp32 index scores of one chunk of query rows) lives in the fixed array
+// below, so the call itself never allocates or frees anything.
+//
+//   * The array holds NOALLOC_SCRATCH_BYTES (32 MiB).  Every GPU that loads this library
+//     keeps it resident until the process exits.
+//   * Its device address is looked up once per device, on the first call made with that
+//     device current (cudaGetSymbolAddress); make that first call outside any stream
+//     capture.
+//   * All calls share the array and it keeps whatever the last call left: calls whose
+//     work overlaps on the GPU (e.g. on two streams without ordering) race on it.  No
+//     part of it needs to start at zero -- every score the top-k reads is written first by
+//     the indexer of the same chunk.
+// ---------------------------------------------------------------------------------------
+namespace {
+
+constexpr size_t NOALLOC_SCRATCH_BYTES = size_t(32) << 20;
+constexpr int NOALLOC_MAX_DEVICES = 64;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
+
+// Per-device address of g_noalloc_scratch (nullptr until looked up).
+void *g_noalloc_addr[NOALLOC_MAX_DEVICES] = {};
+
+dsa_status_t noalloc_scratch(float **scratch) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= NOALLOC_MAX_DEVICES) return DSA_ERR_CUDA;
+    if (g_noalloc_addr[dev] == nullptr) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return DSA_ERR_CUDA;
+        g_noalloc_addr[dev] = ptr;
+    }
+    *scratch = reinterpret_cast<float *>(g_noalloc_addr[dev]);
+    return DSA_OK;
+}
+
+}  // namespace
+
+extern "C" dsa_status_t dsa_forward_noalloc(const dsa_problem_t *p, const void *q_idx, const float *q_scale,
+                                            const void *k_idx, const float *k_scale, const float *w, const void *q,
+                                            const void *kv, int32_t *idx_out, void *out, float *lse,
+                                            dsa_stream_t stream) {
+    dsa_status_t st = check_problem(p);
+    if (st != DSA_OK) return st;
+    if (p->total_q == 0) return DSA_OK;
+    if (!q_idx || !k_idx || !w || !q || !kv || !idx_out || !out || !lse) return DSA_ERR_INVALID_ARG;
+    if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(w) || !aligned16(q) || !aligned16(kv) ||
+        !aligned16(idx_out) || !aligned16(out) || !aligned16(lse))
+        return DSA_ERR_INVALID_ARG;
+    if (p->idx_dtype == DSA_E4M3 && (!q_scale || !k_scale)) return DSA_ERR_INVALID_ARG;
+    // rows of scores that fit in the fixed scratch; a single row must fit
+    const int64_t ld = scores_ld(p);
+    const int64_t rows_fit = (int64_t)(NOALLOC_SCRATCH_BYTES / ((size_t)ld * sizeof(float)));
+    if (rows_fit < 1) return DSA_ERR_WORKSPACE;
+    const int chunk = (int)(rows_fit < p->total_q ? rows_fit : p->total_q);
+    float *scores = nullptr;
+    if ((st = noalloc_scratch(&scores)) != DSA_OK) return st;
+    if ((st = set_smem_attrs()) != DSA_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    for (int r0 = 0; r0 < p->total_q; r0 += chunk) {
+        const int rc = p->total_q - r0 < chunk ? p->total_q - r0 : chunk;
+        st = indexer_launch(p, q_idx, q_scale, k_idx, k_scale, w, scores, ld, r0, rc, s);
+        if (st != DSA_OK) return st;
+        st = topk_launch(p, scores, ld, r0, rc, idx_out + (int64_t)r0 * p->topk, s);
+        if (st != DSA_OK) return st;
+    }
+    return mla_launch(p, q, kv, idx_out, out, lse, s);
+}
+
+extern "C" size_t dsa_forward_noalloc_scratch_bytes(void) { return NOALLOC_SCRATCH_BYTES; }

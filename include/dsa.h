@@ -153,6 +153,28 @@ dsa_status_t dsa_forward(const dsa_problem_t *p, const void *q_idx, const float 
                          void *workspace, size_t workspace_bytes, dsa_stream_t stream);
 
 /*
+ * dsa_forward without a workspace argument, for callers that cannot allocate device
+ * memory where they run the path (host callbacks, runtimes that own all device memory,
+ * serving loops that must not call cudaMalloc).  The pages have no counterpart: this is
+ * a deployment convenience, not part of the method.
+ * The per-chunk score scratch lives in a fixed device array of
+ * dsa_forward_noalloc_scratch_bytes() bytes (32 MiB) inside the library, held by every GPU
+ * that loads the library until the process exits.  Query rows are processed in chunks
+ * of as many rows as fit; a problem whose longest score row alone (max_len_k rounded up
+ * to 4 fp32) does not fit returns DSA_ERR_WORKSPACE before anything is launched.
+ * idx_out is required here (it is the caller's output, not scratch).
+ * The first call on a device looks up the array's device address (make it outside any
+ * stream capture).  All calls share the array: calls that overlap on the GPU race on it.
+ * Nothing is allocated or freed by this call.
+ */
+dsa_status_t dsa_forward_noalloc(const dsa_problem_t *p, const void *q_idx, const float *q_scale,
+                                 const void *k_idx, const float *k_scale, const float *w, const void *q,
+                                 const void *kv, int32_t *idx_out, void *out, float *lse, dsa_stream_t stream);
+
+/* Size in bytes of the fixed scratch array used by dsa_forward_noalloc. */
+size_t dsa_forward_noalloc_scratch_bytes(void);
+
+/*
  * Synchronises `stream`, then reads and clears the device-side error flag of the
  * current device (set by a kernel whose bounded wait gave up).  Returns DSA_OK,
  * DSA_ERR_DEVICE_TIMEOUT, or DSA_ERR_CUDA if the synchronisation itself failed.
