@@ -91,7 +91,10 @@ dsa_status_t set_smem_attrs() {
     static bool done = false;
     if (done) return DSA_OK;
     cudaError_t e = cudaSuccess;
-    e = cudaFuncSetAttribute(dsa::mla::sparse_mla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(dsa::topk::topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             dsa::topk::SMEM);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(dsa::mla::sparse_mla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              dsa::mla::TcCfg::SMEM);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(dsa::indexer::indexer_tc_kernel<8, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -154,7 +157,8 @@ dsa_status_t topk_launch(const dsa_problem_t *p, const float *scores, int64_t ld
                          int32_t *idx, cudaStream_t stream) {
     if (row_count == 0) return DSA_OK;
     Problem P = to_dev(p);
-    dsa::topk::topk_rows_kernel<<<row_count, dsa::topk::THREADS, 0, stream>>>(P, scores, ld, row_begin, idx);
+    dsa::topk::topk_rows_kernel<<<row_count, dsa::topk::THREADS, dsa::topk::SMEM, stream>>>(P, scores, ld, row_begin,
+                                                                                           idx);
     return launch_status();
 }
 

@@ -4,23 +4,22 @@
 // top-k index scores of each query; "Model techniques map -- DeepSeek-V3.2",
 // Indexer-selected sparse attention: k_eff = min(index_topk, #candidates), int32 out.
 //
-// Design (one 256-thread CTA per query row; HBM-bound, several CTAs per SM):
-//   * scores map to order-preserving 32-bit keys (-0.0 folded onto +0.0), so comparing
-//     keys as unsigned integers compares the floats as values;
-//   * pass 1 (the only HBM read of the row): histogram of the top 11 key bits, 4 float4
-//     loads in flight per thread, warp-aggregated shared atomics (match.any);
-//   * the bin holding the k-th largest key is found; pass 2 (an L2 re-read) counts, per
-//     warp range, the keys in higher bins (certainly selected) and compacts the indices
-//     of the keys in that bin (the candidates) into shared memory;
-//   * digits 2 (bits 20..10) and 3 (bits 9..0) are resolved on the candidates only,
-//     giving the exact k-th largest key `thr` and the number `need_eq` of keys equal to
-//     it that are taken (smallest indices first);
-//   * pass 3 (an L2 re-read) writes, in ascending index order, every key > thr followed
-//     by the first need_eq keys == thr, from per-warp offsets and in-warp prefix sums:
-//     the output is deterministic and independent of the launch shape.
-// When the candidates overflow the shared buffer (e.g. a row of identical scores) the
-// later digits and the per-warp counts are taken from the row itself instead (slower,
-// same result).
+// Scores map to order-preserving 32-bit keys (-0.0 folded onto +0.0), so comparing keys
+// as unsigned integers compares the floats as values.  One 256-thread CTA per row.
+//
+// Fast path (one HBM read of the row):
+//   * every 16th float4 of the row is sampled; an exact radix select on the sample gives
+//     a key t_lo that about 1.2 k keys of the full row are expected to reach;
+//   * one pass over the row keeps the keys >= t_lo with their indices, each warp in its
+//     own shared-memory segment and in ascending index order (ballot prefix sums, no
+//     atomics);
+//   * an exact radix select (11/11/10-bit digits) over these candidates gives the k-th
+//     largest key `thr` and how many keys equal to it are taken (smallest indices first);
+//   * the candidates > thr and the first `need_eq` == thr are written in ascending index
+//     order from per-warp offsets: deterministic, independent of the launch shape.
+// If the sample misjudged (fewer than k candidates, or a warp's segment overflows) the
+// general path runs instead: a full-row radix select with candidate compaction and an
+// ordered final pass over the row (same result, more passes).
 #pragma once
 
 #include "dsa_common.cuh"
@@ -31,23 +30,23 @@ namespace topk {
 constexpr int THREADS = 256;
 constexpr int WARPS = THREADS / 32;
 constexpr int BINS = 2048;        // 11-bit digits
-constexpr int CAND_CAP = 6144;    // candidates kept after the first digit
+constexpr int SEG = 1024;         // candidate slots per warp (fast path)
+constexpr int CAND_CAP = WARPS * SEG * 2;   // general-path candidate indices (same bytes)
 constexpr unsigned FULL = 0xffffffffu;
+
+// Dynamic shared memory layout.
+constexpr int OFF_HIST = 0;                               // [BINS] u32
+constexpr int OFF_SEGK = OFF_HIST + BINS * 4;             // [WARPS][SEG] u32 keys (also: samples)
+constexpr int OFF_SEGI = OFF_SEGK + WARPS * SEG * 4;      // [WARPS][SEG] int indices
+constexpr int OFF_SCAL = OFF_SEGI + WARPS * SEG * 4;      // small scalars [64]
+constexpr int SMEM = OFF_SCAL + 64 * 4;
+static_assert(CAND_CAP * 4 == 2 * WARPS * SEG * 4, "general-path candidates reuse both segment arrays");
 
 __device__ __forceinline__ uint32_t order_key(float f) {
     uint32_t u = __float_as_uint(f);
     if (u == 0x80000000u) u = 0u;  // -0.0 == +0.0
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
-
-struct Smem {
-    uint32_t hist[BINS];
-    int cand[CAND_CAP];
-    int warp_gt0[WARPS];   // keys whose first digit is above the threshold bin, per warp range
-    int warp_gt[WARPS];    // candidates above thr, per warp range
-    int warp_eq[WARPS];    // candidates equal to thr, per warp range
-    int scal[8];           // [0] bin  [1] above  [2] ncand
-};
 
 // Warp-aggregated histogram increment; d == BINS means "no key" (lane still participates).
 __device__ __forceinline__ void hist_add(uint32_t *hist, uint32_t d, int lane) {
@@ -102,28 +101,52 @@ __device__ __forceinline__ int warp_excl_scan(int v, int lane, int &total) {
 }
 
 // The lane's 4 consecutive keys i0..i0+3 of the warp range [.., we); invalid ones get 0.
-__device__ __forceinline__ int load4(const float *src, int i0, int we, uint32_t (&k)[4]) {
+__device__ __forceinline__ void load4(const float *src, int i0, int we, uint32_t (&k)[4]) {
     if (i0 + 3 < we) {
         const float4 v = __ldg(reinterpret_cast<const float4 *>(src + i0));
         k[0] = order_key(v.x);
         k[1] = order_key(v.y);
         k[2] = order_key(v.z);
         k[3] = order_key(v.w);
-        return 4;
+        return;
     }
-    int nv = 0;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        k[c] = 0u;
-        if (i0 + c < we) {
-            k[c] = order_key(__ldg(src + i0 + c));
-            ++nv;
-        }
-    }
-    return nv;
+    for (int c = 0; c < 4; ++c) k[c] = i0 + c < we ? order_key(__ldg(src + i0 + c)) : 0u;
 }
 
-// Pass 3: warp w writes, in ascending index order, the keys of its range [wb, we) that
+// Exact radix selection (11/11/10-bit digits, MSB first) of the `rank`-th largest key among
+// the keys get(j), j < m, for which valid(j) holds.  Returns the key; *above receives the
+// number of keys strictly greater.  All threads call it; uses hist and scal[0..1].
+template <class Get>
+__device__ uint32_t radix_select(int m, int rank, Get get, uint32_t *hist, int *scal, int *above) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint32_t prefix = 0, mask = 0;
+    int remaining = rank, above_total = 0;
+    const int m_pad = (m + 31) & ~31;
+    for (int pass = 0; pass < 3; ++pass) {
+        const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+        const int nb = pass == 2 ? 1024 : 2048;
+        for (int i = tid; i < nb; i += THREADS) hist[i] = 0;
+        __syncthreads();
+        for (int j = tid; j < m_pad; j += THREADS) {
+            uint32_t d = (uint32_t)BINS, key = 0;
+            if (j < m && get(j, key) && (key & mask) == prefix) d = (key >> shift) & (uint32_t)(nb - 1);
+            hist_add(hist, d, lane);
+        }
+        __syncthreads();
+        if (warp == 0) select_bin(hist, nb, remaining, scal);
+        __syncthreads();
+        remaining -= scal[1];
+        above_total += scal[1];
+        prefix |= (uint32_t)scal[0] << shift;
+        mask |= (uint32_t)(nb - 1) << shift;
+        __syncthreads();
+    }
+    *above = above_total;
+    return prefix;
+}
+
+// Warp w writes, in ascending index order, the keys of its range [wb, we) of the row that
 // are > thr (from slot gt_off on) and those == thr whose rank among equal keys is below
 // need_eq (from slot count_gt + eq_off on).
 __device__ __forceinline__ void ordered_output(const float *src, int wb, int we, int lane, uint32_t thr, int need_eq,
@@ -158,182 +181,170 @@ __device__ __forceinline__ void ordered_output(const float *src, int wb, int we,
     }
 }
 
-__global__ void __launch_bounds__(THREADS) topk_rows_kernel(Problem P, const float *__restrict__ scores, int64_t ld,
-                                                            int row_begin, int32_t *__restrict__ idx) {
-    __shared__ Smem sm;
+// Fast path.  Returns false (nothing written) when the sample misjudged the row.
+__device__ bool select_row_sampled(const float *src, int n, int K, unsigned char *smem, int32_t *out) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int r = blockIdx.x;
-    const int K = P.topk;
-    int32_t *out = idx + (int64_t)r * K;
-    const RowInfo ri = row_info(P, row_begin + r);
-    const int n = visible_keys(ri);
-    if (n <= K) {   // select every visible key
-        for (int j = tid; j < K; j += THREADS) out[j] = j < n ? j : -1;
-        return;
-    }
-    const float *src = scores + (int64_t)r * ld;
+    uint32_t *hist = reinterpret_cast<uint32_t *>(smem + OFF_HIST);
+    uint32_t *segk = reinterpret_cast<uint32_t *>(smem + OFF_SEGK);
+    int *segi = reinterpret_cast<int *>(smem + OFF_SEGI);
+    int *scal = reinterpret_cast<int *>(smem + OFF_SCAL);   // [0..1] select, [8..15] seg counts, [16] flag
     const float4 *s4 = reinterpret_cast<const float4 *>(src);
     const int n4 = n >> 2;
-    const int R = ((n + WARPS * 128 - 1) / (WARPS * 128)) * 128;   // warp range, multiple of 128
-    const int wb = warp * R;
-    const int we = min(n, wb + R);
+    const int nsamp4 = (n4 + 15) / 16;                       // sampled float4 (every 16th)
+    const int ns = 4 * nsamp4;
+    if (ns < 64 || ns > WARPS * SEG) return false;
 
-    // ---- fast path: a sample fixes a lower digit bound; only keys at or above it are counted
-    for (int i = tid; i < BINS; i += THREADS) sm.hist[i] = 0;
-    if (tid < WARPS) {
-        sm.warp_gt[tid] = 0;
-        sm.warp_eq[tid] = 0;
-    }
-    if (tid < 8) sm.scal[tid] = 0;
-    __syncthreads();
-    int ns = 0;                                            // sampled keys (every 16th float4)
-    for (int m = tid; 16 * m < n4; m += THREADS) {
+    // ---- sample keys into the segment key array (free at this point)
+    for (int m = tid; m < nsamp4; m += THREADS) {
         const float4 v = __ldg(s4 + 16 * m);
-        atomicAdd(&sm.hist[order_key(v.x) >> 21], 1u);
-        atomicAdd(&sm.hist[order_key(v.y) >> 21], 1u);
-        atomicAdd(&sm.hist[order_key(v.z) >> 21], 1u);
-        atomicAdd(&sm.hist[order_key(v.w) >> 21], 1u);
+        segk[4 * m + 0] = order_key(v.x);
+        segk[4 * m + 1] = order_key(v.y);
+        segk[4 * m + 2] = order_key(v.z);
+        segk[4 * m + 3] = order_key(v.w);
     }
-    ns = 4 * ((n4 + 15) / 16);
+    if (tid < WARPS) scal[8 + tid] = 0;
+    if (tid == 0) scal[16] = 0;
     __syncthreads();
-    if (warp == 0) {
-        // lowest bin b_lo whose sampled tail covers ~1.5 K keys of the full row (+ margin)
-        const uint32_t target = (uint32_t)((1.5 * K * (double)ns) / (double)n) + 16u;
-        select_bin(sm.hist, BINS, (int)min(target, (uint32_t)ns), sm.scal);   // scal[0] = b_lo
-    }
-    __syncthreads();
-    const uint32_t b_lo = (uint32_t)sm.scal[0];
-    __syncthreads();
-    for (int i = tid; i < BINS; i += THREADS) sm.hist[i] = 0;
-    if (tid == 0) sm.scal[2] = 0;
-    __syncthreads();
-    {
-        for (int base = 0; base < n4; base += THREADS * 4) {
-            float4 v[4];
+    const int target = min(ns, (int)((1.2 * K * (double)ns) / (double)n) + 16);
+    int dummy;
+    const uint32_t t_lo = radix_select(
+        ns, target, [&](int j, uint32_t &key) { key = segk[j]; return true; }, hist, scal, &dummy);
+    __syncthreads();   // samples no longer needed
+
+    // ---- candidates: keys >= t_lo, per warp in ascending index order
+    const int R = ((n + WARPS * 128 - 1) / (WARPS * 128)) * 128;
+    const int wb = warp * R, we = min(n, wb + R);
+    uint32_t *mk = segk + warp * SEG;
+    int *mi = segi + warp * SEG;
+    int cnt = 0;
+    bool overflow = false;
+    for (int base = wb; base < we; base += 128) {
+        const int i0 = base + lane * 4;
+        uint32_t k[4];
+        load4(src, i0, we, k);
+        int c4 = 0;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int i = base + u * THREADS + tid;
-                v[u] = i < n4 ? __ldg(s4 + i) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-            }
+        for (int c = 0; c < 4; ++c) c4 += (i0 + c < we) && k[c] >= t_lo;
+        int tot;
+        int off = cnt + warp_excl_scan(c4, lane, tot);
+        if (cnt + tot > SEG) overflow = true;
+        if (!overflow) {
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int i4 = base + u * THREADS + tid;
-                const float e[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const uint32_t key = order_key(e[c]);
-                    const bool is = i4 < n4 && (key >> 21) >= b_lo;
-                    const unsigned bal = __ballot_sync(FULL, is);
-                    if (bal) {
-                        int slot0 = 0;
-                        if (lane == __ffs(bal) - 1) slot0 = atomicAdd(&sm.scal[2], __popc(bal));
-                        slot0 = __shfl_sync(FULL, slot0, __ffs(bal) - 1);
-                        if (is) {
-                            const int slot = slot0 + __popc(bal & ((1u << lane) - 1u));
-                            if (slot < CAND_CAP) sm.cand[slot] = 4 * i4 + c;
-                            atomicAdd(&sm.hist[key >> 21], 1u);
-                        }
-                    }
+            for (int c = 0; c < 4; ++c) {
+                if ((i0 + c < we) && k[c] >= t_lo) {
+                    mk[off] = k[c];
+                    mi[off] = i0 + c;
+                    ++off;
                 }
             }
         }
-        const int tail = n - (n4 << 2);
-        if (tid < tail) {
-            const int i = (n4 << 2) + tid;
-            const uint32_t key = order_key(__ldg(src + i));
-            if ((key >> 21) >= b_lo) {
-                const int slot = atomicAdd(&sm.scal[2], 1);
-                if (slot < CAND_CAP) sm.cand[slot] = i;
-                atomicAdd(&sm.hist[key >> 21], 1u);
-            }
-        }
+        cnt += tot;
+    }
+    if (lane == 0) {
+        scal[8 + warp] = overflow ? 0 : cnt;
+        if (overflow) scal[16] = 1;
     }
     __syncthreads();
-    const int ncand_fast = sm.scal[2];
-    const bool fast = ncand_fast >= K && ncand_fast <= CAND_CAP;
-    if (fast) {
-        // exact digits 1..3 on the candidates (bins below b_lo hold no count)
-        if (warp == 0) select_bin(sm.hist, BINS, K, sm.scal);
-        __syncthreads();
-        int remaining = K - sm.scal[1];
-        uint32_t prefix = (uint32_t)sm.scal[0] << 21, mask = 0xFFE00000u;
-        __syncthreads();
-        for (int pass = 1; pass <= 2; ++pass) {
-            const int shift = pass == 1 ? 10 : 0;
-            const int nb = pass == 1 ? 2048 : 1024;
-            for (int i = tid; i < nb; i += THREADS) sm.hist[i] = 0;
-            __syncthreads();
-            const int m_pad = (ncand_fast + 31) & ~31;
-            for (int j = tid; j < m_pad; j += THREADS) {
-                uint32_t d = (uint32_t)BINS;
-                if (j < ncand_fast) {
-                    const uint32_t key = order_key(__ldg(src + sm.cand[j]));
-                    if ((key & mask) == prefix) d = (key >> shift) & (uint32_t)(nb - 1);
-                }
-                hist_add(sm.hist, d, lane);
-            }
-            __syncthreads();
-            if (warp == 0) select_bin(sm.hist, nb, remaining, sm.scal);
-            __syncthreads();
-            remaining -= sm.scal[1];
-            prefix |= (uint32_t)sm.scal[0] << shift;
-            mask |= (uint32_t)(nb - 1) << shift;
-            __syncthreads();
-        }
-        const uint32_t thr = prefix;
-        const int need_eq = remaining;
-        const int count_gt = K - need_eq;
-        // every key > thr is a candidate: per-warp-range counts from the candidate list
-        for (int j = tid; j < ncand_fast; j += THREADS) {
-            const int i = sm.cand[j];
-            const uint32_t key = order_key(__ldg(src + i));
-            if (key > thr) atomicAdd(&sm.warp_gt[i / R], 1);
-            else if (key == thr) atomicAdd(&sm.warp_eq[i / R], 1);
-        }
-        __syncthreads();
-        int gt_off = 0, eq_off = 0;
-        for (int w2 = 0; w2 < warp; ++w2) {
-            gt_off += sm.warp_gt[w2];
-            eq_off += sm.warp_eq[w2];
-        }
-        ordered_output(src, wb, we, lane, thr, need_eq, count_gt, K, gt_off, eq_off, out);
-        return;
+    int total = 0;
+    for (int w = 0; w < WARPS; ++w) total += scal[8 + w];
+    if (scal[16] != 0 || total < K) return false;   // uniform decision
+
+    // ---- exact k-th largest among the candidates
+    int above;
+    const uint32_t thr = radix_select(
+        WARPS * SEG, K,
+        [&](int j, uint32_t &key) {
+            if ((j & (SEG - 1)) >= scal[8 + j / SEG]) return false;
+            key = segk[j];
+            return true;
+        },
+        hist, scal, &above);
+    const int need_eq = K - above;                   // >= 1
+    const int count_gt = above;
+
+    // ---- per-warp counts of > thr and == thr, then ordered writes
+    int cg = 0, ce = 0;
+    for (int j = lane; j < cnt; j += 32) {
+        cg += mk[j] > thr;
+        ce += mk[j] == thr;
     }
-    // ---- general path (the sample was not representative): full radix selection
-    for (int i = tid; i < BINS; i += THREADS) sm.hist[i] = 0;
-    if (tid < WARPS) {
-        sm.warp_gt[tid] = 0;
-        sm.warp_eq[tid] = 0;
+    cg = warp_sum(cg);
+    ce = warp_sum(ce);
+    __syncthreads();
+    if (lane == 0) {
+        scal[24 + warp] = cg;
+        scal[32 + warp] = ce;
     }
-    if (tid == 0) sm.scal[2] = 0;
+    __syncthreads();
+    int gt_off = 0, eq_off = 0;
+    for (int w2 = 0; w2 < warp; ++w2) {
+        gt_off += scal[24 + w2];
+        eq_off += scal[32 + w2];
+    }
+    const unsigned lt = (1u << lane) - 1u;
+    for (int base = 0; base < cnt; base += 32) {
+        const int j = base + lane;
+        const uint32_t key = j < cnt ? mk[j] : 0u;
+        const bool g = j < cnt && key > thr, e = j < cnt && key == thr;
+        const unsigned bg = __ballot_sync(FULL, g), be = __ballot_sync(FULL, e);
+        if (g) {
+            const int slot = gt_off + __popc(bg & lt);
+            if (slot < count_gt) out[slot] = mi[j];
+        }
+        if (e) {
+            const int rank = eq_off + __popc(be & lt);
+            if (rank < need_eq && count_gt + rank < K) out[count_gt + rank] = mi[j];
+        }
+        gt_off += __popc(bg);
+        eq_off += __popc(be);
+    }
+    return true;
+}
+
+// General path: full radix selection over the row.
+__device__ void select_row_general(const float *src, int n, int K, unsigned char *smem, int32_t *out) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint32_t *hist = reinterpret_cast<uint32_t *>(smem + OFF_HIST);
+    int *cand = reinterpret_cast<int *>(smem + OFF_SEGK);   // CAND_CAP entries over both segment arrays
+    int *scal = reinterpret_cast<int *>(smem + OFF_SCAL);   // [0..1] select, [2] ncand, [8..] warp counts
+    const float4 *s4 = reinterpret_cast<const float4 *>(src);
+    const int n4 = n >> 2;
+    const int R = ((n + WARPS * 128 - 1) / (WARPS * 128)) * 128;
+    const int wb = warp * R, we = min(n, wb + R);
+
+    __syncthreads();
+    for (int i = tid; i < BINS; i += THREADS) hist[i] = 0;
+    if (tid < 3 * WARPS) scal[8 + tid] = 0;
+    if (tid == 0) scal[2] = 0;
     __syncthreads();
 
-    // ---- pass 1: histogram of bits 31..21
-    {
-        for (int base = 0; base < n4; base += THREADS * 4) {
-            float4 v[4];
+    // ---- pass 1: histogram of bits 31..21 over the whole row
+    for (int base = 0; base < n4; base += THREADS * 4) {
+        float4 v[4];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int i = base + u * THREADS + tid;
-                v[u] = i < n4 ? __ldg(s4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const bool ok = base + u * THREADS + tid < n4;
-                hist_add(sm.hist, ok ? order_key(v[u].x) >> 21 : (uint32_t)BINS, lane);
-                hist_add(sm.hist, ok ? order_key(v[u].y) >> 21 : (uint32_t)BINS, lane);
-                hist_add(sm.hist, ok ? order_key(v[u].z) >> 21 : (uint32_t)BINS, lane);
-                hist_add(sm.hist, ok ? order_key(v[u].w) >> 21 : (uint32_t)BINS, lane);
-            }
+        for (int u = 0; u < 4; ++u) {
+            const int i = base + u * THREADS + tid;
+            v[u] = i < n4 ? __ldg(s4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const bool ok = base + u * THREADS + tid < n4;
+            hist_add(hist, ok ? order_key(v[u].x) >> 21 : (uint32_t)BINS, lane);
+            hist_add(hist, ok ? order_key(v[u].y) >> 21 : (uint32_t)BINS, lane);
+            hist_add(hist, ok ? order_key(v[u].z) >> 21 : (uint32_t)BINS, lane);
+            hist_add(hist, ok ? order_key(v[u].w) >> 21 : (uint32_t)BINS, lane);
+        }
+    }
+    {
         const int tail = n - (n4 << 2);
-        if (tid < tail) atomicAdd(&sm.hist[order_key(__ldg(src + (n4 << 2) + tid)) >> 21], 1u);
+        if (tid < tail) atomicAdd(&hist[order_key(__ldg(src + (n4 << 2) + tid)) >> 21], 1u);
     }
     __syncthreads();
-    if (warp == 0) select_bin(sm.hist, BINS, K, sm.scal);
+    if (warp == 0) select_bin(hist, BINS, K, scal);
     __syncthreads();
-    const uint32_t b0 = (uint32_t)sm.scal[0];
-    int remaining = K - sm.scal[1];
+    const uint32_t b0 = (uint32_t)scal[0];
+    int remaining = K - scal[1];
+    __syncthreads();
 
     // ---- pass 2: per-warp count of keys above bin b0, compaction of the keys in b0
     {
@@ -349,16 +360,16 @@ __global__ void __launch_bounds__(THREADS) topk_rows_kernel(Problem P, const flo
                 if (d > b0) {
                     ++g0;
                 } else if (d == b0) {
-                    const int slot = atomicAdd(&sm.scal[2], 1);
-                    if (slot < CAND_CAP) sm.cand[slot] = i0 + c;
+                    const int slot = atomicAdd(&scal[2], 1);
+                    if (slot < CAND_CAP) cand[slot] = i0 + c;
                 }
             }
         }
         g0 = warp_sum(g0);
-        if (lane == 0) sm.warp_gt0[warp] = g0;
+        if (lane == 0) scal[8 + warp] = g0;
     }
     __syncthreads();
-    const int ncand = sm.scal[2];
+    const int ncand = scal[2];
     const bool use_cand = ncand <= CAND_CAP;
 
     // ---- digits 2 and 3 on the candidates (or on the whole row after an overflow)
@@ -366,23 +377,23 @@ __global__ void __launch_bounds__(THREADS) topk_rows_kernel(Problem P, const flo
     for (int pass = 1; pass <= 2; ++pass) {
         const int shift = pass == 1 ? 10 : 0;
         const int nb = pass == 1 ? 2048 : 1024;
-        for (int i = tid; i < nb; i += THREADS) sm.hist[i] = 0;
+        for (int i = tid; i < nb; i += THREADS) hist[i] = 0;
         __syncthreads();
         const int m = use_cand ? ncand : n;
         const int m_pad = (m + 31) & ~31;
         for (int j = tid; j < m_pad; j += THREADS) {
             uint32_t d = (uint32_t)BINS;
             if (j < m) {
-                const uint32_t key = order_key(__ldg(src + (use_cand ? sm.cand[j] : j)));
+                const uint32_t key = order_key(__ldg(src + (use_cand ? cand[j] : j)));
                 if ((key & mask) == prefix) d = (key >> shift) & (uint32_t)(nb - 1);
             }
-            hist_add(sm.hist, d, lane);
+            hist_add(hist, d, lane);
         }
         __syncthreads();
-        if (warp == 0) select_bin(sm.hist, nb, remaining, sm.scal);
+        if (warp == 0) select_bin(hist, nb, remaining, scal);
         __syncthreads();
-        remaining -= sm.scal[1];
-        prefix |= (uint32_t)sm.scal[0] << shift;
+        remaining -= scal[1];
+        prefix |= (uint32_t)scal[0] << shift;
         mask |= (uint32_t)(nb - 1) << shift;
         __syncthreads();
     }
@@ -393,10 +404,10 @@ __global__ void __launch_bounds__(THREADS) topk_rows_kernel(Problem P, const flo
     // ---- per-warp counts of the keys > thr and == thr inside bin b0
     if (use_cand) {
         for (int j = tid; j < ncand; j += THREADS) {
-            const int i = sm.cand[j];
+            const int i = cand[j];
             const uint32_t key = order_key(__ldg(src + i));
-            if (key > thr) atomicAdd(&sm.warp_gt[i / R], 1);
-            else if (key == thr) atomicAdd(&sm.warp_eq[i / R], 1);
+            if (key > thr) atomicAdd(&scal[16 + i / R], 1);
+            else if (key == thr) atomicAdd(&scal[24 + i / R], 1);
         }
     } else {
         int cg = 0, ce = 0;
@@ -414,17 +425,34 @@ __global__ void __launch_bounds__(THREADS) topk_rows_kernel(Problem P, const flo
         cg = warp_sum(cg);
         ce = warp_sum(ce);
         if (lane == 0) {
-            sm.warp_gt[warp] = cg;
-            sm.warp_eq[warp] = ce;
+            scal[16 + warp] = cg;
+            scal[24 + warp] = ce;
         }
     }
     __syncthreads();
-    int gt_off0 = 0, eq_off0 = 0;
+    int gt_off = 0, eq_off = 0;
     for (int w2 = 0; w2 < warp; ++w2) {
-        gt_off0 += sm.warp_gt0[w2] + sm.warp_gt[w2];
-        eq_off0 += sm.warp_eq[w2];
+        gt_off += scal[8 + w2] + scal[16 + w2];
+        eq_off += scal[24 + w2];
     }
-    ordered_output(src, wb, we, lane, thr, need_eq, count_gt, K, gt_off0, eq_off0, out);
+    ordered_output(src, wb, we, lane, thr, need_eq, count_gt, K, gt_off, eq_off, out);
+}
+
+// grid = row_count CTAs of THREADS threads, dynamic shared memory SMEM bytes.
+__global__ void __launch_bounds__(THREADS) topk_rows_kernel(Problem P, const float *__restrict__ scores, int64_t ld,
+                                                            int row_begin, int32_t *__restrict__ idx) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int r = blockIdx.x;
+    const int K = P.topk;
+    int32_t *out = idx + (int64_t)r * K;
+    const RowInfo ri = row_info(P, row_begin + r);
+    const int n = visible_keys(ri);
+    if (n <= K) {   // select every visible key
+        for (int j = threadIdx.x; j < K; j += THREADS) out[j] = j < n ? j : -1;
+        return;
+    }
+    const float *src = scores + (int64_t)r * ld;
+    if (!select_row_sampled(src, n, K, smem, out)) select_row_general(src, n, K, smem, out);
 }
 
 }  // namespace topk

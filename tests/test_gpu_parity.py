@@ -72,6 +72,33 @@ def test_topk_long_rows_from_global_memory_and_ragged_batch():
     np.testing.assert_array_equal(sorted_rows(idx.cpu().numpy()), sorted_rows(ref))
 
 
+@pytest.mark.parametrize("pattern", ["constant", "increasing", "two_values", "spike"])
+def test_topk_adversarial_rows_take_every_path(pattern):
+    # Rows built so that the sampled fast path is exact (spike), or must give up (all
+    # keys equal; all top keys clustered in one warp's range; two values) and the general
+    # path decides.  Either way the result must equal the oracle's.
+    L, k = 6000, 2048
+    rows = 8
+    base = torch.arange(L, dtype=torch.float32)
+    if pattern == "constant":
+        sc = torch.full((rows, L), 1.5)
+    elif pattern == "increasing":
+        sc = base.repeat(rows, 1) * 0.25
+    elif pattern == "two_values":
+        sc = (base.repeat(rows, 1) % 7 == 0).float() * 3.0 - 1.0
+    else:
+        sc = torch.randn(rows, L, generator=torch.Generator().manual_seed(3))
+        sc[:, 100] = 1e6
+    p = dsa.make_problem(1, L, L, L, L, k)
+    buf = _scores_buffer(rows, L, fill=0.0)
+    buf[:, :L] = sc.to(DEV)
+    idx = torch.empty((rows, k), dtype=torch.int32, device=DEV)
+    r0 = L - rows
+    dsa.dsa_topk(p, buf, idx, row_begin=r0, row_count=rows)
+    ref = oracle.topk(buf.cpu()[:, :L], k, rows=np.arange(r0, L), cu_q=[0, L], cu_k=[0, L])
+    np.testing.assert_array_equal(sorted_rows(idx.cpu().numpy()), sorted_rows(ref))
+
+
 def test_topk_row_subrange_and_empty_rows():
     L, k = 300, 32
     sc = _tie_heavy_scores(L, L, seed=9)
