@@ -284,6 +284,12 @@ __device__ __forceinline__ void cp_async_wait() {
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+// Arrives on the mbarrier once all of this thread's earlier cp.async copies have landed
+// (without raising the expected count: the barrier is initialised with one arrival per
+// signalling thread).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
 
 }  // namespace sm100
 }  // namespace dsa

@@ -5,26 +5,35 @@
 // tokens; MLA-based implementation in MQA mode (every 576-d latent row is shared by all
 // 128 query heads); value = first 512 dims; softmax scale 1/sqrt(192).
 //
-// One CTA per (query token, value half v).  Per block of 128 selected keys:
-//   S[h, key]  = q[h, :] . kv[key, :]        (M = 128 heads, N = 128 keys, K = 576)
-//   P          = exp2(S * scale * log2 e - m[h])   (online softmax, lazy rescale)
-//   O_v[h, :] += P[h, key] kv[key, 256 v : 256 v + 256]   (M = 128, N = 256, K = 128 keys)
-// Tensor memory (512 columns): O_v [0,256) fp32; q dims 0..255 as the A operand of
-// the first 16 QK k-steps [256,384) (bf16 pairs); S [384,512) fp32, overwritten in
-// place by P as bf16 pairs [384,448) -- the A operand of the PV product.
-// Shared memory: q dims 256..575 (5 swizzled 128-byte atoms, 80 KB) and a 9-slot ring,
-// one slot per 64-dim atom of the current block's 128 gathered latent rows (144 KB);
-// slot a always holds atom a, so the 4 atoms of this CTA's value half are 4
-// consecutive slots and serve directly as the MN-major B operand of the PV product.
-// Rows are gathered by three producer warps with 16-byte cp.async (each warp
-// instruction moves 4 rows x 128 bytes of one atom; the 128-byte swizzle is applied in
-// the shared-memory address).  Small TMA gathers were issue-bound here; the LSU path
-// keeps the gather off the critical path.  The selected indices are compacted on the
-// fly (invalid slots -- -1, future or out-of-range positions -- are skipped); the tail
-// of the last block is padded with a duplicate row and masked in the softmax.
+// One CTA per (query token, value half v).  The selected-index row is cut into blocks
+// of 128 slots; for block b:
+//   S_b[h, key] = q[h, :] . kv[key, :]                 (M = 128 heads, N = 128 keys, K = 576)
+//   P_b         = exp2(S_b * scale * log2 e - m[h])     (online softmax, lazy rescale)
+//   O_v[h, :]  += P_b[h, key] kv[key, 256 v : 256 v + 256]
+// A slot whose index is not a visible key (-1, a future position, out of range) is
+// gathered as key 0 of the sequence and masked out of the softmax.  Blocks past the last
+// visible slot are skipped, so the top-k output (visible slots first, -1 after) costs
+// ceil(k_eff / 128) blocks.
+// Tensor memory (512 columns): O_v [0,256) fp32 and two S/P buffers [256,384), [384,512):
+// S_b lands in buffer b & 1 and is overwritten in place by P_b (bf16 pairs), the A operand
+// of the PV product.  With two buffers the tensor core computes S_{b+1} while the softmax
+// warps turn S_b into P_b.
+// Shared memory: all of q (9 swizzled 64-dim atoms of 128 heads, 144 KB), so every QK MMA
+// reads both operands from shared memory (mixing tensor-memory and shared-memory A
+// operands into one accumulator runs at about half rate), and a 5-slot ring of 64-dim
+// atoms of gathered latent rows (16 KB each) fed in MMA issue order:
+//   QK_0, QK_1, PV_0, QK_2, PV_1, ..., QK_{n-1}, PV_{n-2}, PV_{n-1}
+// (QK: the 9 atoms of the block; PV: the 4 value atoms of the block, gathered again and
+// consumed as two N = 128 pairs; the lower atom of a pair sits in the lower ring slot).
+// Atoms are gathered with 16-byte cp.async (one warp instruction moves 128 bytes of 4
+// rows; the 128-byte swizzle is applied in the shared-memory address) from row numbers
+// held in registers, so the copies issue back to back; each lane signals the slot
+// asynchronously when its copies land (cp.async mbarrier arrive).  One warp issues about
+// 20 bytes per clock and three reach the SM's gather rate of about 57, so three loader
+// warps take the ring positions in turn.
 //
-// Warp roles (12 warps): 0 index compaction + gathers + q TMA, 1 MMA issuer, 2 TMEM
-// allocator then gathers, 3 gathers, 4-11 softmax/epilogue: warp w owns TMEM lane
+// Warp roles (12 warps): 0, 2, 3 gather (0 also issues the q TMA, 2 allocates tensor
+// memory), 1 issues the MMAs (one thread), 4-11 softmax/epilogue: warp w owns TMEM lane
 // quarter w % 4 (32 heads) and key/column half c = (w - 4) / 4.
 #pragma once
 
@@ -35,24 +44,117 @@ namespace dsa {
 namespace mla {
 
 struct TcCfg {
-    static constexpr int BK = 128;                  // keys per block
+    static constexpr int BK = 128;                  // index slots (keys) per block
     static constexpr int NATOM = 9;                 // 64-dim atoms per 576-d row
     static constexpr int ATOM_BYTES = BK * 128;     // one atom of a 128-row tile
-    static constexpr int QHI_ATOMS = 5;             // q dims 256..575 in shared memory
-    static constexpr int OFF_QHI = 0;
-    static constexpr int OFF_KV = QHI_ATOMS * ATOM_BYTES;            // 81920
-    static constexpr int OFF_RED = OFF_KV + NATOM * ATOM_BYTES;      // 229376
-    static constexpr int OFF_STAGE = OFF_RED + 2 * 128 * 4;          // row-max / sum exchange
-    static constexpr int STAGE_CAP = 256;                            // compacted indices
-    static constexpr int OFF_BAR = OFF_STAGE + STAGE_CAP * 4;
-    static constexpr int NBARS = 2 * NATOM + 5;
+    static constexpr int NSLOT = 5;                 // gather ring slots
+    static constexpr int NLOAD = 3;                 // loader warps, taking ring positions in turn
+    // A loader waiting for position p - NSLOT to be consumed has itself seen position
+    // p - NLOAD's slot freed, i.e. p - NLOAD - NSLOT consumed; with NLOAD <= NSLOT that
+    // covers p - 2 NSLOT, so the parity wait cannot alias an older phase.
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_RING = NATOM * ATOM_BYTES;                  // 147456
+    static constexpr int OFF_RED = OFF_RING + NSLOT * ATOM_BYTES;         // [2][128] floats
+    static constexpr int OFF_BAR = OFF_RED + 2 * 128 * 4;
+    // ring_full[5], ring_empty[5], q_full, s_full[2], p_full[2], pv_done, o_ready
+    static constexpr int NBARS = 2 * NSLOT + 1 + 2 + 2 + 1 + 1;
     static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
     static constexpr int SMEM = OFF_MISC + 16;
     static constexpr int THREADS = 384;
-    static constexpr int TMEM_O = 0, TMEM_QLO = 256, TMEM_S = 384;
+    static constexpr int TMEM_O = 0, TMEM_S = 256;
     static constexpr float TAU = 8.0f;              // lazy-rescale threshold (log2 units)
     static_assert(SMEM <= 232448, "shared memory budget");
+    static_assert(NLOAD <= NSLOT, "ring waits need NLOAD <= NSLOT");
 };
+
+// Value atom at offset m (0..3) of a PV group starting at ring position pv_start: pair
+// (m >> 1) holds atoms 4v + 2*pair + {0,1}; the lower atom goes to the lower-addressed
+// ring slot so that the pair is one MN-major operand with a positive atom stride.
+__device__ __forceinline__ int pv_atom(int v, int pv_start, int m) {
+    const int pp = pv_start + (m & ~1);
+    const bool lo_first = (pp % TcCfg::NSLOT) < ((pp + 1) % TcCfg::NSLOT);
+    const int e = m & 1;
+    return 4 * v + 2 * (m >> 1) + (lo_first ? e : 1 - e);
+}
+
+// Group g (0 .. 2n-1) of the ring order QK_0, QK_1, PV_0, QK_2, PV_1, ..., PV_{n-1}:
+// whether it is a QK group, and its block.
+__device__ __forceinline__ void ring_group(int g, int n, bool &qk, int &blk) {
+    if (g == 0) { qk = true; blk = 0; }
+    else if (g == 2 * n - 1) { qk = false; blk = n - 1; }
+    else if (g & 1) { qk = true; blk = (g + 1) >> 1; }
+    else { qk = false; blk = (g >> 1) - 1; }
+}
+
+__device__ __forceinline__ bool visible(int e, const RowInfo &ri) { return e >= 0 && e <= ri.pos && e < ri.len_k; }
+
+// One loader warp's part of the ring: the positions p with p % NLOAD == lw, each a whole
+// atom (32 copy instructions; instruction i moves 128 bytes of rows i, 32+i, 64+i, 96+i:
+// lane l copies 16-byte chunk l % 8 of row 32 (l / 8) + i).  Returns false if a wait gave
+// up or another role aborted.
+__device__ __forceinline__ bool gather_turns(int lw, const int32_t *irow, int K, const RowInfo &ri,
+                                             const char *kv_bytes, uint32_t ring_s, uint32_t bar0, int v, int nblocks,
+                                             volatile uint32_t *misc, int lane) {
+    using C = TcCfg;
+    using namespace sm100;
+    const int ch = lane & 7;
+    const int r0 = (lane >> 3) * 32;                         // this lane's rows: r0 + i, i < 32
+    const bool vec4 = (K & 3) == 0;
+    // index entries of block j for this lane's rows
+    auto fetch = [&](int j, int (&e)[32]) {
+        const int s0 = j * C::BK + r0;
+        if (vec4 && s0 + 31 < K) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int4 x = __ldg(reinterpret_cast<const int4 *>(irow + s0) + i);
+                e[4 * i] = x.x; e[4 * i + 1] = x.y; e[4 * i + 2] = x.z; e[4 * i + 3] = x.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) e[i] = s0 + i < K ? __ldg(irow + s0 + i) : -1;
+        }
+    };
+    // raw: entries of the next QK block (prefetched); rows: row numbers of the current
+    // group's block (a PV group re-reads its block's entries, by then in L1)
+    int raw[32], rows[32];
+    if (nblocks > 0) fetch(0, raw);
+    int p = 0;                                               // ring position of the group's first atom
+    for (int g = 0; g < 2 * nblocks; ++g) {
+        bool qk;
+        int blk;
+        ring_group(g, nblocks, qk, blk);
+        if (qk) {                                            // rows of block blk; prefetch blk + 1
+#pragma unroll
+            for (int i = 0; i < 32; ++i) rows[i] = ri.kbase + (visible(raw[i], ri) ? raw[i] : 0);
+            if (blk + 1 < nblocks) fetch(blk + 1, raw);
+        } else {
+            fetch(blk, rows);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) rows[i] = ri.kbase + (visible(rows[i], ri) ? rows[i] : 0);
+        }
+        const int natoms = qk ? C::NATOM : 4;
+        for (int m = 0; m < natoms; ++m) {
+            const int pp = p + m;
+            if (pp % C::NLOAD != lw) continue;
+            const int a = qk ? m : pv_atom(v, p, m);
+            const int slot_i = pp % C::NSLOT;
+            bool okw = true;
+            if (lane == 0 && pp >= C::NSLOT)
+                okw = mbar_wait(bar0 + 8u * (C::NSLOT + slot_i), ((pp / C::NSLOT) - 1) & 1);
+            if (!__shfl_sync(0xffffffffu, okw, 0) || misc[1]) return false;
+            const uint32_t slot = ring_s + slot_i * C::ATOM_BYTES;
+            const char *src = kv_bytes + a * 128 + ch * 16;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int r = r0 + i;
+                cp_async16(slot + r * 128 + ((ch ^ (r & 7)) << 4), src + (int64_t)rows[i] * 1152);
+            }
+            cp_async_arrive_noinc(bar0 + 8u * slot_i);        // ring_full: fires when this lane's copies land
+        }
+        p += natoms;
+    }
+    return true;
+}
 
 __global__ void __launch_bounds__(384, 1)
 sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, Problem P, const __nv_bfloat16 *__restrict__ q,
@@ -67,231 +169,137 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, Problem P, const 
     const int v = (int)(blockIdx.x & 1);                     // value half
     const int K = P.topk;
     const RowInfo ri = row_info(P, t);
+    const int32_t *irow = idx + (int64_t)t * K;
+    const bool vec4 = (K & 3) == 0;                          // rows of idx are 16-byte aligned
 
     const uint32_t sbase = smem_u32(smem);
     if (sbase & 1023u) {
         if (tid == 0) raise_error(ERR_SMEM_ALIGN);
         return;
     }
-    const uint32_t qhi_s = sbase + C::OFF_QHI;
-    const uint32_t kv_s = sbase + C::OFF_KV;
-    float *red = reinterpret_cast<float *>(smem + C::OFF_RED);      // [2 halves][128]
-    int *stage = reinterpret_cast<int *>(smem + C::OFF_STAGE);
+    const uint32_t q_s = sbase + C::OFF_Q;
+    const uint32_t ring_s = sbase + C::OFF_RING;
+    float *red = reinterpret_cast<float *>(smem + C::OFF_RED);       // [2 halves][128]
     const uint32_t bar0 = sbase + C::OFF_BAR;
-    auto kv_full = [&](int a) { return bar0 + 8u * a; };
-    auto kv_empty = [&](int a) { return bar0 + 8u * (C::NATOM + a); };
-    const uint32_t q_full = bar0 + 8u * (2 * C::NATOM);
-    const uint32_t qlo_ready = q_full + 8;
-    const uint32_t s_full = q_full + 16;
-    const uint32_t p_full = q_full + 24;
-    const uint32_t pv_done = q_full + 32;
-    volatile uint32_t *misc = reinterpret_cast<volatile uint32_t *>(smem + C::OFF_MISC);  // tmem, nvalid, abort
+    auto ring_full = [&](int s) { return bar0 + 8u * s; };
+    auto ring_empty = [&](int s) { return bar0 + 8u * (C::NSLOT + s); };
+    const uint32_t q_full = bar0 + 8u * (2 * C::NSLOT);
+    auto s_full = [&](int b) { return q_full + 8u * (1 + b); };
+    auto p_full = [&](int b) { return q_full + 8u * (3 + b); };
+    const uint32_t pv_done = q_full + 40;
+    // o_ready completes once, after the last PV: pv_done may still have two phases in
+    // flight when the epilogue starts, so its parity alone cannot tell them apart
+    const uint32_t o_ready = q_full + 48;
+    volatile uint32_t *misc = reinterpret_cast<volatile uint32_t *>(smem + C::OFF_MISC);  // tmem, abort
 
     // ---- setup
     if (tid == 0) {
-        for (int a = 0; a < C::NATOM; ++a) {
-            mbar_init(kv_full(a), 32);   // one arrival per lane of the producing warp
-            mbar_init(kv_empty(a), 1);
+        for (int s = 0; s < C::NSLOT; ++s) {
+            mbar_init(ring_full(s), 32);   // every lane of the loading warp arrives
+            mbar_init(ring_empty(s), 1);
         }
         mbar_init(q_full, 1);
-        mbar_init(qlo_ready, 8);
-        mbar_init(s_full, 1);
-        mbar_init(p_full, 8);
+        mbar_init(s_full(0), 1);
+        mbar_init(s_full(1), 1);
+        mbar_init(p_full(0), 8);
+        mbar_init(p_full(1), 8);
         mbar_init(pv_done, 1);
-        misc[2] = 0;
+        mbar_init(o_ready, 1);
+        misc[1] = 0;
         fence_barrier_init();
     }
     if (warp == 2) tmem_alloc(sbase + C::OFF_MISC, 512);
-    if (warp == 0 || warp == 3) {   // number of valid selected indices of this row (2 warps)
-        int cnt = 0;
-        const int32_t *irow = idx + (int64_t)t * K;
+    if (warp == 0 || warp == 3) {   // last visible slot of this row (2 warps, halves of the row)
+        int last = -1;
         const int half = (warp == 0) ? 0 : 1;
-        if ((K & 3) == 0) {
-            // 16-byte loads, all issued before use
+        if (vec4) {
             const int n4 = K >> 2;
 #pragma unroll 4
             for (int i4 = half * 32 + lane; i4 < n4; i4 += 64) {
                 const int4 x = __ldg(reinterpret_cast<const int4 *>(irow) + i4);
-                cnt += (x.x >= 0 && x.x <= ri.pos && x.x < ri.len_k) + (x.y >= 0 && x.y <= ri.pos && x.y < ri.len_k) +
-                       (x.z >= 0 && x.z <= ri.pos && x.z < ri.len_k) + (x.w >= 0 && x.w <= ri.pos && x.w < ri.len_k);
+                if (visible(x.x, ri)) last = 4 * i4;
+                if (visible(x.y, ri)) last = 4 * i4 + 1;
+                if (visible(x.z, ri)) last = 4 * i4 + 2;
+                if (visible(x.w, ri)) last = 4 * i4 + 3;
             }
         } else {
-            for (int i = half * 32 + lane; i < K; i += 64) {
-                const int s = __ldg(irow + i);
-                cnt += s >= 0 && s <= ri.pos && s < ri.len_k;
-            }
+            for (int i = half * 32 + lane; i < K; i += 64)
+                if (visible(__ldg(irow + i), ri)) last = i;
         }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-        if (lane == 0) red[half] = (float)cnt;   // exact for counts <= 2^24
+        for (int o = 16; o > 0; o >>= 1) last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
+        if (lane == 0) reinterpret_cast<int *>(red)[half] = last;
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = misc[0];
-    const int nvalid = (int)red[0] + (int)red[1];
+    const int last_slot = max(reinterpret_cast<int *>(red)[0], reinterpret_cast<int *>(red)[1]);
+    const int nblocks = (last_slot + C::BK) / C::BK;         // 0 when no slot is visible
     __syncthreads();   // red is reused by the softmax warps
-    const int nblocks = (nvalid + C::BK - 1) / C::BK;
-    // QK atom order: the 5 atoms outside this CTA's value half first, then its 4 value atoms
-    auto atom_of = [&](int ai) { return ai < 5 ? (ai + 4 * (1 - v) + (ai >= 4 ? 4 * v : 0)) % 9 : ai - 5 + 4 * v; };
 
     if (warp == 0 || warp == 2 || warp == 3) {
-        // ------------------------------------------------ index compaction, gathers, q TMA
-        const int pw = warp == 0 ? 0 : warp - 1;            // producer 0, 1, 2
+        // ------------------------------------------------ gather loaders (+ q TMA)
+        const int lw = warp == 0 ? 0 : warp - 1;             // ring positions p with p % 3 == lw
         if (warp == 0 && lane == 0 && nblocks > 0) {
             prefetch_tmap(&tm_q);
-            mbar_expect_tx(q_full, C::QHI_ATOMS * C::ATOM_BYTES);
-            for (int a = 0; a < C::QHI_ATOMS; ++a)
-                tma_load_2d(qhi_s + a * C::ATOM_BYTES, &tm_q, q_full, 256 + 64 * a, t * 128);
+            mbar_expect_tx(q_full, C::NATOM * C::ATOM_BYTES);
+            for (int a = 0; a < C::NATOM; ++a) tma_load_2d(q_s + a * C::ATOM_BYTES, &tm_q, q_full, 64 * a, t * 128);
         }
-        const int32_t *irow = idx + (int64_t)t * K;
-        const bool vec4 = (K & 3) == 0;                      // rows of idx are 16-byte aligned
-        auto load_chunk = [&](int rd, int (&e)[4]) {         // entries rd + 4*lane .. +3
-            const int i = rd + 4 * lane;
-            if (vec4 && i + 3 < K) {
-                const int4 x = __ldg(reinterpret_cast<const int4 *>(irow + i));
-                e[0] = x.x; e[1] = x.y; e[2] = x.z; e[3] = x.w;
-            } else {
-#pragma unroll
-                for (int u = 0; u < 4; ++u) e[u] = i + u < K ? __ldg(irow + i + u) : -1;
-            }
-        };
-        int rd = 0, cnt = 0;
-        int nxt[4] = {-1, -1, -1, -1};
-        if (warp == 0 && nblocks > 0) load_chunk(0, nxt);
         const char *kv_bytes = reinterpret_cast<const char *>(kv);
         bool ok_run = true;
-        for (int j = 0; j < nblocks; ++j) {
-            // the three producer warps leave together when any of them gave up
-            if (named_bar_or(2, 96, !ok_run || misc[2] != 0)) { ok_run = false; break; }
-            if (warp == 0) {
-                while (cnt < C::BK && rd < K) {
-                    int cur[4] = {nxt[0], nxt[1], nxt[2], nxt[3]};
-                    rd += 128;
-                    if (rd < K) load_chunk(rd, nxt);            // prefetch the next chunk
-                    int vc = 0;
-                    bool okv[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        okv[u] = cur[u] >= 0 && cur[u] <= ri.pos && cur[u] < ri.len_k;
-                        vc += okv[u];
-                    }
-                    int incl = vc;                            // in-warp prefix of valid entries
-#pragma unroll
-                    for (int o = 1; o < 32; o <<= 1) {
-                        const int x = __shfl_up_sync(0xffffffffu, incl, o);
-                        if (lane >= o) incl += x;
-                    }
-                    const int tot = __shfl_sync(0xffffffffu, incl, 31);
-                    int off = cnt + incl - vc;
-#pragma unroll
-                    for (int u = 0; u < 4; ++u)
-                        if (okv[u]) stage[off++] = ri.kbase + cur[u];
-                    cnt += tot;
-                }
-                if (lane == 0) misc[3] = (uint32_t)min(cnt, C::BK);
-            }
-            named_bar(2, 96);                                 // stage holds this block's rows
-            const int nb = (int)misc[3];
-            const int base_row = stage[0];
-            int rows[32];
-#pragma unroll
-            for (int g = 0; g < 32; ++g) {
-                const int k = 4 * g + (lane >> 3);
-                rows[g] = k < nb ? stage[k] : base_row;
-            }
-            named_bar(2, 96);                                 // all rows read: stage may be rewritten
-            if (warp == 0) {                                  // keep the entries beyond this block
-                const int left = cnt - nb;                    // < 128
-                int keep[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) keep[u] = lane + 32 * u < left ? stage[C::BK + lane + 32 * u] : 0;
-                __syncwarp();
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    if (lane + 32 * u < left) stage[lane + 32 * u] = keep[u];
-                __syncwarp();
-                cnt = left;
-            }
-            // phase 1: atoms outside this CTA's value half (free once QK of the previous
-            // block consumed them); phase 2: the value atoms (free after the previous PV)
-            for (int phase = 0; phase < 2 && ok_run; ++phase) {
-                // this warp's atoms in QK order: ai = first + pw, first + pw + 3 (when in range)
-                const int first = phase == 0 ? 0 : 5, last = phase == 0 ? 5 : 9;
-                const int nmine = (first + pw < last) + (first + pw + 3 < last);
-                for (int q = 0; q < nmine; ++q) {
-                    const int a = atom_of(first + pw + 3 * q);
-                    if (j > 0) {
-                        bool okw = true;
-                        if (lane == 0) okw = mbar_wait(kv_empty(a), (j - 1) & 1);
-                        okw = __shfl_sync(0xffffffffu, okw, 0);
-                        if (!okw || misc[2]) { misc[2] = 1; ok_run = false; break; }
-                    }
-                    const uint32_t slot = kv_s + a * C::ATOM_BYTES;
-                    const int ch = lane & 7;
-#pragma unroll
-                    for (int g = 0; g < 32; ++g) {
-                        const int r = 4 * g + (lane >> 3);
-                        cp_async16(slot + r * 128 + ((ch ^ (r & 7)) << 4),
-                                   kv_bytes + (int64_t)rows[g] * 1152 + a * 128 + ch * 16);
-                    }
-                    cp_async_commit();
-                }
-                if (!ok_run) break;
-                // signal each atom once its copies have landed
-                if (nmine == 2) {
-                    cp_async_wait<1>();
-                    fence_proxy_async_smem();
-                    mbar_arrive(kv_full(atom_of(first + pw)));
-                }
-                if (nmine >= 1) {
-                    cp_async_wait<0>();
-                    fence_proxy_async_smem();
-                    mbar_arrive(kv_full(atom_of(first + pw + 3 * (nmine - 1))));
-                }
-            }
-        }
-        // drain: the MMA commits on the value atoms of the last block must land before exit
-        if (warp == 0 && lane == 0 && ok_run && nblocks > 0)
-            for (int ai = 5; ai < C::NATOM; ++ai)
-                if (!mbar_wait(kv_empty(atom_of(ai)), (nblocks - 1) & 1)) { misc[2] = 1; break; }
+        ok_run = gather_turns(lw, irow, K, ri, kv_bytes, ring_s, bar0, v, nblocks, misc, lane);
+        if (!ok_run) misc[1] = 1;
+        cp_async_wait<0>();
     } else if (warp == 1 && lane == 0 && nblocks > 0) {
         // ------------------------------------------------ MMA issuer
         const uint32_t idesc_qk = idesc_bf16(128, C::BK);
-        const uint32_t idesc_pv = idesc_bf16_bmn(128, 256);
-        bool ok = mbar_wait(q_full, 0) && mbar_wait(qlo_ready, 0);
-        tc_fence_after();
-        for (int j = 0; ok && j < nblocks; ++j) {
-            for (int ai = 0; ai < C::NATOM; ++ai) {
-                const int a = atom_of(ai);
-                // shared-memory operands only: the mbarrier (after the producers' proxy fence)
-                // orders them; no tcgen05 fence is needed here
-                if (!mbar_wait(kv_full(a), j & 1)) { ok = false; break; }
+        const uint32_t idesc_pv = idesc_bf16_bmn(128, 128);
+        bool ok = mbar_wait(q_full, 0);
+        int pos = 0;
+        for (int g = 0; ok && g < 2 * nblocks; ++g) {
+            bool qk;
+            int b;
+            ring_group(g, nblocks, qk, b);
+            if (qk) {                                        // QK_b -> S buffer b & 1
+                const uint32_t d = tmem + C::TMEM_S + 128 * (b & 1);
+                for (int a = 0; a < C::NATOM; ++a, ++pos) {
+                    if (!mbar_wait(ring_full(pos % C::NSLOT), (pos / C::NSLOT) & 1)) { ok = false; break; }
+                    fence_proxy_async_smem();
+                    const uint32_t slot = ring_s + (pos % C::NSLOT) * C::ATOM_BYTES;
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t bdesc = desc_sw128(kv_s + a * C::ATOM_BYTES + kk * 32);
-                    const uint32_t acc = (ai > 0 || kk > 0) ? 1u : 0u;
-                    if (a < 4)
-                        mma_f16_ts(tmem + C::TMEM_S, tmem + C::TMEM_QLO + a * 32 + kk * 8, bdesc, idesc_qk, acc);
-                    else
-                        mma_f16(tmem + C::TMEM_S, desc_sw128(qhi_s + (a - 4) * C::ATOM_BYTES + kk * 32), bdesc,
-                                idesc_qk, acc);
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_f16(d, desc_sw128(q_s + a * C::ATOM_BYTES + kk * 32), desc_sw128(slot + kk * 32), idesc_qk,
+                                (a > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(ring_empty(pos % C::NSLOT));
                 }
-                if (ai < 5) mma_commit(kv_empty(a));
-            }
-            if (!ok) break;
-            mma_commit(s_full);
-            if (!mbar_wait(p_full, j & 1)) { ok = false; break; }
-            tc_fence_after();
-            const uint32_t vbase = kv_s + 4 * v * C::ATOM_BYTES;
+                if (!ok) break;
+                mma_commit(s_full(b & 1));
+            } else {                                         // PV_b
+                if (!mbar_wait(p_full(b & 1), (b >> 1) & 1)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t pa = tmem + C::TMEM_S + 128 * (b & 1);   // P_b as bf16 pairs
+                for (int pair = 0; pair < 2; ++pair, pos += 2) {
+                    if (!mbar_wait(ring_full(pos % C::NSLOT), (pos / C::NSLOT) & 1) ||
+                        !mbar_wait(ring_full((pos + 1) % C::NSLOT), ((pos + 1) / C::NSLOT) & 1)) { ok = false; break; }
+                    fence_proxy_async_smem();
+                    const int s0 = pos % C::NSLOT, s1 = (pos + 1) % C::NSLOT;
+                    const int slo = s0 < s1 ? s0 : s1, shi = s0 < s1 ? s1 : s0;
+                    const uint32_t vb = ring_s + slo * C::ATOM_BYTES;
+                    const uint32_t lbo = (uint32_t)(shi - slo) * C::ATOM_BYTES;
 #pragma unroll
-            for (int kk = 0; kk < C::BK / 16; ++kk)
-                mma_f16_ts(tmem + C::TMEM_O, tmem + C::TMEM_S + kk * 8, desc_sw128_mn(vbase + kk * 2048, C::ATOM_BYTES),
-                           idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-            for (int ai = 5; ai < C::NATOM; ++ai) mma_commit(kv_empty(atom_of(ai)));
-            mma_commit(pv_done);
+                    for (int kk = 0; kk < C::BK / 16; ++kk)
+                        mma_f16_ts(tmem + C::TMEM_O + 128 * pair, pa + kk * 8, desc_sw128_mn(vb + kk * 2048, lbo),
+                                   idesc_pv, (b > 0 || kk > 0) ? 1u : 0u);
+                    mma_commit(ring_empty(s0));
+                    mma_commit(ring_empty(s1));
+                }
+                if (!ok) break;
+                mma_commit(pv_done);
+                if (b == nblocks - 1) mma_commit(o_ready);
+            }
         }
-        if (!ok) misc[2] = 1;
+        if (!ok) misc[1] = 1;
     } else if (warp >= 4) {
         // ------------------------------------------------ softmax + epilogue
         const int quarter = warp & 3;
@@ -299,44 +307,37 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, Problem P, const 
         const int h = quarter * 32 + lane;              // head (TMEM lane)
         const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
         const float sl2 = P.sm_scale * 1.4426950408889634f;   // scale * log2(e)
-        if (nblocks > 0) {
-            // q dims [128c, 128c+128) of head h -> TMEM A operand columns
-            const uint4 *qsrc = reinterpret_cast<const uint4 *>(q + ((int64_t)t * 128 + h) * 576 + 128 * c);
-            uint32_t regs[32];
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const uint4 x = __ldg(qsrc + half * 8 + i);
-                    regs[4 * i + 0] = x.x;
-                    regs[4 * i + 1] = x.y;
-                    regs[4 * i + 2] = x.z;
-                    regs[4 * i + 3] = x.w;
-                }
-                tmem_st32(t_lane + C::TMEM_QLO + 64 * c + 32 * half, regs);
-            }
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(qlo_ready);
-        }
         float m_run = -INFINITY, l_part = 0.f;
         bool ok = true;
-        for (int j = 0; j < nblocks; ++j) {
-            const bool fail = misc[2] != 0 || !mbar_wait(s_full, j & 1);
-            if (named_bar_or(1, 256, fail)) { ok = false; misc[2] = 1; break; }   // all 8 warps leave together
+        // index entries of this thread's key half of block b: slots 64c + lane (e[0]) and
+        // 64c + 32 + lane (e[1]), fetched a block ahead
+        auto fetch_mask = [&](int b, int (&e)[2]) {
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int s = b * C::BK + 64 * c + 32 * u + lane;
+                e[u] = s < K ? __ldg(irow + s) : -1;
+            }
+        };
+        int ent[2] = {-1, -1};
+        if (nblocks > 0) fetch_mask(0, ent);
+        for (int b = 0; b < nblocks; ++b) {
+            // bit i of w0 / w1: key 64c + i / 64c + 32 + i of the block is visible
+            const unsigned w0 = __ballot_sync(0xffffffffu, visible(ent[0], ri));
+            const unsigned w1 = __ballot_sync(0xffffffffu, visible(ent[1], ri));
+            if (b + 1 < nblocks) fetch_mask(b + 1, ent);
+            const bool fail = misc[1] != 0 || !mbar_wait(s_full(b & 1), (b >> 1) & 1);
+            if (named_bar_or(1, 256, fail)) { ok = false; misc[1] = 1; break; }   // all 8 warps leave together
             tc_fence_after();
+            const uint32_t sb = t_lane + C::TMEM_S + 128 * (b & 1);
             uint32_t s0[32], s1[32];
-            tmem_ld32(t_lane + C::TMEM_S + 64 * c, s0);
-            tmem_ld32(t_lane + C::TMEM_S + 64 * c + 32, s1);
+            tmem_ld32(sb + 64 * c, s0);
+            tmem_ld32(sb + 64 * c + 32, s1);
             tmem_wait_ld();
-            const int nb = min(C::BK, nvalid - j * C::BK);
-            const int kbase_c = 64 * c;                  // first key of this thread's half
             float mx = -INFINITY;
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
-                if (kbase_c + i < nb) mx = fmaxf(mx, __uint_as_float(s0[i]));
-                if (kbase_c + 32 + i < nb) mx = fmaxf(mx, __uint_as_float(s1[i]));
+                if ((w0 >> i) & 1u) mx = fmaxf(mx, __uint_as_float(s0[i]));
+                if ((w1 >> i) & 1u) mx = fmaxf(mx, __uint_as_float(s1[i]));
             }
             // red is single-buffered: every thread passed this block's opening barrier
             // only after reading the previous block's values
@@ -346,46 +347,53 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, Problem P, const 
             // Lazy rescale: a row moves its reference max only when the block max exceeds it
             // by more than TAU.  The TMEM load/store is warp-collective, so the whole warp
             // takes that path when any of its rows needs it (factor 1 for the others).
+            // A block without a visible slot has m_blk = -inf and never moves it.
             const bool need = m_blk > m_run + C::TAU;
-            const float f = (need && j > 0) ? exp2f(m_run - m_blk) : 1.0f;
+            const float f = (need && m_run != -INFINITY) ? exp2f(m_run - m_blk) : 1.0f;
             if (need) m_run = m_blk;
-            if (j > 0 && __any_sync(0xffffffffu, need)) {   // previous PV is complete (s_full)
-                l_part *= f;
-#pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    uint32_t o[32];
-                    const uint32_t oa = t_lane + C::TMEM_O + 128 * c + 32 * ch;
-                    tmem_ld32(oa, o);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
-                    tmem_st32(oa, o);
-                }
-            }
             uint32_t pk[32];
             float ls = 0.f;
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const int k0 = kbase_c + 2 * i;
-                const float p0 = k0 < nb ? ex2_approx(fmaf(__uint_as_float(s0[2 * i]), sl2, -m_run)) : 0.f;
-                const float p1 = k0 + 1 < nb ? ex2_approx(fmaf(__uint_as_float(s0[2 * i + 1]), sl2, -m_run)) : 0.f;
+                const float p0 = (w0 >> (2 * i)) & 1u ? ex2_approx(fmaf(__uint_as_float(s0[2 * i]), sl2, -m_run)) : 0.f;
+                const float p1 = (w0 >> (2 * i + 1)) & 1u ? ex2_approx(fmaf(__uint_as_float(s0[2 * i + 1]), sl2, -m_run)) : 0.f;
                 ls += p0 + p1;
                 pk[i] = pack_bf16x2(p0, p1);
             }
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const int k0 = kbase_c + 32 + 2 * i;
-                const float p0 = k0 < nb ? ex2_approx(fmaf(__uint_as_float(s1[2 * i]), sl2, -m_run)) : 0.f;
-                const float p1 = k0 + 1 < nb ? ex2_approx(fmaf(__uint_as_float(s1[2 * i + 1]), sl2, -m_run)) : 0.f;
+                const float p0 = (w1 >> (2 * i)) & 1u ? ex2_approx(fmaf(__uint_as_float(s1[2 * i]), sl2, -m_run)) : 0.f;
+                const float p1 = (w1 >> (2 * i + 1)) & 1u ? ex2_approx(fmaf(__uint_as_float(s1[2 * i + 1]), sl2, -m_run)) : 0.f;
                 ls += p0 + p1;
                 pk[16 + i] = pack_bf16x2(p0, p1);
             }
+            tmem_st32(sb + 32 * c, pk);
+            if (b > 0 && __any_sync(0xffffffffu, need)) {
+                // Rescale O (done after storing P_b, when S_b is no longer live).  O must
+                // include PV_{b-1} first; QK_b was issued after PV_{b-2}, so pv_done has
+                // completed b-1 or b phases here and the parity of phase b-1 is unambiguous.
+                // PV_b cannot start before this warp's p_full arrival below.
+                const bool okp = mbar_wait(pv_done, (b - 1) & 1);
+                tc_fence_after();
+                l_part *= f;
+                if (__all_sync(0xffffffffu, okp)) {
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) {
+                        uint32_t o[32];
+                        const uint32_t oa = t_lane + C::TMEM_O + 128 * c + 32 * ch;
+                        tmem_ld32(oa, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+                        tmem_st32(oa, o);
+                    }
+                }
+            }
             l_part += ls;
-            tmem_st32(t_lane + C::TMEM_S + 32 * c, pk);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(p_full);
+            if (lane == 0) mbar_arrive(p_full(b & 1));
         }
         // ---- epilogue
         const int64_t orow = ((int64_t)t * 128 + h) * 512 + 256 * v + 128 * c;
@@ -394,10 +402,10 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, Problem P, const 
             for (int i = 0; i < 16; ++i) reinterpret_cast<uint4 *>(out + orow)[i] = z;
             if (v == 0 && c == 0) lse[(int64_t)t * 128 + h] = nblocks == 0 ? -INFINITY : NAN;
         } else {
-            bool okw = mbar_wait(pv_done, (nblocks - 1) & 1);
+            bool okw = mbar_wait(o_ready, 0);
             tc_fence_after();
             // the last block's max was read before its p_full arrival, which the last PV
-            // (hence pv_done) waited for: red may be reused
+            // (hence o_ready) waited for: red may be reused
             red[c * 128 + h] = l_part;
             named_bar(1, 256);
             const float l = red[h] + red[128 + h];
