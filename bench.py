@@ -265,6 +265,8 @@ def run_ours(args, ws, rank, local, dist):
 
     if rank == 0 and not args.no_breakdown:
         res["roofline"], res["kernels"] = _breakdown(dsa, p, inp, fa, chunk, dev, stream, flush)
+    if args.workload != "decode_b64" and not args.no_decode:
+        res["decode"] = _decode_secondary(dsa, args, rank, dev, stream, flush, dist)
     if not args.no_e2e:
         res["e2e"] = _e2e(dsa, p, inp, fa, chunk, dev, stream, args, ws, dist)
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -273,7 +275,47 @@ def run_ours(args, ws, rank, local, dist):
         print(json.dumps(res), flush=True)
 
 
-def _breakdown(dsa, p, inp, fa, chunk, dev, stream, flush, reps=2):
+def _decode_secondary(dsa, args, rank, dev, stream, flush, dist):
+    """The metric's second half: decode microseconds per step (64 sequences, one query
+    each, contexts ~U[8192, 65536]), timed like the main step (events, L2 flushed between
+    steps, max over ranks)."""
+    inp = dsa_synth.make_workload("decode_b64", seed=args.seed, device=dev)
+    p = dsa.problem_from_inputs(inp)
+    fa = _forward_args(inp)
+    T = inp["total_q"]
+    out = torch.empty((T, 128, 512), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((T, 128), dtype=torch.float32, device=dev)
+    wsb = torch.empty(dsa.dsa_forward_workspace_size(p, 0), dtype=torch.uint8, device=dev)
+
+    def step():
+        dsa.dsa_forward(p, fa["q_idx"], fa["k_idx"], inp["w"], inp["q"], inp["kv"], out, lse, wsb, chunk_q=0,
+                        stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    n = max(args.steps, 10)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    _barrier(dist)
+    for i in range(n):
+        flush.zero_()
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize(dev)
+    _barrier(dist)
+    total_ms = _max_over_ranks(dist, sum(s.elapsed_time(e) for s, e in zip(starts, ends)))
+    dsa.dsa_check_device_errors()
+    res = {"workload": "decode_b64", "us_per_step": total_ms / n * 1e3, "steps": n, "batch": inp["batch"],
+           "mean_context": float(inp["total_k"]) / inp["batch"], "gpu_launches_per_step": 3,
+           "higher_is_better": False}
+    if rank == 0 and not args.no_breakdown:
+        res["roofline"], res["kernels"] = _breakdown(dsa, p, inp, fa, 0, dev, stream, flush, decode=True)
+    return res
+
+
+def _breakdown(dsa, p, inp, fa, chunk, dev, stream, flush, reps=2, decode=False):
     """Average device time of each kernel of the step, timed with CUDA events on the launch stream."""
     T = inp["total_q"]
     chunk = chunk or T
@@ -320,12 +362,21 @@ def _breakdown(dsa, p, inp, fa, chunk, dev, stream, flush, reps=2):
         "sparse_mla": {"ms_per_launch": t_mla / n_mla, "launches_per_step": 1, "ms_per_step": t_mla / reps,
                        "tflops": mla_pairs * FLOP_PER_PAIR_MLA / (t_mla / reps) / 1e9, "peak_tflops": pk["bf16"]},
     }
+    # algorithmic HBM bytes of each kernel (decode is bandwidth-bound throughout)
+    T, k = inp["total_q"], inp["topk"]
+    eb = 1 if fp8 else 2
+    idx_bytes = (inp["total_k"] * 128 * eb + T * 64 * 128 * eb + T * 64 * 4 + 4 * idx_pairs
+                 + (4 * (T + inp["total_k"]) if fp8 else 0))
+    mla_bytes = mla_pairs * 1152 + T * 128 * (576 + 512) * 2 + T * 128 * 4 + T * k * 4
+    for name, nbytes in (("indexer", idx_bytes), ("sparse_mla", mla_bytes)):
+        kernels[name]["gbs"] = nbytes / (kernels[name]["ms_per_step"]) / 1e6
+        kernels[name]["peak_gbs"] = pk["hbm_gbs"]
     dom = max(kernels, key=lambda k: kernels[k]["ms_per_step"])
     kd = kernels[dom]
-    src = {"indexer": "indexer.cuh", "topk": "topk.cuh", "sparse_mla": "sparse_mla.cuh"}[dom]
+    src = {"indexer": "indexer_tc.cuh", "topk": "topk.cuh", "sparse_mla": "sparse_mla_tc.cuh"}[dom]
     tr = TRAFFIC.get(dom)
     traffic = tr["bytes_per_launch"] if tr and tr.get("src_sha") == _src_sha(src) else None
-    if dom == "topk":
+    if dom == "topk" or decode:
         roof = {"bound": "hbm", "achieved": kd["gbs"], "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": kd["gbs"] / pk["hbm_gbs"], "traffic": traffic}
     else:
@@ -533,6 +584,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-breakdown", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode_b64 secondary measurement")
     ap.add_argument("--kernel", choices=("indexer", "topk", "sparse_mla"), default=None,
                     help="time one kernel on a bounded slice (for profilers) instead of the full step")
     ap.add_argument("--rows", type=int, default=0, help="query rows for --kernel (default: one chunk)")
