@@ -41,8 +41,13 @@ FLOP_PER_PAIR_MLA = 128 * (576 + 512) * 2       # per (query, selected key) pair
 
 # ncu DRAM traffic (read + write bytes per launch) of each kernel, recorded against the
 # sha256 of the source file it was captured from; reported only while the source is
-# unchanged.  Filled from the committed summaries under profiles/.
-TRAFFIC = {}
+# unchanged.
+TRAFFIC = {
+    # ncu capture of the 4096-query prefill launch: 1.141 GB of DRAM traffic (q reads and
+    # out writes, both proportional to the query count; kv rows come from L2), scaled x8 to
+    # the 32768-query launch of the 32K step
+    "sparse_mla": {"bytes_per_launch": 1.141e9 * 8, "src_sha": "ea7e3d9542033c36"},
+}
 
 
 def _peaks():
