@@ -5,7 +5,9 @@
 // Indexer-selected sparse attention: k_eff = min(index_topk, #candidates), int32 out.
 //
 // Scores map to order-preserving 32-bit keys (-0.0 folded onto +0.0), so comparing keys
-// as unsigned integers compares the floats as values.  One 256-thread CTA per row.
+// as unsigned integers compares the floats as values.  One CTA per row: 256 threads when
+// there are many rows (several CTAs share an SM), 512 when a launch has fewer rows than
+// SMs (decode), so a long row is not left to 8 warps.
 //
 // Fast path (one HBM read of the row):
 //   * every 16th float4 of the row is sampled; an exact radix select on the sample gives
@@ -27,20 +29,27 @@
 namespace dsa {
 namespace topk {
 
-constexpr int THREADS = 256;
-constexpr int WARPS = THREADS / 32;
 constexpr int BINS = 2048;        // 11-bit digits
-constexpr int SEG = 1024;         // candidate slots per warp (fast path)
-constexpr int CAND_CAP = WARPS * SEG * 2;   // general-path candidate indices (same bytes)
 constexpr unsigned FULL = 0xffffffffu;
 
-// Dynamic shared memory layout.
-constexpr int OFF_HIST = 0;                               // [BINS] u32
-constexpr int OFF_SEGK = OFF_HIST + BINS * 4;             // [WARPS][SEG] u32 keys (also: samples)
-constexpr int OFF_SEGI = OFF_SEGK + WARPS * SEG * 4;      // [WARPS][SEG] int indices
-constexpr int OFF_SCAL = OFF_SEGI + WARPS * SEG * 4;      // small scalars [64]
-constexpr int SMEM = OFF_SCAL + 64 * 4;
-static_assert(CAND_CAP * 4 == 2 * WARPS * SEG * 4, "general-path candidates reuse both segment arrays");
+template <int NT>
+struct Cfg {
+    static constexpr int THREADS = NT;
+    static constexpr int WARPS = NT / 32;
+    static constexpr int SEG = 8192 / WARPS;                  // candidate slots per warp (fast path)
+    static constexpr int CAND_CAP = WARPS * SEG * 2;          // general-path candidate indices (same bytes)
+    // Dynamic shared memory layout.
+    static constexpr int OFF_HIST = 0;                        // [BINS] u32
+    static constexpr int OFF_SEGK = OFF_HIST + BINS * 4;      // [WARPS][SEG] u32 keys (also: samples)
+    static constexpr int OFF_SEGI = OFF_SEGK + WARPS * SEG * 4;   // [WARPS][SEG] int indices
+    static constexpr int OFF_SCAL = OFF_SEGI + WARPS * SEG * 4;   // scalars, see below
+    // scal: [0..1] select_bin result, [2] candidate count, [3] overflow flag, then three
+    // per-warp arrays A = scal + 8, B = A + WARPS, C = B + WARPS
+    static constexpr int NSCAL = 8 + 3 * WARPS;
+    static constexpr int SMEM = OFF_SCAL + NSCAL * 4;
+    static_assert(CAND_CAP * 4 == 2 * WARPS * SEG * 4, "general-path candidates reuse both segment arrays");
+    static_assert(NT % 32 == 0 && 2048 % (NT / 32) == 0, "whole warps; select_bin splits 2048 bins over 32 lanes");
+};
 
 __device__ __forceinline__ uint32_t order_key(float f) {
     uint32_t u = __float_as_uint(f);
@@ -117,8 +126,9 @@ __device__ __forceinline__ void load4(const float *src, int i0, int we, uint32_t
 // Exact radix selection (11/11/10-bit digits, MSB first) of the `rank`-th largest key among
 // the keys get(j), j < m, for which valid(j) holds.  Returns the key; *above receives the
 // number of keys strictly greater.  All threads call it; uses hist and scal[0..1].
-template <class Get>
+template <class C, class Get>
 __device__ uint32_t radix_select(int m, int rank, Get get, uint32_t *hist, int *scal, int *above) {
+    constexpr int THREADS = C::THREADS;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     uint32_t prefix = 0, mask = 0;
     int remaining = rank, above_total = 0;
@@ -131,6 +141,41 @@ __device__ uint32_t radix_select(int m, int rank, Get get, uint32_t *hist, int *
         for (int j = tid; j < m_pad; j += THREADS) {
             uint32_t d = (uint32_t)BINS, key = 0;
             if (j < m && get(j, key) && (key & mask) == prefix) d = (key >> shift) & (uint32_t)(nb - 1);
+            hist_add(hist, d, lane);
+        }
+        __syncthreads();
+        if (warp == 0) select_bin(hist, nb, remaining, scal);
+        __syncthreads();
+        remaining -= scal[1];
+        above_total += scal[1];
+        prefix |= (uint32_t)scal[0] << shift;
+        mask |= (uint32_t)(nb - 1) << shift;
+        __syncthreads();
+    }
+    *above = above_total;
+    return prefix;
+}
+
+// The same selection when each warp holds its own items: warp w's items are get(j),
+// j < m_w (m_w differs per warp); every warp walks only its own items.
+template <class C, class Get>
+__device__ uint32_t radix_select_per_warp(int m_w, int rank, Get get, uint32_t *hist, int *scal, int *above) {
+    constexpr int THREADS = C::THREADS;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    uint32_t prefix = 0, mask = 0;
+    int remaining = rank, above_total = 0;
+    const int m_pad = (m_w + 31) & ~31;
+    for (int pass = 0; pass < 3; ++pass) {
+        const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+        const int nb = pass == 2 ? 1024 : 2048;
+        for (int i = tid; i < nb; i += THREADS) hist[i] = 0;
+        __syncthreads();
+        for (int j = lane; j < m_pad; j += 32) {
+            uint32_t d = (uint32_t)BINS;
+            if (j < m_w) {
+                const uint32_t key = get(j);
+                if ((key & mask) == prefix) d = (key >> shift) & (uint32_t)(nb - 1);
+            }
             hist_add(hist, d, lane);
         }
         __syncthreads();
@@ -182,12 +227,16 @@ __device__ __forceinline__ void ordered_output(const float *src, int wb, int we,
 }
 
 // Fast path.  Returns false (nothing written) when the sample misjudged the row.
+template <class C>
 __device__ bool select_row_sampled(const float *src, int n, int K, unsigned char *smem, int32_t *out) {
+    constexpr int THREADS = C::THREADS, WARPS = C::WARPS, SEG = C::SEG;
+    constexpr int OFF_HIST = C::OFF_HIST, OFF_SEGK = C::OFF_SEGK, OFF_SEGI = C::OFF_SEGI, OFF_SCAL = C::OFF_SCAL;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     uint32_t *hist = reinterpret_cast<uint32_t *>(smem + OFF_HIST);
     uint32_t *segk = reinterpret_cast<uint32_t *>(smem + OFF_SEGK);
     int *segi = reinterpret_cast<int *>(smem + OFF_SEGI);
-    int *scal = reinterpret_cast<int *>(smem + OFF_SCAL);   // [0..1] select, [8..15] seg counts, [16] flag
+    int *scal = reinterpret_cast<int *>(smem + OFF_SCAL);
+    int *seg_cnt = scal + 8, *wgt = scal + 8 + WARPS, *weq = scal + 8 + 2 * WARPS;
     const float4 *s4 = reinterpret_cast<const float4 *>(src);
     const int n4 = n >> 2;
     const int nsamp4 = (n4 + 15) / 16;                       // sampled float4 (every 16th)
@@ -202,12 +251,12 @@ __device__ bool select_row_sampled(const float *src, int n, int K, unsigned char
         segk[4 * m + 2] = order_key(v.z);
         segk[4 * m + 3] = order_key(v.w);
     }
-    if (tid < WARPS) scal[8 + tid] = 0;
-    if (tid == 0) scal[16] = 0;
+    if (tid < WARPS) seg_cnt[tid] = 0;
+    if (tid == 0) scal[3] = 0;
     __syncthreads();
     const int target = min(ns, (int)((1.2 * K * (double)ns) / (double)n) + 16);
     int dummy;
-    const uint32_t t_lo = radix_select(
+    const uint32_t t_lo = radix_select<C>(
         ns, target, [&](int j, uint32_t &key) { key = segk[j]; return true; }, hist, scal, &dummy);
     __syncthreads();   // samples no longer needed
 
@@ -241,24 +290,17 @@ __device__ bool select_row_sampled(const float *src, int n, int K, unsigned char
         cnt += tot;
     }
     if (lane == 0) {
-        scal[8 + warp] = overflow ? 0 : cnt;
-        if (overflow) scal[16] = 1;
+        seg_cnt[warp] = overflow ? 0 : cnt;
+        if (overflow) scal[3] = 1;
     }
     __syncthreads();
     int total = 0;
-    for (int w = 0; w < WARPS; ++w) total += scal[8 + w];
-    if (scal[16] != 0 || total < K) return false;   // uniform decision
+    for (int w = 0; w < WARPS; ++w) total += seg_cnt[w];
+    if (scal[3] != 0 || total < K) return false;   // uniform decision
 
     // ---- exact k-th largest among the candidates
     int above;
-    const uint32_t thr = radix_select(
-        WARPS * SEG, K,
-        [&](int j, uint32_t &key) {
-            if ((j & (SEG - 1)) >= scal[8 + j / SEG]) return false;
-            key = segk[j];
-            return true;
-        },
-        hist, scal, &above);
+    const uint32_t thr = radix_select_per_warp<C>(cnt, K, [&](int j) { return mk[j]; }, hist, scal, &above);
     const int need_eq = K - above;                   // >= 1
     const int count_gt = above;
 
@@ -272,14 +314,14 @@ __device__ bool select_row_sampled(const float *src, int n, int K, unsigned char
     ce = warp_sum(ce);
     __syncthreads();
     if (lane == 0) {
-        scal[24 + warp] = cg;
-        scal[32 + warp] = ce;
+        wgt[warp] = cg;
+        weq[warp] = ce;
     }
     __syncthreads();
     int gt_off = 0, eq_off = 0;
     for (int w2 = 0; w2 < warp; ++w2) {
-        gt_off += scal[24 + w2];
-        eq_off += scal[32 + w2];
+        gt_off += wgt[w2];
+        eq_off += weq[w2];
     }
     const unsigned lt = (1u << lane) - 1u;
     for (int base = 0; base < cnt; base += 32) {
@@ -302,11 +344,16 @@ __device__ bool select_row_sampled(const float *src, int n, int K, unsigned char
 }
 
 // General path: full radix selection over the row.
+template <class C>
 __device__ void select_row_general(const float *src, int n, int K, unsigned char *smem, int32_t *out) {
+    constexpr int THREADS = C::THREADS, WARPS = C::WARPS, CAND_CAP = C::CAND_CAP;
+    constexpr int OFF_HIST = C::OFF_HIST, OFF_SEGK = C::OFF_SEGK, OFF_SCAL = C::OFF_SCAL;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     uint32_t *hist = reinterpret_cast<uint32_t *>(smem + OFF_HIST);
     int *cand = reinterpret_cast<int *>(smem + OFF_SEGK);   // CAND_CAP entries over both segment arrays
-    int *scal = reinterpret_cast<int *>(smem + OFF_SCAL);   // [0..1] select, [2] ncand, [8..] warp counts
+    int *scal = reinterpret_cast<int *>(smem + OFF_SCAL);
+    // per warp: keys above bin b0, keys in b0 above thr, keys == thr
+    int *w_above = scal + 8, *w_gt = scal + 8 + WARPS, *w_eq = scal + 8 + 2 * WARPS;
     const float4 *s4 = reinterpret_cast<const float4 *>(src);
     const int n4 = n >> 2;
     const int R = ((n + WARPS * 128 - 1) / (WARPS * 128)) * 128;
@@ -314,7 +361,7 @@ __device__ void select_row_general(const float *src, int n, int K, unsigned char
 
     __syncthreads();
     for (int i = tid; i < BINS; i += THREADS) hist[i] = 0;
-    if (tid < 3 * WARPS) scal[8 + tid] = 0;
+    for (int i = tid; i < 3 * WARPS; i += THREADS) scal[8 + i] = 0;
     if (tid == 0) scal[2] = 0;
     __syncthreads();
 
@@ -366,7 +413,7 @@ __device__ void select_row_general(const float *src, int n, int K, unsigned char
             }
         }
         g0 = warp_sum(g0);
-        if (lane == 0) scal[8 + warp] = g0;
+        if (lane == 0) w_above[warp] = g0;
     }
     __syncthreads();
     const int ncand = scal[2];
@@ -406,8 +453,8 @@ __device__ void select_row_general(const float *src, int n, int K, unsigned char
         for (int j = tid; j < ncand; j += THREADS) {
             const int i = cand[j];
             const uint32_t key = order_key(__ldg(src + i));
-            if (key > thr) atomicAdd(&scal[16 + i / R], 1);
-            else if (key == thr) atomicAdd(&scal[24 + i / R], 1);
+            if (key > thr) atomicAdd(&w_gt[i / R], 1);
+            else if (key == thr) atomicAdd(&w_eq[i / R], 1);
         }
     } else {
         int cg = 0, ce = 0;
@@ -425,22 +472,24 @@ __device__ void select_row_general(const float *src, int n, int K, unsigned char
         cg = warp_sum(cg);
         ce = warp_sum(ce);
         if (lane == 0) {
-            scal[16 + warp] = cg;
-            scal[24 + warp] = ce;
+            w_gt[warp] = cg;
+            w_eq[warp] = ce;
         }
     }
     __syncthreads();
     int gt_off = 0, eq_off = 0;
     for (int w2 = 0; w2 < warp; ++w2) {
-        gt_off += scal[8 + w2] + scal[16 + w2];
-        eq_off += scal[24 + w2];
+        gt_off += w_above[w2] + w_gt[w2];
+        eq_off += w_eq[w2];
     }
     ordered_output(src, wb, we, lane, thr, need_eq, count_gt, K, gt_off, eq_off, out);
 }
 
-// grid = row_count CTAs of THREADS threads, dynamic shared memory SMEM bytes.
-__global__ void __launch_bounds__(THREADS) topk_rows_kernel(Problem P, const float *__restrict__ scores, int64_t ld,
-                                                            int row_begin, int32_t *__restrict__ idx) {
+// grid = row_count CTAs of NT threads, dynamic shared memory Cfg<NT>::SMEM bytes.
+template <int NT>
+__global__ void __launch_bounds__(NT, NT >= 512 ? 1 : 3) topk_rows_kernel(Problem P, const float *__restrict__ scores, int64_t ld,
+                                                       int row_begin, int32_t *__restrict__ idx) {
+    using C = Cfg<NT>;
     extern __shared__ __align__(16) unsigned char smem[];
     const int r = blockIdx.x;
     const int K = P.topk;
@@ -448,11 +497,11 @@ __global__ void __launch_bounds__(THREADS) topk_rows_kernel(Problem P, const flo
     const RowInfo ri = row_info(P, row_begin + r);
     const int n = visible_keys(ri);
     if (n <= K) {   // select every visible key
-        for (int j = threadIdx.x; j < K; j += THREADS) out[j] = j < n ? j : -1;
+        for (int j = threadIdx.x; j < K; j += NT) out[j] = j < n ? j : -1;
         return;
     }
     const float *src = scores + (int64_t)r * ld;
-    if (!select_row_sampled(src, n, K, smem, out)) select_row_general(src, n, K, smem, out);
+    if (!select_row_sampled<C>(src, n, K, smem, out)) select_row_general<C>(src, n, K, smem, out);
 }
 
 }  // namespace topk

@@ -72,13 +72,14 @@ def test_topk_long_rows_from_global_memory_and_ragged_batch():
     np.testing.assert_array_equal(sorted_rows(idx.cpu().numpy()), sorted_rows(ref))
 
 
+@pytest.mark.parametrize("rows", [8, 200])
 @pytest.mark.parametrize("pattern", ["constant", "increasing", "two_values", "spike"])
-def test_topk_adversarial_rows_take_every_path(pattern):
+def test_topk_adversarial_rows_take_every_path(pattern, rows):
     # Rows built so that the sampled fast path is exact (spike), or must give up (all
     # keys equal; all top keys clustered in one warp's range; two values) and the general
-    # path decides.  Either way the result must equal the oracle's.
+    # path decides.  Either way the result must equal the oracle's.  8 rows run with
+    # 512 threads per row (fewer rows than SMs), 200 rows with 256.
     L, k = 6000, 2048
-    rows = 8
     base = torch.arange(L, dtype=torch.float32)
     if pattern == "constant":
         sc = torch.full((rows, L), 1.5)
