@@ -115,17 +115,22 @@ def test_topk_row_subrange_and_empty_rows():
 
 # ----------------------------------------------------------------------- indexer
 
+def _host_rows(t, rows):
+    """Rows `rows` of a device tensor, gathered on the device and copied to the host (the
+    full-size inputs are tens of GB; only the sampled rows travel)."""
+    return t[torch.as_tensor(np.asarray(rows), device=t.device)].cpu()
+
+
 def _oracle_scores(inp, rows):
-    rows_t = torch.from_numpy(rows)
     cu_q = inp["cu_q"].cpu().numpy()
     cu_k = inp["cu_k"].cpu().numpy()
     if "q_idx8" in inp:
-        qr = inp["q_idx8"].cpu()[rows_t]
-        qs = inp["q_scale"].cpu()[rows_t]
-        ref = oracle.indexer_fp8(qr, qs, inp["w"].cpu()[rows_t], inp["k_idx8"].cpu(), inp["k_scale"].cpu(),
+        qr = _host_rows(inp["q_idx8"], rows)
+        qs = _host_rows(inp["q_scale"], rows)
+        ref = oracle.indexer_fp8(qr, qs, _host_rows(inp["w"], rows), inp["k_idx8"].cpu(), inp["k_scale"].cpu(),
                                  rows=rows, cu_q=cu_q, cu_k=cu_k, ld=inp["max_len_k"])
         return ref
-    return oracle.indexer(inp["q_idx"].cpu()[rows_t], inp["w"].cpu()[rows_t], inp["k_idx"].cpu(), rows=rows,
+    return oracle.indexer(_host_rows(inp["q_idx"], rows), _host_rows(inp["w"], rows), inp["k_idx"].cpu(), rows=rows,
                           cu_q=cu_q, cu_k=cu_k, ld=inp["max_len_k"])
 
 
@@ -134,20 +139,21 @@ def _bound_rows(inp, rows):
     pos = _positions(inp, rows)
     kb = _kbase(inp, rows)
     if "q_idx8" in inp:
-        q_all = inp["q_idx8"].cpu()
+        q_sel = _host_rows(inp["q_idx8"], rows)
+        qs_sel = _host_rows(inp["q_scale"], rows)
         k_all = fp8_to_f64(inp["k_idx8"].cpu()) * inp["k_scale"].cpu().double()[:, None]
     else:
-        q_all = inp["q_idx"].cpu()
+        q_sel = _host_rows(inp["q_idx"], rows)
         k_all = inp["k_idx"].cpu()
-    w_all = inp["w"].cpu()
+    w_sel = _host_rows(inp["w"], rows)
     out = []
     for i, t in enumerate(rows):
         if "q_idx8" in inp:
-            qr = fp8_to_f64(q_all[int(t)]) * float(inp["q_scale"][int(t)])
+            qr = fp8_to_f64(q_sel[i]) * float(qs_sel[i])
         else:
-            qr = q_all[int(t)]
+            qr = q_sel[i]
         n = int(pos[i]) + 1
-        out.append(score_bound_row(qr, w_all[int(t)], k_all[int(kb[i]):int(kb[i]) + n]))
+        out.append(score_bound_row(qr, w_sel[i], k_all[int(kb[i]):int(kb[i]) + n]))
     return out
 
 
@@ -277,14 +283,13 @@ def _check_forward_rows(inp, rows, chunk=0):
     pos = _positions(inp, rows)
     ref_sc = _oracle_scores(inp, rows)
     bound = _bound_rows(inp, rows)
-    gidx = idx.cpu().numpy()[rows]
+    gidx = _host_rows(idx, rows).numpy()
     recall, wrong = recall_excluding_near_ties(gidx, ref_sc, bound, pos, k)
     assert recall >= RECALL_MIN and wrong == 0, (recall, wrong)
-    rt = torch.from_numpy(rows)
-    o_ref, lse_ref = oracle.sparse_mla(inp["q"].cpu()[rt], inp["kv"].cpu(), gidx, SCALE, rows=rows,
+    o_ref, lse_ref = oracle.sparse_mla(_host_rows(inp["q"], rows), inp["kv"].cpu(), gidx, SCALE, rows=rows,
                                        cu_q=inp["cu_q"].cpu().numpy(), cu_k=inp["cu_k"].cpu().numpy())
-    assert np.max(np.abs(out.cpu()[rt].double().numpy() - o_ref)) <= O_ATOL
-    assert np.max(np.abs(lse.cpu()[rt].double().numpy() - lse_ref)) <= LSE_ATOL
+    assert np.max(np.abs(_host_rows(out, rows).double().numpy() - o_ref)) <= O_ATOL
+    assert np.max(np.abs(_host_rows(lse, rows).double().numpy() - lse_ref)) <= LSE_ATOL
     return idx, out, lse
 
 
@@ -325,6 +330,16 @@ def test_prefill_32k_full_size_sampled_bench_config():
     inp = dsa_synth.make_workload("prefill_32k", seed=0, device=DEV)
     rows = sample_rows(32768, 2048, n_rand=12, seed=2, edge=4)
     _check_forward_rows(inp, rows, chunk=dsa_synth.WORKLOADS["prefill_32k"].chunk)
+
+
+def test_prefill_128k_fp8_full_size_sampled_bench_config():
+    # 131072 tokens, FP8 indexer with per-token scales, 4096-query chunks (the bench's launch
+    # configuration); the oracle checks a handful of rows (each scores up to 128K keys)
+    inp = dsa_synth.make_workload("prefill_128k_fp8", seed=0, device=DEV)
+    rows = sample_rows(131072, 2048, n_rand=3, seed=4, edge=2)
+    _check_forward_rows(inp, rows, chunk=dsa_synth.WORKLOADS["prefill_128k_fp8"].chunk)
+    del inp
+    torch.cuda.empty_cache()
 
 
 def test_decode_b64_full_size_sampled():
