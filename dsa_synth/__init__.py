@@ -58,7 +58,7 @@ WORKLOADS: Dict[str, Workload] = {
     "pr_ref_256": Workload("pr_ref_256", "prefill", seq_len=256, topk=64, structured_keys=False,
                            latent_std=1.0 / 24.0),
     "prefill_4k": Workload("prefill_4k", "prefill", seq_len=4096),
-    "prefill_32k": Workload("prefill_32k", "prefill", seq_len=32768, chunk=4096),
+    "prefill_32k": Workload("prefill_32k", "prefill", seq_len=32768, chunk=8192),
     "decode_b64": Workload("decode_b64", "decode", batch=64, ctx_min=8192, ctx_max=65536),
     "prefill_128k_fp8": Workload("prefill_128k_fp8", "prefill", seq_len=131072, fp8_indexer=True,
                                  chunk=4096),
