@@ -92,42 +92,76 @@ __device__ __forceinline__ bool visible(int e, const RowInfo &ri) { return e >= 
 // atom (32 copy instructions; instruction i moves 128 bytes of rows i, 32+i, 64+i, 96+i:
 // lane l copies 16-byte chunk l % 8 of row 32 (l / 8) + i).  Returns false if a wait gave
 // up or another role aborted.
-__device__ __forceinline__ bool gather_turns(int lw, const int32_t *irow, int K, const RowInfo &ri,
-                                             const char *kv_bytes, uint32_t ring_s, uint32_t bar0, int v, int nblocks,
-                                             volatile uint32_t *misc, int lane) {
-    using C = TcCfg;
+// Index entries of block j for lane `lane`'s rows (32 (lane / 8) + i, i < 32); slots past
+// the end of the row read as -1.
+__device__ __forceinline__ void fetch_rows(const int32_t *irow, int K, int j, int lane, int (&e)[32]) {
+    const int s0 = j * TcCfg::BK + (lane >> 3) * 32;
+    if ((K & 3) == 0 && s0 + 31 < K) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int4 x = __ldg(reinterpret_cast<const int4 *>(irow + s0) + i);
+            e[4 * i] = x.x; e[4 * i + 1] = x.y; e[4 * i + 2] = x.z; e[4 * i + 3] = x.w;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) e[i] = s0 + i < K ? __ldg(irow + s0 + i) : -1;
+    }
+}
+
+// One atom's 32 copy instructions into a ring slot, then the lane's asynchronous arrival on
+// the slot's ring_full barrier.
+__device__ __forceinline__ void gather_atom(const char *kv_bytes, const int (&rows)[32], int a, uint32_t slot,
+                                            uint32_t full_bar, int lane) {
     using namespace sm100;
     const int ch = lane & 7;
-    const int r0 = (lane >> 3) * 32;                         // this lane's rows: r0 + i, i < 32
-    const bool vec4 = (K & 3) == 0;
+    const int r0 = (lane >> 3) * 32;
+    const char *src = kv_bytes + a * 128 + ch * 16;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const int r = r0 + i;
+        cp_async16(slot + r * 128 + ((ch ^ (r & 7)) << 4), src + (int64_t)rows[i] * 1152);
+    }
+    cp_async_arrive_noinc(full_bar);                         // fires when this lane's copies land
+}
+
+// Before the visible extent of the row is known: the first NSLOT atoms of QK_0 (ring
+// positions 0 .. NSLOT-1 need no slot wait), this warp's share of them.  `rows` keeps
+// block 0's row numbers for gather_turns.
+__device__ __forceinline__ void gather_first(int lw, const int32_t *irow, int K, const RowInfo &ri,
+                                             const char *kv_bytes, uint32_t ring_s, uint32_t bar0, int lane,
+                                             int (&rows)[32]) {
+    using C = TcCfg;
+    fetch_rows(irow, K, 0, lane, rows);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) rows[i] = ri.kbase + (visible(rows[i], ri) ? rows[i] : 0);
+    for (int pp = lw; pp < C::NSLOT; pp += C::NLOAD)
+        gather_atom(kv_bytes, rows, pp, ring_s + pp * C::ATOM_BYTES, bar0 + 8u * pp, lane);
+}
+
+__device__ __forceinline__ bool gather_turns(int lw, const int32_t *irow, int K, const RowInfo &ri,
+                                             const char *kv_bytes, uint32_t ring_s, uint32_t bar0, int v, int nblocks,
+                                             volatile uint32_t *misc, int lane, int (&rows)[32]) {
+    using C = TcCfg;
+    using namespace sm100;
+    static_assert(C::NSLOT <= C::NATOM, "the early positions all belong to QK_0");
     // index entries of block j for this lane's rows
     auto fetch = [&](int j, int (&e)[32]) {
-        const int s0 = j * C::BK + r0;
-        if (vec4 && s0 + 31 < K) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int4 x = __ldg(reinterpret_cast<const int4 *>(irow + s0) + i);
-                e[4 * i] = x.x; e[4 * i + 1] = x.y; e[4 * i + 2] = x.z; e[4 * i + 3] = x.w;
-            }
-        } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) e[i] = s0 + i < K ? __ldg(irow + s0 + i) : -1;
-        }
+        fetch_rows(irow, K, j, lane, e);
     };
     // raw: entries of the next QK block (prefetched); rows: row numbers of the current
-    // group's block (a PV group re-reads its block's entries, by then in L1)
-    int raw[32], rows[32];
-    if (nblocks > 0) fetch(0, raw);
+    // group's block (block 0's on entry; a PV group re-reads its block's entries, by then in L1)
+    int raw[32];
+    if (nblocks > 1) fetch(1, raw);
     int p = 0;                                               // ring position of the group's first atom
     for (int g = 0; g < 2 * nblocks; ++g) {
         bool qk;
         int blk;
         ring_group(g, nblocks, qk, blk);
-        if (qk) {                                            // rows of block blk; prefetch blk + 1
+        if (qk && blk > 0) {                                 // rows of block blk; prefetch blk + 1
 #pragma unroll
             for (int i = 0; i < 32; ++i) rows[i] = ri.kbase + (visible(raw[i], ri) ? raw[i] : 0);
             if (blk + 1 < nblocks) fetch(blk + 1, raw);
-        } else {
+        } else if (!qk) {
             fetch(blk, rows);
 #pragma unroll
             for (int i = 0; i < 32; ++i) rows[i] = ri.kbase + (visible(rows[i], ri) ? rows[i] : 0);
@@ -135,21 +169,13 @@ __device__ __forceinline__ bool gather_turns(int lw, const int32_t *irow, int K,
         const int natoms = qk ? C::NATOM : 4;
         for (int m = 0; m < natoms; ++m) {
             const int pp = p + m;
-            if (pp % C::NLOAD != lw) continue;
+            if (pp % C::NLOAD != lw || pp < C::NSLOT) continue;   // positions < NSLOT: gather_first
             const int a = qk ? m : pv_atom(v, p, m);
             const int slot_i = pp % C::NSLOT;
             bool okw = true;
-            if (lane == 0 && pp >= C::NSLOT)
-                okw = mbar_wait(bar0 + 8u * (C::NSLOT + slot_i), ((pp / C::NSLOT) - 1) & 1);
+            if (lane == 0) okw = mbar_wait(bar0 + 8u * (C::NSLOT + slot_i), ((pp / C::NSLOT) - 1) & 1);
             if (!__shfl_sync(0xffffffffu, okw, 0) || misc[1]) return false;
-            const uint32_t slot = ring_s + slot_i * C::ATOM_BYTES;
-            const char *src = kv_bytes + a * 128 + ch * 16;
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int r = r0 + i;
-                cp_async16(slot + r * 128 + ((ch ^ (r & 7)) << 4), src + (int64_t)rows[i] * 1152);
-            }
-            cp_async_arrive_noinc(bar0 + 8u * slot_i);        // ring_full: fires when this lane's copies land
+            gather_atom(kv_bytes, rows, a, ring_s + slot_i * C::ATOM_BYTES, bar0 + 8u * slot_i, lane);
         }
         p += natoms;
     }
@@ -207,15 +233,30 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, Problem P, const 
         mbar_init(o_ready, 1);
         misc[1] = 0;
         fence_barrier_init();
+        // q lands while the index row is scanned (waited for before exit even when the row
+        // has no visible slot)
+        prefetch_tmap(&tm_q);
+        mbar_expect_tx(q_full, C::NATOM * C::ATOM_BYTES);
+        for (int a = 0; a < C::NATOM; ++a) tma_load_2d(q_s + a * C::ATOM_BYTES, &tm_q, q_full, 64 * a, t * 128);
     }
     if (warp == 2) tmem_alloc(sbase + C::OFF_MISC, 512);
-    if (warp == 0 || warp == 3) {   // last visible slot of this row (2 warps, halves of the row)
+    const char *kv_bytes = reinterpret_cast<const char *>(kv);
+    const int lw = warp == 0 ? 0 : warp - 1;                 // loader warps 0, 2, 3: ring positions p % 3 == lw
+    int rows0[32];                                           // a loader's row numbers of block 0
+    if (warp == 0 || warp == 2 || warp == 3) {
+        // the first ring positions are gathered while the row is scanned: they hold atoms of
+        // block 0, which exists whenever any slot is visible (otherwise nothing consumes them)
+        __syncwarp();
+        named_bar(3, 96);                                    // the barriers are initialised
+        gather_first(lw, irow, K, ri, kv_bytes, ring_s, bar0, lane, rows0);
+    }
+    if (warp >= 4) {   // last visible slot of this row (8 warps, interleaved int4 groups)
         int last = -1;
-        const int half = (warp == 0) ? 0 : 1;
+        const int part = warp - 4;
         if (vec4) {
             const int n4 = K >> 2;
-#pragma unroll 4
-            for (int i4 = half * 32 + lane; i4 < n4; i4 += 64) {
+#pragma unroll 2
+            for (int i4 = part * 32 + lane; i4 < n4; i4 += 256) {
                 const int4 x = __ldg(reinterpret_cast<const int4 *>(irow) + i4);
                 if (visible(x.x, ri)) last = 4 * i4;
                 if (visible(x.y, ri)) last = 4 * i4 + 1;
@@ -223,34 +264,30 @@ sparse_mla_tc_kernel(const __grid_constant__ CUtensorMap tm_q, Problem P, const 
                 if (visible(x.w, ri)) last = 4 * i4 + 3;
             }
         } else {
-            for (int i = half * 32 + lane; i < K; i += 64)
+            for (int i = part * 32 + lane; i < K; i += 256)
                 if (visible(__ldg(irow + i), ri)) last = i;
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
-        if (lane == 0) reinterpret_cast<int *>(red)[half] = last;
+        if (lane == 0) reinterpret_cast<int *>(red)[part] = last;
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = misc[0];
-    const int last_slot = max(reinterpret_cast<int *>(red)[0], reinterpret_cast<int *>(red)[1]);
+    int last_slot = -1;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) last_slot = max(last_slot, reinterpret_cast<int *>(red)[i]);
     const int nblocks = (last_slot + C::BK) / C::BK;         // 0 when no slot is visible
     __syncthreads();   // red is reused by the softmax warps
 
     if (warp == 0 || warp == 2 || warp == 3) {
         // ------------------------------------------------ gather loaders (+ q TMA)
-        const int lw = warp == 0 ? 0 : warp - 1;             // ring positions p with p % 3 == lw
-        if (warp == 0 && lane == 0 && nblocks > 0) {
-            prefetch_tmap(&tm_q);
-            mbar_expect_tx(q_full, C::NATOM * C::ATOM_BYTES);
-            for (int a = 0; a < C::NATOM; ++a) tma_load_2d(q_s + a * C::ATOM_BYTES, &tm_q, q_full, 64 * a, t * 128);
-        }
-        const char *kv_bytes = reinterpret_cast<const char *>(kv);
-        bool ok_run = true;
-        ok_run = gather_turns(lw, irow, K, ri, kv_bytes, ring_s, bar0, v, nblocks, misc, lane);
+        const bool ok_run = gather_turns(lw, irow, K, ri, kv_bytes, ring_s, bar0, v, nblocks, misc, lane, rows0);
         if (!ok_run) misc[1] = 1;
         cp_async_wait<0>();
+        // a row without a visible slot: the q tile was still loaded; let it land before exit
+        if (nblocks == 0 && warp == 0 && lane == 0) mbar_wait(q_full, 0);
     } else if (warp == 1 && lane == 0 && nblocks > 0) {
         // ------------------------------------------------ MMA issuer
         const uint32_t idesc_qk = idesc_bf16(128, C::BK);
