@@ -393,27 +393,85 @@ def _breakdown(dsa, p, inp, fa, chunk, dev, stream, flush, reps=2, decode=False)
 
 
 def _e2e(dsa, p, inp, fa, chunk, dev, stream, args, ws, dist):
-    """Same metric through the public call with host buffers: H2D of the step's inputs from
-    pinned memory, dsa_forward, D2H of the result (out + lse), all inside the timed region."""
-    names = [n for n in ("q_idx", "q_idx8", "q_scale", "k_idx", "k_idx8", "k_scale", "w", "q", "kv") if n in inp]
+    """Same metric end to end through the public calls with host buffers: every step copies
+    its inputs from pinned host memory, runs the path and copies out + lse back, all inside
+    the timed region.  The step is pipelined over the query chunks on three streams: the
+    chunk's indexer inputs and q go up (copy stream), indexer -> top-k -> sparse MLA run on
+    the chunk (compute stream, the MLA on the chunk's rows as a sub-problem whose queries are
+    the last rows of a prefix of the sequence), and the chunk's out / lse come down (second
+    copy stream), so the two copy directions and the kernels overlap.  Ragged batches run as
+    one chunk."""
+    fp8 = "q_idx8" in inp
+    qi_name, ki_name = ("q_idx8", "k_idx8") if fp8 else ("q_idx", "k_idx")
+    key_names = [n for n in (ki_name, "k_scale", "kv") if n in inp]
+    row_names = [n for n in (qi_name, "q_scale", "w", "q") if n in inp]
+    names = key_names + row_names
     host = {n: inp[n].cpu().pin_memory() for n in names}
     devb = {n: torch.empty_like(inp[n]) for n in names}
     T = inp["total_q"]
+    ragged = p.cu_q is not None
+    ch = T if (ragged or not chunk) else min(chunk, args.e2e_chunk)
+    chunks = [(r0, min(ch, T - r0)) for r0 in range(0, T, ch)]
     out = torch.empty((T, 128, 512), dtype=torch.bfloat16, device=dev)
     lse = torch.empty((T, 128), dtype=torch.float32, device=dev)
+    idx = torch.empty((T, inp["topk"]), dtype=torch.int32, device=dev)
+    scores = torch.empty((ch, dsa.scores_ld(inp["max_len_k"])), dtype=torch.float32, device=dev)
     out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
-    wsb = torch.empty(dsa.dsa_forward_workspace_size(p, chunk), dtype=torch.uint8, device=dev)
-    fp8 = "q_idx8" in inp
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    s_cmp = stream
+    ev = lambda: torch.cuda.Event()                                   # noqa: E731
+    last = {"keys_free": None, "rows_free": [None] * len(chunks), "out_free": [None] * len(chunks)}
+
+    def mla_sub(r0, rc):
+        if ragged:
+            return p
+        return dsa.make_problem(1, rc, r0 + rc, rc, r0 + rc, inp["topk"], sm_scale=p.sm_scale)
+
+    subs = [mla_sub(r0, rc) for r0, rc in chunks]
 
     def step():
-        for n in names:
-            devb[n].copy_(host[n], non_blocking=True)
-        dsa.dsa_forward(p, devb["q_idx8" if fp8 else "q_idx"], devb["k_idx8" if fp8 else "k_idx"], devb["w"],
-                        devb["q"], devb["kv"], out, lse, wsb, chunk_q=chunk, q_scale=devb.get("q_scale"),
-                        k_scale=devb.get("k_scale"), stream=stream)
-        out_h.copy_(out, non_blocking=True)
-        lse_h.copy_(lse, non_blocking=True)
+        # keys (and kv) once per step, after the previous step's last kernel that reads them
+        if last["keys_free"] is not None:
+            s_in.wait_event(last["keys_free"])
+        with torch.cuda.stream(s_in):
+            for n in key_names:
+                devb[n].copy_(host[n], non_blocking=True)
+        keys_in = ev()
+        keys_in.record(s_in)
+        rows_in = []
+        for c, (r0, rc) in enumerate(chunks):
+            if last["rows_free"][c] is not None:
+                s_in.wait_event(last["rows_free"][c])
+            with torch.cuda.stream(s_in):
+                for n in row_names:
+                    devb[n][r0:r0 + rc].copy_(host[n][r0:r0 + rc], non_blocking=True)
+            e = ev()
+            e.record(s_in)
+            rows_in.append(e)
+        s_cmp.wait_event(keys_in)
+        for c, (r0, rc) in enumerate(chunks):
+            s_cmp.wait_event(rows_in[c])
+            dsa.dsa_indexer_scores(p, devb[qi_name], devb[ki_name], devb["w"], scores, row_begin=r0, row_count=rc,
+                                   q_scale=devb.get("q_scale"), k_scale=devb.get("k_scale"), stream=s_cmp)
+            dsa.dsa_topk(p, scores, idx[r0:r0 + rc], row_begin=r0, row_count=rc, stream=s_cmp)
+            if last["out_free"][c] is not None:
+                s_cmp.wait_event(last["out_free"][c])
+            dsa.dsa_sparse_mla_fwd(subs[c], devb["q"][r0:r0 + rc], devb["kv"], idx[r0:r0 + rc], out[r0:r0 + rc],
+                                   lse[r0:r0 + rc], stream=s_cmp)
+            done = ev()
+            done.record(s_cmp)
+            last["rows_free"][c] = done
+            s_out.wait_event(done)
+            with torch.cuda.stream(s_out):
+                out_h[r0:r0 + rc].copy_(out[r0:r0 + rc], non_blocking=True)
+                lse_h[r0:r0 + rc].copy_(lse[r0:r0 + rc], non_blocking=True)
+            e = ev()
+            e.record(s_out)
+            last["out_free"][c] = e
+        kf = ev()
+        kf.record(s_cmp)
+        last["keys_free"] = kf
 
     step()
     torch.cuda.synchronize(dev)
@@ -422,17 +480,27 @@ def _e2e(dsa, p, inp, fa, chunk, dev, stream, args, ws, dist):
     b = torch.cuda.Event(enable_timing=True)
     _barrier(dist)
     torch.cuda.synchronize(dev)
-    a.record(stream)
+    a.record(s_in)
     for _ in range(steps):
         step()
-    b.record(stream)
+    s_in.wait_stream(s_out)
+    b.record(s_in)
     torch.cuda.synchronize(dev)
     _barrier(dist)
     ms = _max_over_ranks(dist, a.elapsed_time(b)) / steps
     h2d = sum(host[n].numel() * host[n].element_size() for n in names)
     d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * lse_h.element_size()
+    # the pipelined calls must give exactly what dsa_forward gives on the same inputs
+    out_ref, lse_ref = torch.empty_like(out), torch.empty_like(lse)
+    wsb = torch.empty(dsa.dsa_forward_workspace_size(p, ch), dtype=torch.uint8, device=dev)
+    dsa.dsa_forward(p, devb[qi_name], devb[ki_name], devb["w"], devb["q"], devb["kv"], out_ref, lse_ref, wsb,
+                    chunk_q=ch, q_scale=devb.get("q_scale"), k_scale=devb.get("k_scale"), stream=s_cmp)
+    torch.cuda.synchronize(dev)
+    same = bool(torch.equal(out_h, out_ref.cpu()) and torch.equal(lse_h, lse_ref.cpu()))
     return {"value": ws * _tokens(inp) / (ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps}
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": steps,
+            "pipelined": f"{len(chunks)} query chunks over 3 streams (H2D / kernels / D2H)",
+            "gpu_launches_per_step": 3 * len(chunks), "identical_to_dsa_forward": same}
 
 
 # ----------------------------------------------------------------- oracle (CPU) arms
@@ -590,6 +658,7 @@ def main():
     ap.add_argument("--no-breakdown", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode_b64 secondary measurement")
+    ap.add_argument("--e2e-chunk", type=int, default=2048, help="query rows per pipelined chunk of the e2e step")
     ap.add_argument("--kernel", choices=("indexer", "topk", "sparse_mla"), default=None,
                     help="time one kernel on a bounded slice (for profilers) instead of the full step")
     ap.add_argument("--rows", type=int, default=0, help="query rows for --kernel (default: one chunk)")
