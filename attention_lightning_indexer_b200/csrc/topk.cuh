@@ -64,30 +64,47 @@ __device__ __forceinline__ void hist_add(uint32_t *hist, uint32_t d, int lane) {
 }
 
 // Warp 0: the bin holding the `remaining`-th largest key; writes bin and the count of
-// keys in strictly higher bins to scal[0], scal[1].
+// keys in strictly higher bins to scal[0], scal[1].  Lane L first sums its block of
+// nbins/32 consecutive bins (lane 0 owns the highest; the loop is skewed by the lane so the
+// 32 lanes hit 32 different banks), a warp scan finds the lane whose block holds the
+// target, and the warp then scans that block (per/32 bins per lane) to find the bin.
 __device__ __forceinline__ void select_bin(const uint32_t *hist, int nbins, int remaining, int *scal) {
     const int lane = threadIdx.x & 31;
-    const int per = nbins / 32;
+    const int per = nbins / 32;               // 64 or 32 bins per lane
     const int top = nbins - 1 - lane * per;   // lane 0 owns the highest bins
     uint32_t mine = 0;
-    for (int i = 0; i < per; ++i) mine += hist[top - i];
+    for (int i = 0; i < per; ++i) mine += hist[top - ((i + lane) & (per - 1))];
     uint32_t incl = mine;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
         const uint32_t v = __shfl_up_sync(FULL, incl, off);
         if (lane >= off) incl += v;
     }
-    const uint32_t above = incl - mine;
-    if (above < (uint32_t)remaining && (uint32_t)remaining <= incl) {
-        uint32_t acc = above;
-        for (int i = 0; i < per; ++i) {
-            const uint32_t h = hist[top - i];
-            if (acc + h >= (uint32_t)remaining) {
-                scal[0] = top - i;
-                scal[1] = (int)acc;
-                break;
-            }
-            acc += h;
+    // the lane whose block holds the target (exactly one: remaining <= total keys)
+    const unsigned hit = __ballot_sync(FULL, (incl - mine) < (uint32_t)remaining && (uint32_t)remaining <= incl);
+    const int src = hit ? __ffs(hit) - 1 : 0;  // hit == 0 cannot happen (remaining <= count); stay in range
+    const uint32_t above_blk = __shfl_sync(FULL, incl - mine, src);
+    const int btop = nbins - 1 - src * per;
+    // that block, highest bin first: lane l holds bins btop - l*q .. btop - l*q - (q-1), q = per/32
+    const int q = per / 32;
+    uint32_t h[2] = {0, 0};
+    for (int j = 0; j < q; ++j) h[j] = hist[btop - lane * q - j];
+    const uint32_t lsum = h[0] + (q > 1 ? h[1] : 0u);
+    uint32_t lincl = lsum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t v = __shfl_up_sync(FULL, lincl, off);
+        if (lane >= off) lincl += v;
+    }
+    const uint32_t lbefore = above_blk + lincl - lsum;
+    const bool mine_hit = lbefore < (uint32_t)remaining && (uint32_t)remaining <= lbefore + lsum;
+    if (hit != 0 && mine_hit) {
+        if (lbefore + h[0] >= (uint32_t)remaining) {
+            scal[0] = btop - lane * q;
+            scal[1] = (int)lbefore;
+        } else {
+            scal[0] = btop - lane * q - 1;
+            scal[1] = (int)(lbefore + h[0]);
         }
     }
 }
@@ -267,27 +284,32 @@ __device__ bool select_row_sampled(const float *src, int n, int K, unsigned char
     int *mi = segi + warp * SEG;
     int cnt = 0;
     bool overflow = false;
-    for (int base = wb; base < we; base += 128) {
-        const int i0 = base + lane * 4;
-        uint32_t k[4];
-        load4(src, i0, we, k);
-        int c4 = 0;
+    for (int base = wb; base < we; base += 512) {
+        // four 128-key chunks per step, all loads issued before any is used
+        uint32_t kk[4][4];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) c4 += (i0 + c < we) && k[c] >= t_lo;
-        int tot;
-        int off = cnt + warp_excl_scan(c4, lane, tot);
-        if (cnt + tot > SEG) overflow = true;
-        if (!overflow) {
+        for (int u = 0; u < 4; ++u) load4(src, base + 128 * u + lane * 4, we, kk[u]);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                if ((i0 + c < we) && k[c] >= t_lo) {
-                    mk[off] = k[c];
-                    mi[off] = i0 + c;
-                    ++off;
+        for (int u = 0; u < 4; ++u) {
+            const int i0 = base + 128 * u + lane * 4;
+            int c4 = 0;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) c4 += (i0 + c < we) && kk[u][c] >= t_lo;
+            int tot;
+            int off = cnt + warp_excl_scan(c4, lane, tot);
+            if (cnt + tot > SEG) overflow = true;
+            if (!overflow) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    if ((i0 + c < we) && kk[u][c] >= t_lo) {
+                        mk[off] = kk[u][c];
+                        mi[off] = i0 + c;
+                        ++off;
+                    }
                 }
             }
+            cnt += tot;
         }
-        cnt += tot;
     }
     if (lane == 0) {
         seg_cnt[warp] = overflow ? 0 : cnt;
