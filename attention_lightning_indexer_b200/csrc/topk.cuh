@@ -10,8 +10,8 @@
 // SMs (decode), so a long row is not left to 8 warps.
 //
 // Fast path (one HBM read of the row):
-//   * every 16th float4 of the row is sampled; an exact radix select on the sample gives
-//     a key t_lo that about 1.2 k keys of the full row are expected to reach;
+//   * every 16th float4 of the row is sampled; a radix select on the sample (two 11-bit
+//     digits) gives a key t_lo that about 1.2 k keys of the full row are expected to reach;
 //   * one pass over the row keeps the keys >= t_lo with their indices, each warp in its
 //     own shared-memory segment and in ascending index order (ballot prefix sums, no
 //     atomics);
@@ -143,14 +143,16 @@ __device__ __forceinline__ void load4(const float *src, int i0, int we, uint32_t
 // Exact radix selection (11/11/10-bit digits, MSB first) of the `rank`-th largest key among
 // the keys get(j), j < m, for which valid(j) holds.  Returns the key; *above receives the
 // number of keys strictly greater.  All threads call it; uses hist and scal[0..1].
+// With passes == 2 the result is only a lower bound of that key: the smallest key of the
+// 22-bit bin that holds it (enough for a candidate threshold).
 template <class C, class Get>
-__device__ uint32_t radix_select(int m, int rank, Get get, uint32_t *hist, int *scal, int *above) {
+__device__ uint32_t radix_select(int m, int rank, Get get, uint32_t *hist, int *scal, int *above, int passes = 3) {
     constexpr int THREADS = C::THREADS;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     uint32_t prefix = 0, mask = 0;
     int remaining = rank, above_total = 0;
     const int m_pad = (m + 31) & ~31;
-    for (int pass = 0; pass < 3; ++pass) {
+    for (int pass = 0; pass < passes; ++pass) {
         const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
         const int nb = pass == 2 ? 1024 : 2048;
         for (int i = tid; i < nb; i += THREADS) hist[i] = 0;
@@ -273,8 +275,10 @@ __device__ bool select_row_sampled(const float *src, int n, int K, unsigned char
     __syncthreads();
     const int target = min(ns, (int)((1.2 * K * (double)ns) / (double)n) + 16);
     int dummy;
+    // a lower bound of the sample's target-th key is all the candidate pass needs: two
+    // digit passes (22 bits)
     const uint32_t t_lo = radix_select<C>(
-        ns, target, [&](int j, uint32_t &key) { key = segk[j]; return true; }, hist, scal, &dummy);
+        ns, target, [&](int j, uint32_t &key) { key = segk[j]; return true; }, hist, scal, &dummy, 2);
     __syncthreads();   // samples no longer needed
 
     // ---- candidates: keys >= t_lo, per warp in ascending index order
