@@ -288,33 +288,32 @@ __device__ bool select_row_sampled(const float *src, int n, int K, unsigned char
     int *mi = segi + warp * SEG;
     int cnt = 0;
     bool overflow = false;
+    const unsigned lt = (1u << lane) - 1u;
     for (int base = wb; base < we; base += 512) {
-        // four 128-key chunks per step, all loads issued before any is used
-        uint32_t kk[4][4];
+        // 16 coalesced loads per lane, keys base + 32 j + lane: the order (j, lane) is the
+        // index order, so ballot prefix counts keep the segment sorted by index
+        uint32_t kk[16];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) load4(src, base + 128 * u + lane * 4, we, kk[u]);
+        for (int j = 0; j < 16; ++j) {
+            const int i = base + 32 * j + lane;
+            kk[j] = i < we ? order_key(__ldg(src + i)) : 0u;
+        }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int i0 = base + 128 * u + lane * 4;
-            int c4 = 0;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) c4 += (i0 + c < we) && kk[u][c] >= t_lo;
-            int tot;
-            int off = cnt + warp_excl_scan(c4, lane, tot);
-            if (cnt + tot > SEG) overflow = true;
-            if (!overflow) {
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    if ((i0 + c < we) && kk[u][c] >= t_lo) {
-                        mk[off] = kk[u][c];
-                        mi[off] = i0 + c;
-                        ++off;
-                    }
+        for (int j = 0; j < 16; ++j) {
+            const int i = base + 32 * j + lane;
+            const bool take = i < we && kk[j] >= t_lo;
+            const unsigned m = __ballot_sync(FULL, take);
+            if (take) {
+                const int off = cnt + __popc(m & lt);
+                if (off < SEG) {
+                    mk[off] = kk[j];
+                    mi[off] = i;
                 }
             }
-            cnt += tot;
+            cnt += __popc(m);
         }
     }
+    overflow = cnt > SEG;
     if (lane == 0) {
         seg_cnt[warp] = overflow ? 0 : cnt;
         if (overflow) scal[3] = 1;
@@ -349,7 +348,6 @@ __device__ bool select_row_sampled(const float *src, int n, int K, unsigned char
         gt_off += wgt[w2];
         eq_off += weq[w2];
     }
-    const unsigned lt = (1u << lane) - 1u;
     for (int base = 0; base < cnt; base += 32) {
         const int j = base + lane;
         const uint32_t key = j < cnt ? mk[j] : 0u;
