@@ -32,9 +32,11 @@
 // 20 bytes per clock and three reach the SM's gather rate of about 57, so three loader
 // warps take the ring positions in turn.
 //
-// Warp roles (12 warps): 0, 2, 3 gather (0 also issues the q TMA, 2 allocates tensor
-// memory), 1 issues the MMAs (one thread), 4-11 softmax/epilogue: warp w owns TMEM lane
-// quarter w % 4 (32 heads) and key/column half c = (w - 4) / 4.
+// Warp roles (12 warps): 0, 2, 3 gather (2 also allocates tensor memory), 1 issues the
+// MMAs (one thread), 4-11 scan the index row for its last visible slot, then run the
+// softmax and the epilogue: warp w owns TMEM lane quarter w % 4 (32 heads) and key/column
+// half c = (w - 4) / 4.  Thread 0 issues the q TMA right after initialising the barriers,
+// and the loaders gather the first five atoms of block 0 while the row is scanned.
 #pragma once
 
 #include "dsa_common.cuh"
