@@ -46,8 +46,7 @@ TRAFFIC = {
     # ncu capture of the 4096-query prefill launch: 1.138 GB of DRAM traffic (q reads and
     # out writes, both proportional to the query count; kv rows come from L2), scaled x8 to
     # the 32768-query launch of the 32K step
-    "sparse_mla": {"bytes_per_launch": 1.1384e9 * 8, "src_sha": ""},
-}
+    "sparse_mla": {"bytes_per_launch": 1.1384e9 * 8, "src_sha": "19f132b0bd22c041"},
 }
 
 
