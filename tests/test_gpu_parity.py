@@ -256,6 +256,36 @@ def test_sparse_mla_rows_without_valid_keys():
     assert torch.all(out[9] == 0) and torch.all(torch.isneginf(lse[9]))
 
 
+def test_sparse_mla_topk_not_multiple_of_four_with_repeated_indices():
+    # 130 slots: rows of idx are not 16-byte aligned (scalar index loads) and the second
+    # block is partial; some rows list a visible key twice (it counts once per occurrence)
+    L, k = 400, 130
+    inp = dsa_synth.make_prefill(L, topk=k, seed=13, device=DEV)
+    idx = _random_idx(inp, k, seed=13)
+    rng = np.random.default_rng(14)
+    for t in rng.choice(np.arange(200, L), 40, replace=False):
+        valid = np.nonzero((idx[t] >= 0) & (idx[t] <= t))[0]
+        idx[t, valid[1]] = idx[t, valid[0]]
+    _check_mla(inp, idx)
+
+
+def test_empty_query_set_is_a_no_op():
+    S, k = 300, 64
+    p = dsa.make_problem(1, 0, S, 0, S, k)
+    kv = torch.zeros((S, 576), dtype=torch.bfloat16, device=DEV)
+    q = torch.zeros((0, 128, 576), dtype=torch.bfloat16, device=DEV)
+    idx = torch.zeros((0, k), dtype=torch.int32, device=DEV)
+    out = torch.zeros((0, 128, 512), dtype=torch.bfloat16, device=DEV)
+    lse = torch.zeros((0, 128), dtype=torch.float32, device=DEV)
+    dsa.dsa_sparse_mla_fwd(p, q, kv, idx, out, lse)
+    ws = torch.empty(dsa.dsa_forward_workspace_size(p, 0), dtype=torch.uint8, device=DEV)
+    qi = torch.zeros((0, 64, 128), dtype=torch.bfloat16, device=DEV)
+    ki = torch.zeros((S, 128), dtype=torch.bfloat16, device=DEV)
+    w = torch.zeros((0, 64), dtype=torch.float32, device=DEV)
+    dsa.dsa_forward(p, qi, ki, w, q, kv, out, lse, ws, idx_out=idx)
+    dsa.dsa_check_device_errors()
+
+
 def test_sparse_mla_decode_ragged():
     inp = dsa_synth.make_decode(6, 300, 3000, topk=256, seed=12, device=DEV)
     _check_mla(inp, _random_idx(inp, 256, seed=12))
@@ -311,6 +341,11 @@ def test_forward_chunking_is_bit_identical():
 def test_forward_fp8_indexer_small():
     inp = dsa_synth.make_prefill(1200, topk=256, seed=22, device=DEV, fp8_indexer=True)
     _check_forward_rows(inp, sample_rows(1200, 256, n_rand=48, seed=22), chunk=512)
+
+
+def test_forward_topk_not_multiple_of_four():
+    inp = dsa_synth.make_prefill(600, topk=77, seed=24, device=DEV)
+    _check_forward_rows(inp, np.arange(600), chunk=256)
 
 
 def test_forward_decode_small_ragged():
