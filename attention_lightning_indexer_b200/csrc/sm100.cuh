@@ -207,16 +207,6 @@ __device__ __forceinline__ uint64_t desc_sw128_mn(uint32_t smem_addr, uint32_t l
     return d;
 }
 
-// 4 rows (row0..row3) x one 128-byte box column `x` of a 2-D tensor map into smem.
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap *map, uint32_t bar, int x, int r0, int r1,
-                                            int r2, int r3) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes "
-        "[%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
-        : "memory");
-}
-
 // registers -> TMEM: thread i of the warp writes row (lane base + i), 32 consecutive columns.
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
     asm volatile(
@@ -274,13 +264,13 @@ namespace sm100 {
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
-// Makes this thread's completed generic-proxy shared-memory writes visible to the
-// async proxy (tensor-core operand reads) before it signals them.
+// Orders shared-memory data written through the generic proxy (cp.async copies whose
+// completion this thread has observed on an mbarrier) before this thread's following
+// async-proxy operations (tensor-core operand reads).
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
