@@ -207,18 +207,20 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 tmem_ld32(t_lane + col, v0);
                 tmem_ld32(t_lane + col + 32, v1);
                 tmem_wait_ld();
-                const float *wq = w_s + (h * C::QPI + qi) * 64;
-                float acc0 = 0.f, acc1 = 0.f;
+                // sum over heads of w * ReLU(x): even heads in the low lane, odd heads in
+                // the high lane of packed fp32 FMAs (each lane rounds like a scalar fmaf)
+                const uint64_t *wq2 = reinterpret_cast<const uint64_t *>(w_s + (h * C::QPI + qi) * 64);
+                uint64_t acc = 0;
 #pragma unroll
-                for (int c = 0; c < 32; c += 2) {
-                    acc0 = fmaf(wq[c], fmaxf(__uint_as_float(v0[c]), 0.f), acc0);
-                    acc1 = fmaf(wq[c + 1], fmaxf(__uint_as_float(v0[c + 1]), 0.f), acc1);
-                }
+                for (int c = 0; c < 32; c += 2)
+                    fma_f32x2(acc, pack_f32x2(fmaxf(__uint_as_float(v0[c]), 0.f), fmaxf(__uint_as_float(v0[c + 1]), 0.f)),
+                              wq2[c / 2]);
 #pragma unroll
-                for (int c = 0; c < 32; c += 2) {
-                    acc0 = fmaf(wq[32 + c], fmaxf(__uint_as_float(v1[c]), 0.f), acc0);
-                    acc1 = fmaf(wq[32 + c + 1], fmaxf(__uint_as_float(v1[c + 1]), 0.f), acc1);
-                }
+                for (int c = 0; c < 32; c += 2)
+                    fma_f32x2(acc, pack_f32x2(fmaxf(__uint_as_float(v1[c]), 0.f), fmaxf(__uint_as_float(v1[c + 1]), 0.f)),
+                              wq2[16 + c / 2]);
+                float acc0, acc1;
+                unpack_f32x2(acc, acc0, acc1);
                 res[qi] = acc0 + acc1;
             }
             tc_fence_before();
