@@ -36,6 +36,7 @@ EXPORTED = (
     "dsa_forward_noalloc",
     "dsa_forward_noalloc_scratch_bytes",
     "dsa_check_device_errors",
+    "dsa_selftest_bounded_wait",
     "dsa_status_string",
     "dsa_abi_version",
 )
@@ -98,11 +99,12 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.dsa_forward_noalloc_scratch_bytes.argtypes = []
     lib.dsa_forward_noalloc_scratch_bytes.restype = sz
     lib.dsa_check_device_errors.argtypes = [P]
+    lib.dsa_selftest_bounded_wait.argtypes = [ctypes.c_uint32, P]
     lib.dsa_status_string.argtypes = [ctypes.c_int]
     lib.dsa_status_string.restype = ctypes.c_char_p
     lib.dsa_abi_version.restype = i32
     for name in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_forward", "dsa_forward_noalloc",
-                 "dsa_check_device_errors"):
+                 "dsa_check_device_errors", "dsa_selftest_bounded_wait"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -208,3 +210,8 @@ def dsa_forward_noalloc_scratch_bytes() -> int:
 
 def dsa_check_device_errors(stream=None) -> None:
     _check(load().dsa_check_device_errors(_stream(stream)), "dsa_check_device_errors")
+
+
+def dsa_selftest_bounded_wait(limit_us: int = 1000, stream=None) -> None:
+    """Launch the one-CTA kernel whose bounded wait runs out (see include/dsa.h)."""
+    _check(load().dsa_selftest_bounded_wait(limit_us, _stream(stream)), "dsa_selftest_bounded_wait")

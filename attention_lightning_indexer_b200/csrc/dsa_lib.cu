@@ -86,10 +86,16 @@ inline dsa_status_t launch_status() {
     return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
-// One-time per-process opt-in to large dynamic shared memory for each kernel.
+// Opt-in to large dynamic shared memory for each kernel.  The attribute is a setting of
+// the current device, so it is applied once per device (the first call made with that
+// device current).
+constexpr int MAX_DEVICES = 64;
+
 dsa_status_t set_smem_attrs() {
-    static bool done = false;
-    if (done) return DSA_OK;
+    static bool done[MAX_DEVICES] = {};
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return DSA_ERR_CUDA;
+    if (done[dev]) return DSA_OK;
     cudaError_t e = cudaSuccess;
     e = cudaFuncSetAttribute(dsa::topk::topk_rows_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              dsa::topk::Cfg<256>::SMEM);
@@ -112,7 +118,7 @@ dsa_status_t set_smem_attrs() {
         e = cudaFuncSetAttribute(dsa::indexer::indexer_tc_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  dsa::indexer::TcCfg<1, true>::SMEM);
     if (e != cudaSuccess) return DSA_ERR_CUDA;
-    done = true;
+    done[dev] = true;
     return DSA_OK;
 }
 
@@ -186,6 +192,20 @@ dsa_status_t mla_launch(const dsa_problem_t *p, const void *q, const void *kv, c
                                                reinterpret_cast<const __nv_bfloat16 *>(kv), idx,
                                                reinterpret_cast<__nv_bfloat16 *>(out), lse);
     return launch_status();
+}
+
+// One CTA waits on an mbarrier that nothing arrives at, so its bounded wait runs out
+// after `limit_ns`: exercises the give-up path (error flag, no hang) with no copy or MMA
+// in flight.
+__global__ void bounded_wait_selftest_kernel(uint64_t limit_ns) {
+    using namespace dsa::sm100;
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t b = smem_u32(&bar);
+    if (threadIdx.x == 0) {
+        mbar_init(b, 1);
+        fence_barrier_init();
+        mbar_wait_for(b, 0, limit_ns);
+    }
 }
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -303,6 +323,12 @@ dsa_status_t dsa_forward(const dsa_problem_t *p, const void *q_idx, const float 
     return mla_launch(p, q, kv, idx, out, lse, s);
 }
 
+dsa_status_t dsa_selftest_bounded_wait(uint32_t limit_us, dsa_stream_t stream) {
+    if (limit_us < 1 || limit_us > 10000) return DSA_ERR_INVALID_ARG;
+    bounded_wait_selftest_kernel<<<1, 32, 0, (cudaStream_t)stream>>>((uint64_t)limit_us * 1000ull);
+    return launch_status();
+}
+
 dsa_status_t dsa_check_device_errors(dsa_stream_t stream) {
     if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return DSA_ERR_CUDA;
     unsigned int flag = 0, zero = 0;
@@ -336,7 +362,7 @@ dsa_status_t dsa_check_device_errors(dsa_stream_t stream) {
 namespace {
 
 constexpr size_t NOALLOC_SCRATCH_BYTES = size_t(32) << 20;
-constexpr int NOALLOC_MAX_DEVICES = 64;
+constexpr int NOALLOC_MAX_DEVICES = MAX_DEVICES;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
 

@@ -530,18 +530,38 @@ def _oracle_forward_rows(inp, keys, rows):
     oracle.sparse_mla(q, keys["kv"], ix, dsa_synth.SM_SCALE, rows=rows, cu_q=cu_q, cu_k=cu_k)
 
 
-def _cpu_baseline(inp, n_rows, seed):
+def _cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def _cpu_baseline(inp, n_rows, seed, target_s=12.0):
+    """The oracle as it stands on the host cores, on uniformly drawn query rows of the
+    same workload.  A first draw of `n_rows` rows calibrates the per-row time; the timed
+    sample is then sized to about `target_s` seconds of CPU work."""
     import oracle
 
     keys = _oracle_inputs_host(inp)
     rng = np.random.default_rng(seed + 1234)
-    rows = np.sort(rng.choice(inp["total_q"], size=min(n_rows, inp["total_q"]), replace=False)).astype(np.int64)
+    T = inp["total_q"]
+    cal = np.sort(rng.choice(T, size=min(n_rows, T), replace=False)).astype(np.int64)
+    t0 = time.perf_counter()
+    _oracle_forward_rows(inp, keys, cal)
+    per_row = (time.perf_counter() - t0) / len(cal)
+    n = int(min(T, max(len(cal), target_s / max(per_row, 1e-6))))
+    rows = np.sort(rng.choice(T, size=n, replace=False)).astype(np.int64)
     t0 = time.perf_counter()
     _oracle_forward_rows(inp, keys, rows)
     dt = time.perf_counter() - t0
     return {"value": len(rows) / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "cpu_model": _cpu_model(),
             "sample": f"{len(rows)} uniformly drawn query rows of the same workload (full indexer row, top-k, "
-                      f"sparse MLA per row), fp64, {dt:.1f} s"}
+                      f"sparse MLA per row), fp64, {dt:.1f} s of CPU work"}
 
 
 def run_reference(args, ws, rank, local):
@@ -575,6 +595,7 @@ def run_reference(args, ws, rank, local):
         "config": {"workload": args.workload, "global_batch": inp["batch"], "seq_len": int(inp["max_len_k"]),
                    "topk": inp["topk"], "chunk_q": wl.chunk, "parallelism": "host cores (rank 0 only)"},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "cpu_model": _cpu_model(),
                          "sample": f"{per_step} uniformly drawn query rows per step of the same workload, fp64"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,

@@ -95,6 +95,10 @@ typedef struct dsa_problem {
  *   w       : [T, H_I] fp32
  *   scores  : [row_count, ld_scores] fp32, ld_scores >= max_len_k, ld_scores % 4 == 0
  * Accumulation is fp32 (tensor cores); the e4m3 scales are applied in fp32.
+ * The e4m3 scales must be finite and > 0: the kernel multiplies them into the finished
+ * head sum, which equals the definition only because ReLU(a*x) = a*ReLU(x) for a > 0
+ * (a non-positive scale gives unspecified scores; they live in device memory, so the
+ * host cannot check them).
  */
 dsa_status_t dsa_indexer_scores(const dsa_problem_t *p, const void *q_idx, const float *q_scale,
                                 const void *k_idx, const float *k_scale, const float *w,
@@ -163,6 +167,9 @@ dsa_status_t dsa_forward(const dsa_problem_t *p, const void *q_idx, const float 
  * of as many rows as fit; a problem whose longest score row alone (max_len_k rounded up
  * to 4 fp32) does not fit returns DSA_ERR_WORKSPACE before anything is launched.
  * idx_out is required here (it is the caller's output, not scratch).
+ * Rows per chunk = 32 MiB / (4 * ceil4(max_len_k)) (8192 rows at 1K keys, 64 rows at
+ * 128K keys): at long contexts the chunks get small and the indexer launches run with
+ * few CTAs, so throughput falls far below dsa_forward with a large workspace.
  * The first call on a device looks up the array's device address (make it outside any
  * stream capture).  All calls share the array: calls that overlap on the GPU race on it.
  * Nothing is allocated or freed by this call.
@@ -180,6 +187,15 @@ size_t dsa_forward_noalloc_scratch_bytes(void);
  * DSA_ERR_DEVICE_TIMEOUT, or DSA_ERR_CUDA if the synchronisation itself failed.
  */
 dsa_status_t dsa_check_device_errors(dsa_stream_t stream);
+
+/*
+ * Self-test of the device-side failure path (no counterpart on the pages): launches one
+ * CTA whose bounded wait on a barrier that nothing signals gives up after `limit_us`
+ * microseconds (1 .. 10000), as a stalled pipeline wait would.  No copy or tensor-core
+ * operation is in flight.  The next dsa_check_device_errors() then returns
+ * DSA_ERR_DEVICE_TIMEOUT and clears the flag; the device stays usable.
+ */
+dsa_status_t dsa_selftest_bounded_wait(uint32_t limit_us, dsa_stream_t stream);
 
 /* Static English description of a status code (never NULL). */
 const char *dsa_status_string(dsa_status_t s);

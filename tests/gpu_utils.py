@@ -64,6 +64,8 @@ def recall_excluding_near_ties(gpu_idx: np.ndarray, ora_scores: np.ndarray, boun
         keff = min(k, n)
         sel = set(int(x) for x in gpu_idx[r] if x >= 0)
         assert len(sel) == keff, f"row {r}: {len(sel)} distinct indices, expected {keff}"
+        npad = int(np.count_nonzero(gpu_idx[r] == -1))
+        assert npad == k - keff, f"row {r}: {npad} slots of -1 padding, expected {k - keff}"
         assert max(sel) <= n - 1
         if keff == n:
             assert sel == set(range(n))

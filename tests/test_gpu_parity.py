@@ -378,5 +378,23 @@ def test_prefill_128k_fp8_full_size_sampled_bench_config():
 
 
 def test_decode_b64_full_size_sampled():
+    # every one of the 64 sequences: each seeded context length is covered
     inp = dsa_synth.make_workload("decode_b64", seed=0, device=DEV)
-    _check_forward_rows(inp, np.array([0, 7, 31, 63]))
+    _check_forward_rows(inp, np.arange(64))
+
+
+# ------------------------------------------------------------ failure path
+
+def test_bounded_wait_gives_up_reports_and_clears():
+    # A one-CTA kernel waits ~1 ms on a barrier that nothing signals: the wait gives up
+    # instead of hanging, the sticky flag reports DSA_ERR_DEVICE_TIMEOUT once, and the
+    # device keeps working (a real forward right after is still exact).
+    dsa.dsa_check_device_errors()                       # start from a clear flag
+    dsa.dsa_selftest_bounded_wait(1000)
+    with pytest.raises(dsa.DsaError) as e:
+        dsa.dsa_check_device_errors()
+    assert e.value.code == 5
+    dsa.dsa_check_device_errors()                       # cleared by the read
+    inp = dsa_synth.make_workload("pr_ref_256", seed=0, device=DEV)
+    _check_forward_rows(inp, np.arange(0, 256, 17))
+    dsa.dsa_check_device_errors()

@@ -135,6 +135,30 @@ def test_indexer_ragged_batch_uses_own_keys_and_last_token_positions():
     assert np.all(got[4:, 7:] == -np.inf)
 
 
+def test_positions_hand_worked_ragged_and_match_the_indexer_extent():
+    # The boundary's ragged reading: the queries of sequence b are its last len_q(b)
+    # tokens.  cu_q = [0, 4, 11], cu_k = [0, 11, 18]: sequence 0 has 11 keys and its 4
+    # queries sit at positions 7..10; sequence 1 has 7 keys and 7 queries at 0..6.
+    cu_q = np.array([0, 4, 11], dtype=np.int32)
+    cu_k = np.array([0, 11, 18], dtype=np.int32)
+    pos = oracle.positions(np.arange(11), cu_q, cu_k)
+    np.testing.assert_array_equal(pos, [7, 8, 9, 10, 0, 1, 2, 3, 4, 5, 6])
+    # The same positions, read off the C indexer: the last finite column of each row is
+    # pos(t) (w > 0 and q = k = 1 make every visible score positive).
+    H, D = 2, 4
+    q = np.ones((11, H, D))
+    k = np.ones((18, D))
+    w = np.ones((11, H))
+    sc = oracle.indexer(q, w, k, cu_q=cu_q, cu_k=cu_k)
+    last = np.array([np.nonzero(np.isfinite(row))[0].max() for row in sc])
+    np.testing.assert_array_equal(last, pos)
+    # plain prefill (cu arrays of one sequence, T = L) and a decode batch (one query each)
+    np.testing.assert_array_equal(oracle.positions(np.arange(5), [0, 5], [0, 5]), np.arange(5))
+    np.testing.assert_array_equal(oracle.positions(np.arange(3), [0, 1, 2, 3], [0, 9, 10, 40]), [8, 0, 29])
+    # queries that are the last 3 tokens of a 10-token prefix
+    np.testing.assert_array_equal(oracle.positions(np.arange(3), [0, 3], [0, 10]), [7, 8, 9])
+
+
 def test_e4m3_decoder_matches_library_cast():
     codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
     lib = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
