@@ -10,7 +10,7 @@
 #include "../../include/dsa.h"
 #include "dsa_common.cuh"
 #include "indexer_tc.cuh"
-#include "sparse_mla_tc.cuh"
+#include "sparse_mla_pair.cuh"
 #include "topk.cuh"
 
 namespace {
@@ -81,6 +81,22 @@ bool make_tmap_rows(CUtensorMap *m, const void *base, bool fp8, uint64_t cols, u
     return r == CUDA_SUCCESS;
 }
 
+// 2-D row-major bf16 tensor map (`cols` x `rows`) with a `box_cols` x `box_rows` box and
+// no swizzle (TMA stores of row-major tiles staged in shared memory).
+bool make_tmap_plain_bf16(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint32_t box_cols,
+                          uint32_t box_rows) {
+    auto enc = tensor_map_encoder();
+    if (enc == nullptr) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 inline dsa_status_t launch_status() {
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
@@ -103,8 +119,8 @@ dsa_status_t set_smem_attrs() {
         e = cudaFuncSetAttribute(dsa::topk::topk_rows_kernel<512>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  dsa::topk::Cfg<512>::SMEM);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(dsa::mla::sparse_mla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             dsa::mla::TcCfg::SMEM);
+        e = cudaFuncSetAttribute(dsa::mla::sparse_mla_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 dsa::mla::PairCfg::SMEM);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(dsa::indexer::indexer_tc_kernel<8, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  dsa::indexer::TcCfg<8, false>::SMEM);
@@ -184,13 +200,15 @@ dsa_status_t mla_launch(const dsa_problem_t *p, const void *q, const void *kv, c
                         float *lse, cudaStream_t stream) {
     if (p->total_q == 0) return DSA_OK;
     Problem P = to_dev(p);
-    CUtensorMap tq;
-    // q: [T*128 rows, 576] read as 128-row boxes of 64 dims (the latent rows are gathered with cp.async)
-    if (!make_tmap_rows(&tq, q, false, 576, (uint64_t)p->total_q * 128, 128)) return DSA_ERR_CUDA;
-    dsa::mla::sparse_mla_tc_kernel<<<2u * (unsigned)p->total_q, dsa::mla::TcCfg::THREADS, dsa::mla::TcCfg::SMEM,
-                                     stream>>>(tq, P, reinterpret_cast<const __nv_bfloat16 *>(q),
-                                               reinterpret_cast<const __nv_bfloat16 *>(kv), idx,
-                                               reinterpret_cast<__nv_bfloat16 *>(out), lse);
+    CUtensorMap tq, to;
+    // q: [T*128 rows, 576] read as 64-row boxes of 64 dims (each CTA of a pair loads its 64
+    // heads; the latent rows are gathered with cp.async); out: [T*128 rows, 512] written as
+    // 128 x 128 tiles
+    if (!make_tmap_rows(&tq, q, false, 576, (uint64_t)p->total_q * 128, 64)) return DSA_ERR_CUDA;
+    if (!make_tmap_plain_bf16(&to, out, 512, (uint64_t)p->total_q * 128, 128, 128)) return DSA_ERR_CUDA;
+    dsa::mla::sparse_mla_pair_kernel<<<2u * (unsigned)p->total_q, dsa::mla::PairCfg::THREADS,
+                                       dsa::mla::PairCfg::SMEM, stream>>>(
+        tq, to, P, reinterpret_cast<const __nv_bfloat16 *>(kv), idx, reinterpret_cast<__nv_bfloat16 *>(out), lse);
     return launch_status();
 }
 

@@ -1,0 +1,615 @@
+// sparse_mla_pair.cuh -- attention over the selected latent rows (MLA in MQA mode) on a
+// pair of SMs: one 2-CTA cluster per query token, 2-SM tensor-core MMAs (cta_group::2).
+//
+// "DeepSeek-V3.2 tech report summary", §1 DSA: full attention only over the k selected
+// tokens; MLA-based implementation in MQA mode (every 576-d latent row is shared by all
+// 128 query heads); value = first 512 dims; softmax scale 1/sqrt(192).
+//
+// The index row is cut into blocks of 256 slots.  CTA c of the pair owns slots
+// [256 b + 128 c, 256 b + 128 c + 128) of block b ("its keys") and heads 64 c .. 64 c + 63.
+//   QK_b   S^T[key, h] = kv[key, :576] . q[h, :576]          M = 256 keys (128 per CTA,
+//          A = the gathered rows in each CTA), N = 128 heads (B = q, 64 heads per CTA),
+//          K = 576: each CTA receives S^T of its own 128 keys for all heads in TMEM.
+//   softmax  each CTA turns its S^T into P^T = exp2(S^T * scale * log2 e - m[h]) for its
+//          keys; m[h] is the pair's running per-head reference maximum (exact block maxima
+//          are exchanged every block, the reference moves lazily, only when a block
+//          maximum exceeds it by more than TAU).
+//   PV_b   O^T[d, h] += V^T[d, key] . P^T[key, h] over the 256 keys of the block:
+//          M = 256 value dims per instruction (two instructions cover 512), A = value
+//          atoms in each CTA (CTA c holds dims 256 i + 128 c .. + 127 for every key of the
+//          block), N = 128 heads (B = P^T, CTA c holds heads 64 c .. + 63 for all 256
+//          keys): each CTA stores the P^T of its keys for the other CTA's heads straight
+//          into the other CTA's shared memory (16 KB per block).
+// So every flop of the definition is executed once, each selected row is gathered once
+// whole (QK) plus the value dims each CTA needs for PV, and q is split between the CTAs.
+//
+// Tensor memory per CTA (512 columns): S^T double buffer [0,128) [128,256) (lanes = the
+// CTA's keys, columns = heads); O^T [256,384) for value dims 128 c + [0,128) and
+// [384,512) for 256 + 128 c + [0,128) (lanes = value dims, columns = heads).
+// Shared memory per CTA: q half (9 swizzled 64-dim atoms of 64 heads, 72 KB), P^T buffer
+// (256 keys x 64 heads, MN-major, 32 KB), a 7-slot ring of gathered 16 KB atoms (128 keys x
+// 64 dims, 128-byte swizzle applied in the address) fed in MMA order QK_0, QK_1, PV_0,
+// QK_2, PV_1, ..., PV_{n-1}:
+//   QK_b  9 atoms of the CTA's own keys;
+//   PV_b  8 atoms: for i = 0, 1 and key half h = 0, 1 (the keys of CTA h), the CTA's two
+//         64-dim value atoms 4 i + 2 c + {0, 1}.
+// Both CTAs lay the ring out identically (same positions, same slots); the even CTA
+// issues every MMA once both CTAs' operands have landed and commits to the barriers of
+// both.  Gathers are 16-byte cp.async (one warp instruction moves 4 rows x 128 bytes),
+// whose issue rate is about 20 GB/s per warp, so seven loader warps take the ring
+// positions in turn, one slot each; a loader signals the even CTA's barrier of its slot
+// itself once its copies have landed (wait, proxy fence, cluster-scope arrive), and the
+// softmax warps of both CTAs signal the even CTA's P^T barrier the same way, so no
+// thread relays the odd CTA's state.
+//
+// Warp roles (16 warps per CTA): 0-6 gather (0 also issues the q TMA and allocates tensor
+// memory), 7 issues the MMAs (even CTA), 8-15 scan the index row, then run the softmax
+// and the epilogue: warp w owns TMEM lane quarter w % 4 and head half (w - 8) / 4.  The
+// first two warpgroups give registers to the last two (setmaxnreg).
+#pragma once
+
+#include "dsa_common.cuh"
+#include "sm100.cuh"
+
+namespace dsa {
+namespace mla {
+
+struct PairCfg {
+    static constexpr int BLK = 256;                 // index slots per block (128 per CTA)
+    static constexpr int NATOM = 9;                 // 64-dim atoms per 576-d row
+    static constexpr int ATOM = 128 * 128;          // one gathered atom: 128 keys x 128 bytes
+    static constexpr int QATOM = 64 * 128;          // one q atom: 64 heads x 128 bytes
+    static constexpr int NSLOT = 7;
+    static constexpr int NLOAD = 7;                 // loader warps, one ring slot each
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_P = OFF_Q + NATOM * QATOM;        // 73728
+    static constexpr int OFF_RING = OFF_P + 256 * 128;         // 106496
+    static constexpr int OFF_RED = OFF_RING + NSLOT * ATOM;    // [4][128] f32
+    static constexpr int OFF_XM = OFF_RED + 4 * 128 * 4;       // [2][128] f32, peer block maxima
+    static constexpr int OFF_XL = OFF_XM + 2 * 128 * 4;        // [128] f32, peer row sums
+    static constexpr int OFF_MR = OFF_XL + 128 * 4;            // [128] f32, running reference max
+    static constexpr int OFF_FS = OFF_MR + 128 * 4;            // [128] f32, rescale factor / 1/l
+    static constexpr int OFF_BAR = OFF_FS + 128 * 4;
+    // (unused)[7] empty[7] pfull[7] q_full q_peer s_full[2] s_free[2] p_full (unused)
+    // pv_done o_ready xbar[2] lbar drain
+    static constexpr int NBARS = 3 * NSLOT + 2 + 2 + 2 + 2 + 2 + 2 + 1 + 1;
+    static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
+    static constexpr int SMEM = OFF_MISC + 16;
+    static constexpr int THREADS = 512;
+    static constexpr int SOFT0 = 8;                 // first softmax warp
+    static constexpr int REG_LOW = 88, REG_HIGH = 168;   // 256 x 88 + 256 x 168 = 512 x 128
+    static constexpr int TMEM_S = 0, TMEM_O = 256;
+    static constexpr float TAU = 8.0f;              // lazy-rescale threshold (log2 units)
+    static_assert(SMEM <= 232448, "shared memory budget");
+    static_assert(NLOAD <= NSLOT, "ring waits need NLOAD <= NSLOT");
+    static_assert(256 * REG_LOW + 256 * REG_HIGH <= 65536 / THREADS * THREADS, "register split");
+    static_assert(2 * 128 * 128 * 2 <= NSLOT * ATOM, "output staging fits in the ring");
+};
+
+__device__ __forceinline__ bool pair_visible(int e, const RowInfo &ri) { return e >= 0 && e <= ri.pos && e < ri.len_k; }
+
+// Group g (0 .. 2n-1) of the ring order QK_0, QK_1, PV_0, QK_2, PV_1, ..., PV_{n-1}.
+__device__ __forceinline__ void pair_group(int g, int n, bool &qk, int &blk) {
+    if (g == 0) { qk = true; blk = 0; }
+    else if (g == 2 * n - 1) { qk = false; blk = n - 1; }
+    else if (g & 1) { qk = true; blk = (g + 1) >> 1; }
+    else { qk = false; blk = (g >> 1) - 1; }
+}
+
+// PV position m (0..7) of a group starting at ring position p: instruction i, key half h,
+// and the 64-dim value atom it holds.  The two atoms of one (i, h) pair form one MN-major
+// operand whose lower-addressed slot must hold the lower dims.
+__device__ __forceinline__ int pv_value_atom(int c, int p, int m) {
+    const int i = m >> 2, h = (m >> 1) & 1, e = m & 1;
+    const int s0 = (p + 4 * i + 2 * h) % PairCfg::NSLOT;
+    const int s1 = (s0 + 1) % PairCfg::NSLOT;
+    const bool lo_first = s0 < s1;
+    return 4 * i + 2 * c + (lo_first ? e : 1 - e);
+}
+
+// Index entries of slots s0 + 32 (lane / 8) + i, i < 32, of the row (-1 past its end).
+__device__ __forceinline__ void pair_fetch(const int32_t *irow, int K, int s0, int lane, int (&e)[32]) {
+    const int s = s0 + (lane >> 3) * 32;
+    if ((K & 3) == 0 && s + 31 < K) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int4 x = __ldg(reinterpret_cast<const int4 *>(irow + s) + i);
+            e[4 * i] = x.x; e[4 * i + 1] = x.y; e[4 * i + 2] = x.z; e[4 * i + 3] = x.w;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) e[i] = s + i < K ? __ldg(irow + s + i) : -1;
+    }
+}
+
+// One atom (32 copy instructions, lane l: 16-byte chunk l % 8 of rows 32 (l / 8) + i)
+// into a ring slot, committed as one cp.async group of the lane.
+__device__ __forceinline__ void pair_gather_atom(const char *kv_bytes, const int (&rows)[32], int a, uint32_t slot,
+                                                 int lane) {
+    using namespace sm100;
+    const int ch = lane & 7;
+    const int r0 = (lane >> 3) * 32;
+    const char *src = kv_bytes + a * 128 + ch * 16;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const int r = r0 + i;
+        cp_async16(slot + r * 128 + ((ch ^ (r & 7)) << 4), src + (int64_t)rows[i] * 1152);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+// The warp's last atom has landed (all its lanes' copies): make it visible to the tensor
+// core and count it on the even CTA's barrier of its slot.
+__device__ __forceinline__ void pair_signal_atom(uint32_t lead_bar, int lane) {
+    using namespace sm100;
+    cp_async_wait<0>();
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive_cluster(lead_bar);
+}
+
+// Lane l ends with the reduction (max or sum) over the 32 lanes of element l of v.
+template <bool MAX>
+__device__ __forceinline__ float transpose_reduce32(float (&v)[32], int lane) {
+#pragma unroll
+    for (int m = 16, n = 32; m >= 1; m >>= 1, n >>= 1) {
+        const bool upper = (lane & m) != 0;
+#pragma unroll
+        for (int i = 0; i < n / 2; ++i) {
+            const float send = upper ? v[i] : v[i + n / 2];
+            const float keep = upper ? v[i + n / 2] : v[i];
+            const float recv = __shfl_xor_sync(0xffffffffu, send, m);
+            v[i] = MAX ? fmaxf(keep, recv) : keep + recv;
+        }
+    }
+    return v[0];
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
+sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_out, Problem P,
+                       const __nv_bfloat16 *__restrict__ kv, const int32_t *__restrict__ idx,
+                       __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
+    using C = PairCfg;
+    using namespace sm100;
+    extern __shared__ __align__(1024) unsigned char smem[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int cr = (int)cluster_ctarank();                   // 0: issues the MMAs
+    const int peer = cr ^ 1;
+    const int T = P.total_q;
+    const int t = T - 1 - (int)(blockIdx.x >> 1);           // heavier (later) tokens first
+    const int K = P.topk;
+    const RowInfo ri = row_info(P, t);
+    const int32_t *irow = idx + (int64_t)t * K;
+
+    const uint32_t sbase = smem_u32(smem);
+    const bool misaligned = (sbase & 1023u) != 0;           // uniform; checked below without an early exit
+    const uint32_t q_s = sbase + C::OFF_Q;
+    const uint32_t p_s = sbase + C::OFF_P;
+    const uint32_t ring_s = sbase + C::OFF_RING;
+    float *red = reinterpret_cast<float *>(smem + C::OFF_RED);
+    float *xm = reinterpret_cast<float *>(smem + C::OFF_XM);
+    float *xl = reinterpret_cast<float *>(smem + C::OFF_XL);
+    float *mr = reinterpret_cast<float *>(smem + C::OFF_MR);
+    float *fs = reinterpret_cast<float *>(smem + C::OFF_FS);
+    const uint32_t bar0 = sbase + C::OFF_BAR;
+    auto empty = [&](int s) { return bar0 + 8u * (C::NSLOT + s); };
+    auto pfull = [&](int s) { return bar0 + 8u * (2 * C::NSLOT + s); };
+    const uint32_t q_full = bar0 + 8u * (3 * C::NSLOT);
+    const uint32_t q_peer = q_full + 8;
+    auto s_full = [&](int b) { return q_full + 16 + 8u * b; };
+    auto s_free = [&](int b) { return q_full + 32 + 8u * b; };
+    const uint32_t p_full = q_full + 48;                    // P^T of both CTAs written (even CTA)
+    const uint32_t pv_done = q_full + 64;
+    const uint32_t o_ready = q_full + 72;
+    auto xbar = [&](int b) { return q_full + 80 + 8u * b; };
+    const uint32_t lbar = q_full + 96;
+    const uint32_t drain = q_full + 104;
+    volatile uint32_t *misc = reinterpret_cast<volatile uint32_t *>(smem + C::OFF_MISC);  // [0] tmem, [1] abort
+
+    // ---- setup (every thread of both CTAs reaches the cluster barriers below)
+    if (tid == 0 && !misaligned) {
+        for (int s = 0; s < C::NSLOT; ++s) {
+            mbar_init(empty(s), 1);
+            mbar_init(pfull(s), 2);       // the loader warp of this position in each CTA
+        }
+        mbar_init(q_full, 1);
+        mbar_init(q_peer, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(s_full(b), 1);
+            mbar_init(s_free(b), 16);     // 8 softmax warps of each CTA
+            mbar_init(xbar(b), 1);
+        }
+        mbar_init(p_full, 16);            // 8 softmax warps of each CTA
+        mbar_init(pv_done, 1);
+        mbar_init(o_ready, 1);
+        mbar_init(lbar, 1);
+        mbar_init(drain, 1);
+        misc[1] = 0;
+        fence_barrier_init();
+        // this CTA's 64 heads of q land while the index row is scanned
+        prefetch_tmap(&tm_q);
+        mbar_expect_tx(q_full, C::NATOM * C::QATOM);
+        for (int a = 0; a < C::NATOM; ++a) tma_load_2d(q_s + a * C::QATOM, &tm_q, q_full, 64 * a, t * 128 + 64 * cr);
+    }
+    if (tid == 0 && misaligned) {
+        raise_error(ERR_SMEM_ALIGN);
+        misc[1] = 1;
+    }
+    const char *kv_bytes = reinterpret_cast<const char *>(kv);
+    const int lw = warp;                                     // loader warps 0 .. NLOAD-1
+    const bool loader = warp < C::NLOAD;
+    int rows[32];
+    if (loader && !misaligned) {
+        // the first ring positions (QK_0 atoms 0 .. NSLOT-1 of this CTA's keys) are gathered
+        // while the row is scanned
+        __syncwarp();
+        named_bar(3, 32 * C::NLOAD);
+        pair_fetch(irow, K, 128 * cr, lane, rows);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) rows[i] = ri.kbase + (pair_visible(rows[i], ri) ? rows[i] : 0);
+        for (int pp = lw; pp < C::NSLOT; pp += C::NLOAD) pair_gather_atom(kv_bytes, rows, pp, ring_s + pp * C::ATOM, lane);
+    }
+    if (warp >= C::SOFT0) {   // last visible slot of the row (8 warps, interleaved int4 groups)
+        int last = -1;
+        const int part = warp - C::SOFT0;
+        if ((K & 3) == 0) {
+            const int n4 = K >> 2;
+#pragma unroll 2
+            for (int i4 = part * 32 + lane; i4 < n4; i4 += 256) {
+                const int4 x = __ldg(reinterpret_cast<const int4 *>(irow) + i4);
+                if (pair_visible(x.x, ri)) last = 4 * i4;
+                if (pair_visible(x.y, ri)) last = 4 * i4 + 1;
+                if (pair_visible(x.z, ri)) last = 4 * i4 + 2;
+                if (pair_visible(x.w, ri)) last = 4 * i4 + 3;
+            }
+        } else {
+            for (int i = part * 32 + lane; i < K; i += 256)
+                if (pair_visible(__ldg(irow + i), ri)) last = i;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
+        if (lane == 0) reinterpret_cast<int *>(red)[part] = last;
+        if (warp < C::SOFT0 + 4) mr[tid - 32 * C::SOFT0] = -INFINITY;   // reference maxima of the 128 heads
+    }
+    cluster_sync();   // both CTAs running, their barriers initialised
+    if (warp == 0) tmem_alloc_pair(sbase + C::OFF_MISC, 512);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = misc[0];
+    int last_slot = -1;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) last_slot = max(last_slot, reinterpret_cast<int *>(red)[i]);
+    const int nblocks = misaligned ? 0 : (last_slot + C::BLK) / C::BLK;   // 0 when no slot is visible
+    __syncthreads();   // red is reused by the softmax warps
+    const uint32_t peer_misc1 = mapa_shared(sbase + C::OFF_MISC + 4, (uint32_t)peer);
+    auto abort_pair = [&]() {                                // stop both CTAs of the pair
+        misc[1] = 1;
+        st_cluster_u32(peer_misc1, 1u);
+    };
+
+    if (warp < C::SOFT0) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REG_LOW));
+    if (loader) {
+        // ------------------------------------------------ gather loaders
+        bool ok = true;
+        int p = 0, cached = -1;                              // cached: slot base of `rows`
+        const uint32_t lead_pfull = mapa_shared(pfull(0), 0);
+        int pend = -1;                                       // slot of this warp's atom in flight
+        if (!misaligned) {
+            cached = 128 * cr;
+            if (lw < C::NSLOT) pend = lw;                    // gathered during the scan
+        }
+        for (int g = 0; ok && g < 2 * nblocks; ++g) {
+            bool qk;
+            int b;
+            pair_group(g, nblocks, qk, b);
+            const int natoms = qk ? C::NATOM : 8;
+            for (int m = 0; m < natoms; ++m) {
+                const int pp = p + m;
+                if (pp % C::NLOAD != lw || pp < C::NSLOT) continue;
+                if (pend >= 0) {                             // first: the landed atom (no cycle with the slot wait)
+                    pair_signal_atom(lead_pfull + 8u * pend, lane);
+                    pend = -1;
+                }
+                const int h = qk ? cr : ((m >> 1) & 1);
+                const int s0 = C::BLK * b + 128 * h;
+                if (s0 != cached) {
+                    pair_fetch(irow, K, s0, lane, rows);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) rows[i] = ri.kbase + (pair_visible(rows[i], ri) ? rows[i] : 0);
+                    cached = s0;
+                }
+                const int a = qk ? m : pv_value_atom(cr, p, m);
+                const int slot = pp % C::NSLOT;
+                bool okw = true;
+                if (lane == 0) okw = mbar_wait(empty(slot), ((pp / C::NSLOT) - 1) & 1);
+                if (!__shfl_sync(0xffffffffu, okw, 0) || misc[1]) { ok = false; break; }
+                pair_gather_atom(kv_bytes, rows, a, ring_s + slot * C::ATOM, lane);
+                pend = slot;
+            }
+            p += natoms;
+        }
+        if (pend >= 0 && ok && nblocks > 0) pair_signal_atom(lead_pfull + 8u * pend, lane);
+        if (!ok && lane == 0) abort_pair();
+        cp_async_wait<0>();
+        if (warp == 0 && lane == 0 && !misaligned) mbar_wait(q_full, 0);   // q landed before exit
+    } else if (warp == 7 && lane == 0 && cr == 0 && nblocks > 0) {
+        // ------------------------------------------------ MMA issuer (even CTA)
+        const uint32_t idesc_qk = idesc_bf16(256, 128);
+        const uint32_t idesc_pv = idesc_bf16_mn_mn(256, 128);
+        bool ok = mbar_wait(q_full, 0) && mbar_wait_cluster(q_peer, 0);
+        bool issued = false;
+        int pos = 0;
+        for (int g = 0; ok && g < 2 * nblocks; ++g) {
+            bool qk;
+            int b;
+            pair_group(g, nblocks, qk, b);
+            if (qk) {                                        // QK_b -> S^T buffer b & 1
+                if (b >= 2 && !mbar_wait_cluster(s_free(b & 1), ((b >> 1) - 1) & 1)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d = tmem + C::TMEM_S + 128 * (b & 1);
+                for (int a = 0; a < C::NATOM; ++a, ++pos) {
+                    const int slot = pos % C::NSLOT;
+                    const uint32_t par = (pos / C::NSLOT) & 1;
+                    if (!mbar_wait_cluster(pfull(slot), par) || misc[1]) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t sa = ring_s + slot * C::ATOM;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_f16_pair(d, desc_sw128(sa + kk * 32), desc_sw128(q_s + a * C::QATOM + kk * 32), idesc_qk,
+                                     (a > 0 || kk > 0) ? 1u : 0u);
+                    issued = true;
+                    mma_commit_pair_both(empty(slot));
+                }
+                if (!ok) break;
+                mma_commit_pair_both(s_full(b & 1));
+            } else {                                         // PV_b
+                if (!mbar_wait_cluster(p_full, b & 1)) { ok = false; break; }
+                tc_fence_after();
+                for (int i = 0; ok && i < 2; ++i) {
+                    const uint32_t d = tmem + C::TMEM_O + 128 * i;
+                    for (int h = 0; h < 2; ++h, pos += 2) {
+                        const int s0 = pos % C::NSLOT, s1 = (pos + 1) % C::NSLOT;
+                        const uint32_t par0 = (pos / C::NSLOT) & 1, par1 = ((pos + 1) / C::NSLOT) & 1;
+                        if (!mbar_wait_cluster(pfull(s0), par0) || !mbar_wait_cluster(pfull(s1), par1) || misc[1]) {
+                            ok = false;
+                            break;
+                        }
+                        const int slo = s0 < s1 ? s0 : s1, shi = s0 < s1 ? s1 : s0;
+                        const uint32_t vb = ring_s + slo * C::ATOM;
+                        const uint32_t lbo = (uint32_t)(shi - slo) * C::ATOM;
+#pragma unroll
+                        for (int k8 = 0; k8 < 8; ++k8)
+                            mma_f16_pair(d, desc_sw128_mn(vb + k8 * 2048, lbo),
+                                         desc_sw128_mn(p_s + (8 * h + k8) * 2048, 16384), idesc_pv,
+                                         (b > 0 || h > 0 || k8 > 0) ? 1u : 0u);
+                        issued = true;
+                        mma_commit_pair_both(empty(s0));
+                        mma_commit_pair_both(empty(s1));
+                    }
+                }
+                if (!ok) break;
+                mma_commit_pair_both(pv_done);
+                if (b == nblocks - 1) mma_commit_pair_both(o_ready);
+            }
+        }
+        if (!ok) {
+            abort_pair();
+            if (issued) {                                    // nothing may be in flight at dealloc
+                mma_commit_pair_both(drain);
+                mbar_wait(drain, 0);
+            }
+        }
+    } else if (warp == 7 && lane == 0 && cr == 1 && nblocks > 0) {
+        // ------------------------------------------------ the odd CTA's q has landed
+        if (mbar_wait(q_full, 0)) mbar_arrive_cluster(mapa_shared(q_peer, 0));
+        else abort_pair();
+    }
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::REG_HIGH));
+        // ------------------------------------------------ softmax + epilogue
+        const int st = tid - 32 * C::SOFT0;                  // 0 .. 255
+        const int quarter = warp & 3;
+        const int h2 = (warp - C::SOFT0) >> 2;               // head half handled by this warp
+        const int key = quarter * 32 + lane;                 // this thread's key among the CTA's 128
+        const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
+        const float sl2 = P.sm_scale * 1.4426950408889634f;
+        const uint32_t xm_peer = mapa_shared(sbase + C::OFF_XM, (uint32_t)peer);
+        const uint32_t xbar_peer = mapa_shared(xbar(0), (uint32_t)peer);
+        const uint32_t s_free_lead = mapa_shared(s_free(0), 0);
+        const uint32_t p_full_lead = mapa_shared(p_full, 0);
+        const uint32_t p_peer_s = mapa_shared(p_s, (uint32_t)peer);
+        float l[64];
+#pragma unroll
+        for (int j = 0; j < 64; ++j) l[j] = 0.f;
+        bool ok = true;
+        const int sown = 128 * cr + key;                     // slot of this thread's key within a block
+        int ent = nblocks > 0 && sown < K ? __ldg(irow + sown) : -1;
+        for (int b = 0; b < nblocks; ++b) {
+            const bool vis = pair_visible(ent, ri);
+            {
+                const int s = C::BLK * (b + 1) + sown;
+                ent = (b + 1 < nblocks && s < K) ? __ldg(irow + s) : -1;
+            }
+            const bool fail = misc[1] != 0 || !mbar_wait_cluster(s_full(b & 1), (b >> 1) & 1);
+            if (named_bar_or(1, 256, fail)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t sb = t_lane + C::TMEM_S + 128 * (b & 1) + 64 * h2;
+            // ---- exact block maxima of this CTA's keys (per head), then of the pair
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                uint32_t sr[32];
+                float v[32];
+                tmem_ld32(sb + 32 * j, sr);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = vis ? __uint_as_float(sr[i]) : -INFINITY;
+                red[quarter * 128 + 64 * h2 + 32 * j + lane] = transpose_reduce32<true>(v, lane);
+            }
+            named_bar(1, 256);
+            bool need = false;
+            if (st < 128) {
+                const int h = st;
+                const float m_cta = fmaxf(fmaxf(red[h], red[128 + h]), fmaxf(red[256 + h], red[384 + h]));
+                st_async_f32(xm_peer + 4u * (128 * (b & 1) + h), m_cta, xbar_peer + 8u * (b & 1));
+                if (st == 0) mbar_expect_tx(xbar(b & 1), 128 * 4);
+                const bool okx = mbar_wait_cluster(xbar(b & 1), (b >> 1) & 1);
+                const float m_blk = fmaxf(m_cta, okx ? xm[128 * (b & 1) + h] : m_cta) * sl2;
+                const float m_old = mr[h];
+                need = m_blk > m_old + C::TAU;
+                const float m_new = need ? m_blk : m_old;
+                fs[h] = (need && m_old != -INFINITY) ? exp2f(m_old - m_new) : 1.0f;
+                mr[h] = m_new;
+                if (!okx) misc[1] = 1;
+            }
+            // every exit decision below is taken through a barrier, so the 8 warps stay together
+            const bool any = named_bar_or(1, 256, need);
+            bool pv_waited = false;
+            if (any) {
+#pragma unroll
+                for (int j = 0; j < 64; ++j) l[j] *= fs[64 * h2 + j];
+                if (b > 0) {
+                    // O^T must hold PV_{b-1} before it is rescaled; PV_b cannot start before
+                    // this CTA's P^T arrives below
+                    const bool okp = mbar_wait_cluster(pv_done, (b - 1) & 1);
+                    pv_waited = true;
+                    tc_fence_after();
+                    if (__all_sync(0xffffffffu, okp)) {
+#pragma unroll 1
+                        for (int ch = 0; ch < 4; ++ch) {
+                            uint32_t o[32];
+                            const uint32_t oa = t_lane + C::TMEM_O + 128 * h2 + 32 * ch;
+                            tmem_ld32(oa, o);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * fs[32 * ch + i]);
+                            tmem_st32(oa, o);
+                        }
+                        tmem_wait_st();
+                    }
+                }
+            }
+            // ---- P^T of this thread's key for its 64 heads (bf16 pairs)
+            uint32_t pk[32];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                uint32_t sr[32];
+                tmem_ld32(sb + 32 * j, sr);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float2 m2 = reinterpret_cast<const float2 *>(mr)[32 * h2 + 16 * j + i];
+                    const float p0 = vis ? ex2_approx(fmaf(__uint_as_float(sr[2 * i]), sl2, -m2.x)) : 0.f;
+                    const float p1 = vis ? ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -m2.y)) : 0.f;
+                    l[32 * j + 2 * i] += p0;
+                    l[32 * j + 2 * i + 1] += p1;
+                    pk[16 * j + i] = pack_bf16x2(p0, p1);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(s_free_lead + 8u * (b & 1));   // S^T_b consumed
+            if (b > 0 && !pv_waited) {
+                // PV_{b-1} still reads the P^T buffer
+                const bool okp = mbar_wait_cluster(pv_done, (b - 1) & 1);
+                if (!okp) misc[1] = 1;
+            }
+            {
+                // row 128 cr + key of the P^T buffer of the CTA holding heads 64 h2 .. + 63
+                const uint32_t row = (uint32_t)(128 * cr + key);
+                if (h2 == cr) {
+                    const uint32_t base = p_s + row * 128;
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        st_shared_v4(base + ((u ^ (row & 7)) << 4), pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+                    fence_proxy_async_smem();
+                } else {
+                    const uint32_t base = p_peer_s + row * 128;
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        st_cluster_v4(base + ((u ^ (row & 7)) << 4), pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+                    fence_proxy_async_cluster();
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(p_full_lead);   // this warp's 32 rows are in place
+            if (named_bar_or(1, 256, misc[1] != 0)) { ok = false; break; }
+        }
+        if (!ok && st == 0) abort_pair();
+
+        // ---- epilogue: row sums of the pair, lse, O^T / l transposed into out
+        const int64_t obase = (int64_t)t * 128;
+        if (nblocks > 0 && ok) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                float v[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = l[32 * j + i];
+                red[quarter * 128 + 64 * h2 + 32 * j + lane] = transpose_reduce32<false>(v, lane);
+            }
+            named_bar(1, 256);
+            if (st < 128) {
+                const int h = st;
+                const float l_cta = (red[h] + red[128 + h]) + (red[256 + h] + red[384 + h]);
+                st_async_f32(mapa_shared(sbase + C::OFF_XL + 4u * h, (uint32_t)peer), l_cta,
+                             mapa_shared(lbar, (uint32_t)peer));
+                if (st == 0) mbar_expect_tx(lbar, 128 * 4);
+                const bool okl = mbar_wait_cluster(lbar, 0);
+                // the two CTAs add the same two numbers in the same order
+                const float l_tot = cr == 0 ? l_cta + xl[h] : xl[h] + l_cta;
+                const bool fine = okl && l_tot > 0.f;
+                fs[h] = fine ? 1.0f / l_tot : 0.f;
+                if ((h >> 6) == cr)
+                    lse[obase + h] = okl ? (l_tot > 0.f ? (mr[h] + log2f(l_tot)) * 0.6931471805599453f : -INFINITY) : NAN;
+            }
+            const bool oko = mbar_wait_cluster(o_ready, 0);
+            named_bar(1, 256);
+            tc_fence_after();
+            // O^T block i = h2: lanes = value dims 256 h2 + 128 cr + quarter*32 + lane, columns = heads
+            const uint32_t ostg = ring_s + (uint32_t)h2 * (128 * 256);
+#pragma unroll 1
+            for (int ch = 0; ch < 4; ++ch) {
+                uint32_t o[32];
+                tmem_ld32(t_lane + C::TMEM_O + 128 * h2 + 32 * ch, o);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int h = 32 * ch + i;
+                    const float val = oko ? __uint_as_float(o[i]) * fs[h] : 0.f;
+                    st_shared_u16(ostg + h * 256 + key * 2, __bfloat16_as_ushort(__float2bfloat16_rn(val)));
+                }
+            }
+            fence_proxy_async_smem();
+            named_bar(1, 256);
+            if (st == 0) {
+                prefetch_tmap(&tm_out);
+                for (int i = 0; i < 2; ++i)
+                    tma_store_2d(&tm_out, ring_s + (uint32_t)i * (128 * 256), 256 * i + 128 * cr, (int)obase);
+                bulk_commit();
+                bulk_wait_all();
+            }
+        } else {
+            // no visible slot (or an aborted pipeline): out = 0, lse = -inf (NaN if aborted)
+            for (int e = st; e < 128 * 32; e += 256) {
+                const int h = e >> 5, part = e & 31;          // 32 x 16 bytes per head: the CTA's 2 x 128 dims
+                const int d0 = 256 * (part >> 4) + 128 * cr + 8 * (part & 15);
+                *reinterpret_cast<uint4 *>(out + (obase + h) * 512 + d0) = make_uint4(0, 0, 0, 0);
+            }
+            if (st < 128 && (st >> 6) == cr) lse[obase + st] = nblocks == 0 ? -INFINITY : NAN;
+            if (st == 0) bulk_wait_all();
+        }
+    }
+    // ---- teardown: nothing of either CTA is in flight past this point
+    tc_fence_before();
+    cluster_sync();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, 512);
+    }
+}
+
+}  // namespace mla
+}  // namespace dsa

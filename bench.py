@@ -378,7 +378,7 @@ def _breakdown(dsa, p, inp, fa, chunk, dev, stream, flush, reps=2, decode=False)
         kernels[name]["peak_gbs"] = pk["hbm_gbs"]
     dom = max(kernels, key=lambda k: kernels[k]["ms_per_step"])
     kd = kernels[dom]
-    src = {"indexer": "indexer_tc.cuh", "topk": "topk.cuh", "sparse_mla": "sparse_mla_tc.cuh"}[dom]
+    src = {"indexer": "indexer_tc.cuh", "topk": "topk.cuh", "sparse_mla": "sparse_mla_pair.cuh"}[dom]
     tr = TRAFFIC.get(dom)
     traffic = tr["bytes_per_launch"] if tr and tr.get("src_sha") == _src_sha(src) else None
     if dom == "topk" or decode:
