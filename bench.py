@@ -43,10 +43,10 @@ FLOP_PER_PAIR_MLA = 128 * (576 + 512) * 2       # per (query, selected key) pair
 # sha256 of the source file it was captured from; reported only while the source is
 # unchanged.
 TRAFFIC = {
-    # ncu capture of the 4096-query prefill launch: 1.138 GB of DRAM traffic (q reads and
+    # ncu capture of the 4096-query prefill launch: 1.142 GB of DRAM traffic (q reads and
     # out writes, both proportional to the query count; kv rows come from L2), scaled x8 to
     # the 32768-query launch of the 32K step
-    "sparse_mla": {"bytes_per_launch": 1.1384e9 * 8, "src_sha": "19f132b0bd22c041"},
+    "sparse_mla": {"bytes_per_launch": 1.14244e9 * 8, "src_sha": "2de55da9dd0e8b6b"},
 }
 
 
