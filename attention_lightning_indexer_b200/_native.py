@@ -31,6 +31,7 @@ EXPORTED = (
     "dsa_indexer_scores",
     "dsa_topk",
     "dsa_sparse_mla_fwd",
+    "dsa_dense_mla_fwd",
     "dsa_forward_workspace_size",
     "dsa_forward",
     "dsa_forward_noalloc",
@@ -67,6 +68,9 @@ class DsaProblem(ctypes.Structure):
         ("topk", ctypes.c_int32),
         ("idx_dtype", ctypes.c_int32),
         ("sm_scale", ctypes.c_float),
+        ("block_table", ctypes.c_void_p),
+        ("page_size", ctypes.c_int32),
+        ("max_pages", ctypes.c_int32),
     ]
 
 
@@ -92,6 +96,7 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.dsa_indexer_scores.argtypes = [pp, P, P, P, P, P, P, i64, i32, i32, P]
     lib.dsa_topk.argtypes = [pp, P, i64, i32, i32, P, P]
     lib.dsa_sparse_mla_fwd.argtypes = [pp, P, P, P, P, P, P]
+    lib.dsa_dense_mla_fwd.argtypes = [pp, P, P, P, P, P, P]
     lib.dsa_forward_workspace_size.argtypes = [pp, i32]
     lib.dsa_forward_workspace_size.restype = sz
     lib.dsa_forward.argtypes = [pp, P, P, P, P, P, P, P, i32, P, P, P, P, sz, P]
@@ -103,7 +108,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.dsa_status_string.argtypes = [ctypes.c_int]
     lib.dsa_status_string.restype = ctypes.c_char_p
     lib.dsa_abi_version.restype = i32
-    for name in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_forward", "dsa_forward_noalloc",
+    for name in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_dense_mla_fwd", "dsa_forward",
+                 "dsa_forward_noalloc",
                  "dsa_check_device_errors", "dsa_selftest_bounded_wait"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
@@ -135,21 +141,28 @@ def make_problem(batch: int, total_q: int, total_k: int, max_len_q: int, max_len
                  cu_q: Optional[torch.Tensor] = None, cu_k: Optional[torch.Tensor] = None,
                  idx_dtype: int = DSA_BF16, sm_scale: float = 1.0 / 192 ** 0.5,
                  n_idx_heads: int = 64, idx_dim: int = 128, n_heads: int = 128, d_qk: int = 576,
-                 d_v: int = 512) -> DsaProblem:
+                 d_v: int = 512, block_table: Optional[torch.Tensor] = None, page_size: int = 64) -> DsaProblem:
     if cu_q is not None:
         assert cu_q.dtype == torch.int32 and cu_k is not None and cu_k.dtype == torch.int32
+    max_pages = 0
+    if block_table is not None:
+        assert block_table.dtype == torch.int32 and block_table.dim() == 2
+        max_pages = block_table.shape[1]
     return DsaProblem(batch, _ptr(cu_q), _ptr(cu_k), total_q, total_k, max_len_q, max_len_k, n_idx_heads,
-                      idx_dim, n_heads, d_qk, d_v, topk, idx_dtype, sm_scale)
+                      idx_dim, n_heads, d_qk, d_v, topk, idx_dtype, sm_scale, _ptr(block_table), page_size,
+                      max_pages)
 
 
 def problem_from_inputs(inp: dict, sm_scale: float = 1.0 / 192 ** 0.5) -> DsaProblem:
     """dsa_problem_t for a dict produced by the seeded input generators (tensors on the GPU)."""
     fp8 = "q_idx8" in inp
-    cu_q = inp.get("cu_q") if inp["batch"] > 1 else None
-    cu_k = inp.get("cu_k") if inp["batch"] > 1 else None
-    return make_problem(inp["batch"], inp["total_q"], inp["total_k"], inp["max_len_q"], inp["max_len_k"],
+    paged = "block_table" in inp
+    cu_q = inp.get("cu_q") if inp["batch"] > 1 or paged else None
+    cu_k = inp.get("cu_k") if inp["batch"] > 1 or paged else None
+    total_k = inp["phys_k"] if paged else inp["total_k"]
+    return make_problem(inp["batch"], inp["total_q"], total_k, inp["max_len_q"], inp["max_len_k"],
                         inp["topk"], cu_q=cu_q, cu_k=cu_k, idx_dtype=DSA_E4M3 if fp8 else DSA_BF16,
-                        sm_scale=sm_scale)
+                        sm_scale=sm_scale, block_table=inp.get("block_table"), page_size=inp.get("page_size", 64))
 
 
 def scores_ld(max_len_k: int) -> int:
@@ -180,6 +193,13 @@ def dsa_sparse_mla_fwd(p: DsaProblem, q, kv, idx, out, lse, stream=None) -> None
     lib = load()
     _check(lib.dsa_sparse_mla_fwd(ctypes.byref(p), _ptr(q), _ptr(kv), _ptr(idx), _ptr(out), _ptr(lse),
                                   _stream(stream)), "dsa_sparse_mla_fwd")
+
+
+def dsa_dense_mla_fwd(p: DsaProblem, q, kv, idx, out, lse, stream=None) -> None:
+    """Dense (masked MHA) form: all causal keys, restricted to idx's keys when idx is given."""
+    lib = load()
+    _check(lib.dsa_dense_mla_fwd(ctypes.byref(p), _ptr(q), _ptr(kv), _ptr(idx), _ptr(out), _ptr(lse),
+                                 _stream(stream)), "dsa_dense_mla_fwd")
 
 
 def dsa_forward_workspace_size(p: DsaProblem, chunk_q: int = 0) -> int:

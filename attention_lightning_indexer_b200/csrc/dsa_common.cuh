@@ -17,6 +17,8 @@ struct Problem {
     int total_q, total_k, max_len_q, max_len_k;
     int topk;
     float sm_scale;
+    const int32_t *block_table;   // nullptr: packed rows; else [batch, max_pages] pages of 64 keys
+    int max_pages;
 };
 
 // Sequence facts for one global query row t (the boundary's ragged reading: the
@@ -50,6 +52,17 @@ __device__ __forceinline__ RowInfo row_info(const Problem &P, int t) {
     r.len_k = k1 - k0;
     r.pos = (k1 - k0) - (q1 - q0) + (t - q0);
     return r;
+}
+
+// Row of the key arrays (k_idx, k_scale, kv) that holds key position s of the row's
+// sequence: packed (kbase + s) or through the block table (pages of 64 keys).  A position
+// past the sequence's last page maps to the sequence's first page (only loaded, never used).
+__device__ __forceinline__ int key_row(const Problem &P, const RowInfo &r, int s) {
+    if (P.block_table == nullptr) return r.kbase + s;
+    const int pg = s >> 6;
+    const int npg = (r.len_k + 63) >> 6;
+    const int32_t *tab = P.block_table + (int64_t)r.seq * P.max_pages;
+    return __ldg(tab + (pg < npg ? pg : 0)) * 64 + (s & 63);
 }
 
 // Number of visible keys of a row: keys 0..pos that exist in the sequence.

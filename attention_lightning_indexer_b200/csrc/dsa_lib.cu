@@ -35,6 +35,11 @@ dsa_status_t check_problem(const dsa_problem_t *p) {
     if (p->topk > 2048) return DSA_ERR_UNSUPPORTED;
     if (p->idx_dtype != DSA_BF16 && p->idx_dtype != DSA_E4M3) return DSA_ERR_UNSUPPORTED;
     if (!(p->sm_scale > 0.0f)) return DSA_ERR_INVALID_ARG;
+    if (p->block_table != nullptr) {
+        if (p->cu_q == nullptr || p->max_pages < 1) return DSA_ERR_INVALID_ARG;
+        if (p->page_size != 64) return DSA_ERR_UNSUPPORTED;
+        if ((int64_t)p->max_len_k > (int64_t)p->max_pages * 64 || (p->total_k & 63) != 0) return DSA_ERR_INVALID_ARG;
+    }
     return DSA_OK;
 }
 
@@ -49,6 +54,8 @@ Problem to_dev(const dsa_problem_t *p) {
     P.max_len_k = p->max_len_k;
     P.topk = p->topk;
     P.sm_scale = p->sm_scale;
+    P.block_table = p->block_table;
+    P.max_pages = p->block_table != nullptr ? p->max_pages : 0;
     return P;
 }
 
@@ -119,7 +126,10 @@ dsa_status_t set_smem_attrs() {
         e = cudaFuncSetAttribute(dsa::topk::topk_rows_kernel<512>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  dsa::topk::Cfg<512>::SMEM);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(dsa::mla::sparse_mla_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(dsa::mla::sparse_mla_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 dsa::mla::PairCfg::SMEM);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(dsa::mla::sparse_mla_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  dsa::mla::PairCfg::SMEM);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(dsa::indexer::indexer_tc_kernel<8, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -145,7 +155,8 @@ dsa_status_t indexer_tc_launch(const dsa_problem_t *p, const void *q_idx, const 
     using C = dsa::indexer::TcCfg<QG, FP8>;
     CUtensorMap tq, tk;
     if (!make_tmap_rows(&tq, q_idx, FP8, 128, (uint64_t)p->total_q * 64, 64)) return DSA_ERR_CUDA;
-    if (!make_tmap_rows(&tk, k_idx, FP8, 128, (uint64_t)p->total_k, 128)) return DSA_ERR_CUDA;
+    // key tiles: 128-row boxes, or 64-row boxes (one page) through the block table
+    if (!make_tmap_rows(&tk, k_idx, FP8, 128, (uint64_t)p->total_k, p->block_table ? 64 : 128)) return DSA_ERR_CUDA;
     Problem P = to_dev(p);
     int nsplit = 1;
     unsigned grid;
@@ -196,19 +207,30 @@ dsa_status_t topk_launch(const dsa_problem_t *p, const float *scores, int64_t ld
     return launch_status();
 }
 
+// Sparse (gathered rows of idx) or dense (keys 0 .. pos(t), restricted to idx when idx is
+// given) attention of every query row.
 dsa_status_t mla_launch(const dsa_problem_t *p, const void *q, const void *kv, const int32_t *idx, void *out,
-                        float *lse, cudaStream_t stream) {
+                        float *lse, cudaStream_t stream, bool dense = false) {
     if (p->total_q == 0) return DSA_OK;
     Problem P = to_dev(p);
-    CUtensorMap tq, to;
+    CUtensorMap tq, to, tkv;
     // q: [T*128 rows, 576] read as 64-row boxes of 64 dims (each CTA of a pair loads its 64
     // heads; the latent rows are gathered with cp.async); out: [T*128 rows, 512] written as
     // 128 x 128 tiles
     if (!make_tmap_rows(&tq, q, false, 576, (uint64_t)p->total_q * 128, 64)) return DSA_ERR_CUDA;
     if (!make_tmap_plain_bf16(&to, out, 512, (uint64_t)p->total_q * 128, 128, 128)) return DSA_ERR_CUDA;
-    dsa::mla::sparse_mla_pair_kernel<<<2u * (unsigned)p->total_q, dsa::mla::PairCfg::THREADS,
-                                       dsa::mla::PairCfg::SMEM, stream>>>(
-        tq, to, P, reinterpret_cast<const __nv_bfloat16 *>(kv), idx, reinterpret_cast<__nv_bfloat16 *>(out), lse);
+    const unsigned grid = 2u * (unsigned)p->total_q;
+    const auto *kvb = reinterpret_cast<const __nv_bfloat16 *>(kv);
+    auto *ob = reinterpret_cast<__nv_bfloat16 *>(out);
+    if (dense) {
+        // kv: [S rows, 576] read as 128-row boxes of 64 dims (contiguous keys)
+        if (!make_tmap_rows(&tkv, kv, false, 576, (uint64_t)(p->total_k > 0 ? p->total_k : 1), 128)) return DSA_ERR_CUDA;
+        dsa::mla::sparse_mla_pair_kernel<true><<<grid, dsa::mla::PairCfg::THREADS, dsa::mla::PairCfg::SMEM, stream>>>(
+            tq, to, tkv, P, kvb, idx, ob, lse);
+    } else {
+        dsa::mla::sparse_mla_pair_kernel<false><<<grid, dsa::mla::PairCfg::THREADS, dsa::mla::PairCfg::SMEM, stream>>>(
+            tq, to, tq, P, kvb, idx, ob, lse);
+    }
     return launch_status();
 }
 
@@ -227,6 +249,14 @@ __global__ void bounded_wait_selftest_kernel(uint64_t limit_ns) {
 }
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Key length up to which the fused forward runs the attention in the dense ("masked MHA")
+// form over the selected keys: on B200 its contiguous TMA tile loads beat the row gathers
+// up to here even though it multiplies every causal key (measured 3.79 vs 4.10 ms at 4096
+// keys with index_topk 2048).
+constexpr int DENSE_KV_THRESHOLD = 4096;
+
+bool dense_for(const dsa_problem_t *p) { return p->block_table == nullptr && p->max_len_k <= DENSE_KV_THRESHOLD; }
 
 int64_t scores_ld(const dsa_problem_t *p) { return (int64_t)align_up((size_t)(p->max_len_k > 0 ? p->max_len_k : 1), 4); }
 
@@ -297,6 +327,21 @@ dsa_status_t dsa_sparse_mla_fwd(const dsa_problem_t *p, const void *q, const voi
     return mla_launch(p, q, kv, idx, out, lse, (cudaStream_t)stream);
 }
 
+dsa_status_t dsa_dense_mla_fwd(const dsa_problem_t *p, const void *q, const void *kv, const int32_t *idx, void *out,
+                               float *lse, dsa_stream_t stream) {
+    dsa_status_t st = check_problem(p);
+    if (st != DSA_OK) return st;
+    if (idx != nullptr && p->max_len_k > dsa::mla::PairCfg::DENSE_MAX_KEYS) return DSA_ERR_UNSUPPORTED;
+    if (p->block_table != nullptr) return DSA_ERR_UNSUPPORTED;
+    if (p->total_q > 0) {
+        if (!q || !kv || !out || !lse) return DSA_ERR_INVALID_ARG;
+        if (!aligned16(q) || !aligned16(kv) || !aligned16(out) || !aligned16(lse) || (idx && !aligned16(idx)))
+            return DSA_ERR_INVALID_ARG;
+    }
+    if ((st = set_smem_attrs()) != DSA_OK) return st;
+    return mla_launch(p, q, kv, idx, out, lse, (cudaStream_t)stream, true);
+}
+
 size_t dsa_forward_workspace_size(const dsa_problem_t *p, int32_t chunk_q) {
     if (check_problem(p) != DSA_OK) return 0;
     size_t chunk = (size_t)effective_chunk(p, chunk_q);
@@ -326,6 +371,13 @@ dsa_status_t dsa_forward(const dsa_problem_t *p, const void *q_idx, const float 
     const int chunk = effective_chunk(p, chunk_q);
     const int64_t ld = scores_ld(p);
     float *scores = reinterpret_cast<float *>(workspace);
+    if (p->max_len_k <= p->topk && p->block_table == nullptr) {
+        // Every row has at most topk visible keys, so the selection keeps all of them: no
+        // scores are needed, and the attention runs over the contiguous keys (dense mode,
+        // the same MMAs as the gathered form on the same operands).
+        if (idx_out && (st = topk_launch(p, scores, ld, 0, p->total_q, idx_out, s)) != DSA_OK) return st;
+        return mla_launch(p, q, kv, nullptr, out, lse, s, true);
+    }
     int32_t *idx = idx_out;
     if (!idx) {
         size_t off = align_up((size_t)chunk * (size_t)ld * sizeof(float), 256);
@@ -338,7 +390,7 @@ dsa_status_t dsa_forward(const dsa_problem_t *p, const void *q_idx, const float 
         st = topk_launch(p, scores, ld, r0, rc, idx + (int64_t)r0 * p->topk, s);
         if (st != DSA_OK) return st;
     }
-    return mla_launch(p, q, kv, idx, out, lse, s);
+    return mla_launch(p, q, kv, idx, out, lse, s, dense_for(p));
 }
 
 dsa_status_t dsa_selftest_bounded_wait(uint32_t limit_us, dsa_stream_t stream) {
@@ -422,6 +474,10 @@ extern "C" dsa_status_t dsa_forward_noalloc(const dsa_problem_t *p, const void *
     if ((st = noalloc_scratch(&scores)) != DSA_OK) return st;
     if ((st = set_smem_attrs()) != DSA_OK) return st;
     cudaStream_t s = (cudaStream_t)stream;
+    if (p->max_len_k <= p->topk && p->block_table == nullptr) {   // every visible key is selected
+        if ((st = topk_launch(p, scores, ld, 0, p->total_q, idx_out, s)) != DSA_OK) return st;
+        return mla_launch(p, q, kv, nullptr, out, lse, s, true);
+    }
     for (int r0 = 0; r0 < p->total_q; r0 += chunk) {
         const int rc = p->total_q - r0 < chunk ? p->total_q - r0 : chunk;
         st = indexer_launch(p, q_idx, q_scale, k_idx, k_scale, w, scores, ld, r0, rc, s);
@@ -429,7 +485,7 @@ extern "C" dsa_status_t dsa_forward_noalloc(const dsa_problem_t *p, const void *
         st = topk_launch(p, scores, ld, r0, rc, idx_out + (int64_t)r0 * p->topk, s);
         if (st != DSA_OK) return st;
     }
-    return mla_launch(p, q, kv, idx_out, out, lse, s);
+    return mla_launch(p, q, kv, idx_out, out, lse, s, dense_for(p));
 }
 
 extern "C" size_t dsa_forward_noalloc_scratch_bytes(void) { return NOALLOC_SCRATCH_BYTES; }

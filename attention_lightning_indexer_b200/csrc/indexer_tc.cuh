@@ -71,12 +71,14 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     // ---- which query rows and which key range this CTA owns
     int t0, qcount, kbase, key0, nkeys_total;
     int pos0;   // position of query t0 (queries of a group are consecutive positions)
+    RowInfo rk; // the group's sequence (key rows through key_row when the cache is paged)
     if (QG > 1) {
         const int ngroups = (row_count + QG - 1) / QG;
         const int g = ngroups - 1 - (int)blockIdx.x;          // heaviest (latest) groups first
         t0 = row_begin + g * QG;
         qcount = min(QG, row_begin + row_count - t0);
         const RowInfo ri = row_info(P, t0);                   // single sequence (cu arrays absent)
+        rk = ri;
         kbase = ri.kbase;
         pos0 = ri.pos;
         key0 = 0;
@@ -86,6 +88,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         t0 = row_begin + r;
         qcount = 1;
         const RowInfo ri = row_info(P, t0);
+        rk = ri;
         kbase = ri.kbase;
         pos0 = ri.pos;
         key0 = split * C::SPLIT_KEYS;
@@ -148,9 +151,16 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (j >= C::STAGES && !mbar_wait(k_empty(s), ((j / C::STAGES) - 1) & 1)) { misc[1] = 1; break; }
             if (misc[1]) break;
             mbar_expect_tx(k_full(s), C::KTILE_BYTES);
-            for (int a = 0; a < C::ATOMS; ++a)
-                tma_load_2d(k_s + s * C::KTILE_BYTES + a * C::KATOM_BYTES, &tm_k, k_full(s), a * 128 / C::EB,
-                            kbase + key0 + j * C::BM);
+            const int kk0 = key0 + j * C::BM;
+            for (int a = 0; a < C::ATOMS; ++a) {
+                const uint32_t dst = k_s + s * C::KTILE_BYTES + a * C::KATOM_BYTES;
+                if (P.block_table == nullptr) {
+                    tma_load_2d(dst, &tm_k, k_full(s), a * 128 / C::EB, kbase + kk0);
+                } else {   // a 128-key tile is two pages of 64 rows (the map's box is 64 rows)
+                    tma_load_2d(dst, &tm_k, k_full(s), a * 128 / C::EB, key_row(P, rk, kk0));
+                    tma_load_2d(dst + 64 * 128, &tm_k, k_full(s), a * 128 / C::EB, key_row(P, rk, kk0 + 64));
+                }
+            }
         }
         // drain: the last commits on k_empty must land before the CTA may exit
         for (int j = max(0, ntiles - C::STAGES); j < ntiles && !misc[1]; ++j)
@@ -228,7 +238,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (lane == 0) mbar_arrive(acc_empty(g));
             const int key = key0 + j * C::BM + row;
             float ks = 1.f;
-            if (FP8 && key < nkeys_total) ks = __ldg(k_scale + kbase + key);
+            if (FP8 && key < nkeys_total) ks = __ldg(k_scale + key_row(P, rk, key));
 #pragma unroll
             for (int qi = 0; qi < C::QPI; ++qi) {
                 const int q = h * C::QPI + qi;

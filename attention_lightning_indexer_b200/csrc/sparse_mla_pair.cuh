@@ -41,6 +41,12 @@
 // itself once its copies have landed (wait, proxy fence, cluster-scope arrive), and the
 // softmax warps of both CTAs signal the even CTA's P^T barrier the same way, so no
 // thread relays the odd CTA's state.
+// Dense mode (DENSE = true, the short-sequence "masked MHA" form of the same attention):
+// slot s of block b is key 256 b + s itself, keys 0 .. pos(t) in order, restricted to the
+// keys listed in idx when idx is given (a bitmask built in shared memory; each listed key
+// counts once).  The keys of an atom are contiguous rows, so one thread per CTA loads each
+// atom with a 2-SM TMA tile load that completes on the even CTA's barrier.  With all
+// visible keys listed in order the two modes run the same MMAs on the same operands.
 //
 // Warp roles (16 warps per CTA): 0-6 gather (0 also issues the q TMA and allocates tensor
 // memory), 7 issues the MMAs (even CTA), 8-15 scan the index row, then run the softmax
@@ -69,7 +75,9 @@ struct PairCfg {
     static constexpr int OFF_XL = OFF_XM + 2 * 128 * 4;        // [128] f32, peer row sums
     static constexpr int OFF_MR = OFF_XL + 128 * 4;            // [128] f32, running reference max
     static constexpr int OFF_FS = OFF_MR + 128 * 4;            // [128] f32, rescale factor / 1/l
-    static constexpr int OFF_BAR = OFF_FS + 128 * 4;
+    static constexpr int OFF_MASK = OFF_FS + 128 * 4;          // dense mode: listed-key bitmask
+    static constexpr int DENSE_MAX_KEYS = 16384;               // keys a masked dense row may have
+    static constexpr int OFF_BAR = OFF_MASK + DENSE_MAX_KEYS / 8;
     // (unused)[7] empty[7] pfull[7] q_full q_peer s_full[2] s_free[2] p_full (unused)
     // pv_done o_ready xbar[2] lbar drain
     static constexpr int NBARS = 3 * NSLOT + 2 + 2 + 2 + 2 + 2 + 2 + 1 + 1;
@@ -165,8 +173,10 @@ __device__ __forceinline__ float transpose_reduce32(float (&v)[32], int lane) {
     return v[0];
 }
 
+template <bool DENSE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
-sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_out, Problem P,
+sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_out,
+                       const __grid_constant__ CUtensorMap tm_kv, Problem P,
                        const __nv_bfloat16 *__restrict__ kv, const int32_t *__restrict__ idx,
                        __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
     using C = PairCfg;
@@ -179,7 +189,8 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     const int t = T - 1 - (int)(blockIdx.x >> 1);           // heavier (later) tokens first
     const int K = P.topk;
     const RowInfo ri = row_info(P, t);
-    const int32_t *irow = idx + (int64_t)t * K;
+    const int32_t *irow = idx != nullptr ? idx + (int64_t)t * K : nullptr;
+    const bool masked = DENSE && idx != nullptr;
 
     const uint32_t sbase = smem_u32(smem);
     const bool misaligned = (sbase & 1023u) != 0;           // uniform; checked below without an early exit
@@ -191,6 +202,7 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     float *xl = reinterpret_cast<float *>(smem + C::OFF_XL);
     float *mr = reinterpret_cast<float *>(smem + C::OFF_MR);
     float *fs = reinterpret_cast<float *>(smem + C::OFF_FS);
+    uint32_t *maskw = reinterpret_cast<uint32_t *>(smem + C::OFF_MASK);
     const uint32_t bar0 = sbase + C::OFF_BAR;
     auto empty = [&](int s) { return bar0 + 8u * (C::NSLOT + s); };
     auto pfull = [&](int s) { return bar0 + 8u * (2 * C::NSLOT + s); };
@@ -210,7 +222,8 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     if (tid == 0 && !misaligned) {
         for (int s = 0; s < C::NSLOT; ++s) {
             mbar_init(empty(s), 1);
-            mbar_init(pfull(s), 2);       // the loader warp of this position in each CTA
+            mbar_init(pfull(s), DENSE ? 1 : 2);   // sparse: the loader warp of this position in each
+                                                  // CTA; dense: the even CTA's expect-tx for both
         }
         mbar_init(q_full, 1);
         mbar_init(q_peer, 1);
@@ -239,17 +252,31 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     const int lw = warp;                                     // loader warps 0 .. NLOAD-1
     const bool loader = warp < C::NLOAD;
     int rows[32];
-    if (loader && !misaligned) {
+    if (!DENSE && loader && !misaligned) {
         // the first ring positions (QK_0 atoms 0 .. NSLOT-1 of this CTA's keys) are gathered
         // while the row is scanned
         __syncwarp();
         named_bar(3, 32 * C::NLOAD);
         pair_fetch(irow, K, 128 * cr, lane, rows);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) rows[i] = ri.kbase + (pair_visible(rows[i], ri) ? rows[i] : 0);
+        for (int i = 0; i < 32; ++i) rows[i] = key_row(P, ri, pair_visible(rows[i], ri) ? rows[i] : 0);
         for (int pp = lw; pp < C::NSLOT; pp += C::NLOAD) pair_gather_atom(kv_bytes, rows, pp, ring_s + pp * C::ATOM, lane);
     }
-    if (warp >= C::SOFT0) {   // last visible slot of the row (8 warps, interleaved int4 groups)
+    if (DENSE && warp >= C::SOFT0) {
+        // last visible key; the bitmask of the listed keys (keys 0 .. last)
+        const int part = warp - C::SOFT0;
+        const int last = min(ri.pos, ri.len_k - 1);
+        if (masked && last >= 0) {
+            for (int i = part * 32 + lane; i <= (last >> 5); i += 256) maskw[i] = 0u;
+            named_bar(1, 256);
+            for (int i = part * 32 + lane; i < K; i += 256) {
+                const int e = __ldg(irow + i);
+                if (pair_visible(e, ri)) atomicOr(maskw + (e >> 5), 1u << (e & 31));
+            }
+        }
+        if (lane == 0) reinterpret_cast<int *>(red)[part] = last;
+        if (warp < C::SOFT0 + 4) mr[tid - 32 * C::SOFT0] = -INFINITY;   // reference maxima of the 128 heads
+    } else if (warp >= C::SOFT0) {   // last visible slot of the row (8 warps, interleaved int4 groups)
         int last = -1;
         const int part = warp - C::SOFT0;
         if ((K & 3) == 0) {
@@ -290,7 +317,33 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
 
     if (warp < C::SOFT0) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REG_LOW));
-    if (loader) {
+    if (DENSE && loader) {
+        // ------------------------------------------------ TMA tile loads (one thread per CTA)
+        if (warp == 0 && lane == 0 && nblocks > 0) {
+            const uint32_t lead_pfull = mapa_shared(pfull(0), 0);
+            prefetch_tmap(&tm_kv);
+            bool ok = true;
+            int p = 0;
+            for (int g = 0; ok && g < 2 * nblocks; ++g) {
+                bool qk;
+                int b;
+                pair_group(g, nblocks, qk, b);
+                const int natoms = qk ? C::NATOM : 8;
+                for (int m = 0; m < natoms; ++m) {
+                    const int pp = p + m, slot = pp % C::NSLOT;
+                    if (pp >= C::NSLOT && !mbar_wait(empty(slot), ((pp / C::NSLOT) - 1) & 1)) { ok = false; break; }
+                    if (misc[1]) { ok = false; break; }
+                    const int h = qk ? cr : ((m >> 1) & 1);
+                    const int a = qk ? m : pv_value_atom(cr, p, m);
+                    if (cr == 0) mbar_expect_tx(pfull(slot), 2 * C::ATOM);   // both CTAs' tiles
+                    tma_load_2d_pair(ring_s + slot * C::ATOM, &tm_kv, lead_pfull + 8u * slot, 64 * a,
+                                     ri.kbase + C::BLK * b + 128 * h);
+                }
+                p += natoms;
+            }
+            if (!ok) abort_pair();
+        }
+    } else if (loader) {
         // ------------------------------------------------ gather loaders
         bool ok = true;
         int p = 0, cached = -1;                              // cached: slot base of `rows`
@@ -317,7 +370,7 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 if (s0 != cached) {
                     pair_fetch(irow, K, s0, lane, rows);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) rows[i] = ri.kbase + (pair_visible(rows[i], ri) ? rows[i] : 0);
+                    for (int i = 0; i < 32; ++i) rows[i] = key_row(P, ri, pair_visible(rows[i], ri) ? rows[i] : 0);
                     cached = s0;
                 }
                 const int a = qk ? m : pv_value_atom(cr, p, m);
@@ -427,10 +480,14 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         for (int j = 0; j < 64; ++j) l[j] = 0.f;
         bool ok = true;
         const int sown = 128 * cr + key;                     // slot of this thread's key within a block
-        int ent = nblocks > 0 && sown < K ? __ldg(irow + sown) : -1;
+        int ent = !DENSE && nblocks > 0 && sown < K ? __ldg(irow + sown) : -1;
         for (int b = 0; b < nblocks; ++b) {
-            const bool vis = pair_visible(ent, ri);
-            {
+            bool vis;
+            if (DENSE) {
+                const int sk = C::BLK * b + sown;            // the key itself
+                vis = sk <= ri.pos && sk < ri.len_k && (!masked || ((maskw[sk >> 5] >> (sk & 31)) & 1u));
+            } else {
+                vis = pair_visible(ent, ri);
                 const int s = C::BLK * (b + 1) + sown;
                 ent = (b + 1 < nblocks && s < K) ? __ldg(irow + s) : -1;
             }

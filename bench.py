@@ -315,6 +315,25 @@ def _decode_secondary(dsa, args, rank, dev, stream, flush, dist):
     res = {"workload": "decode_b64", "us_per_step": total_ms / n * 1e3, "steps": n, "batch": inp["batch"],
            "mean_context": float(inp["total_k"]) / inp["batch"], "gpu_launches_per_step": 3,
            "higher_is_better": False}
+    # the same step with the key caches in shuffled 64-token pages (block table)
+    pg = dsa_synth.to_paged(inp, page_size=64, seed=args.seed + 7)
+    pp = dsa.problem_from_inputs(pg)
+    for _ in range(3):
+        dsa.dsa_forward(pp, pg["q_idx"], pg["k_idx"], pg["w"], pg["q"], pg["kv"], out, lse, wsb, chunk_q=0,
+                        stream=stream)
+    torch.cuda.synchronize(dev)
+    _barrier(dist)
+    for i in range(n):
+        flush.zero_()
+        starts[i].record(stream)
+        dsa.dsa_forward(pp, pg["q_idx"], pg["k_idx"], pg["w"], pg["q"], pg["kv"], out, lse, wsb, chunk_q=0,
+                        stream=stream)
+        ends[i].record(stream)
+    torch.cuda.synchronize(dev)
+    _barrier(dist)
+    res["us_per_step_paged_cache"] = _max_over_ranks(dist, sum(s.elapsed_time(e) for s, e in zip(starts, ends))) / n * 1e3
+    dsa.dsa_check_device_errors()
+    del pg
     if rank == 0 and not args.no_breakdown:
         res["roofline"], res["kernels"] = _breakdown(dsa, p, inp, fa, 0, dev, stream, flush, decode=True)
     return res
@@ -612,7 +631,7 @@ def run_kernel(args, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     wl = dsa_synth.WORKLOADS[args.workload]
-    need_latent = args.kernel == "sparse_mla"
+    need_latent = args.kernel in ("sparse_mla", "dense_mla")
     inp = dsa_synth.make_workload(args.workload, seed=args.seed, device=dev, with_latent=need_latent)
     p = dsa.problem_from_inputs(inp)
     fa = _forward_args(inp)
@@ -648,7 +667,10 @@ def run_kernel(args, local):
         out = torch.empty((rows, 128, 512), dtype=torch.bfloat16, device=dev)
         lse = torch.empty((rows, 128), dtype=torch.float32, device=dev)
         ix = idx[r0:]
-        fn = lambda: dsa.dsa_sparse_mla_fwd(sub, q, inp["kv"], ix, out, lse, stream=stream)
+        if args.kernel == "dense_mla":      # the same attention in the dense (masked MHA) form
+            fn = lambda: dsa.dsa_dense_mla_fwd(sub, q, inp["kv"], ix, out, lse, stream=stream)
+        else:
+            fn = lambda: dsa.dsa_sparse_mla_fwd(sub, q, inp["kv"], ix, out, lse, stream=stream)
     for _ in range(args.warmup):
         fn()
     torch.cuda.synchronize(dev)
@@ -680,7 +702,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode_b64 secondary measurement")
     ap.add_argument("--e2e-chunk", type=int, default=2048, help="query rows per pipelined chunk of the e2e step")
-    ap.add_argument("--kernel", choices=("indexer", "topk", "sparse_mla"), default=None,
+    ap.add_argument("--kernel", choices=("indexer", "topk", "sparse_mla", "dense_mla"), default=None,
                     help="time one kernel on a bounded slice (for profilers) instead of the full step")
     ap.add_argument("--rows", type=int, default=0, help="query rows for --kernel (default: one chunk)")
     args = ap.parse_args()

@@ -11,6 +11,7 @@ heads over a 576-d latent = 512 KV-LoRA + 64 RoPE, value = first 512 dims):
 
   ``pr_ref_256``       L=256 prefill, topk 64, q_I,k_I ~ N(0,1), w ~ N(0,1)/8,
                        q, kv ~ N(0,1)/sqrt(576)
+  ``prefill_2k``       L=2048 prefill, topk 2048 (every causal key is selected: short sequence)
   ``prefill_4k``       L=4096 prefill, topk 2048, structured keys (below), q, kv ~ N(0,1)
   ``prefill_32k``      L=32768, otherwise as prefill_4k (the headline workload)
   ``decode_b64``       64 sequences, one query each, context ~ U[8192, 65536]
@@ -57,6 +58,7 @@ class Workload:
 WORKLOADS: Dict[str, Workload] = {
     "pr_ref_256": Workload("pr_ref_256", "prefill", seq_len=256, topk=64, structured_keys=False,
                            latent_std=1.0 / 24.0),
+    "prefill_2k": Workload("prefill_2k", "prefill", seq_len=2048),
     "prefill_4k": Workload("prefill_4k", "prefill", seq_len=4096),
     "prefill_32k": Workload("prefill_32k", "prefill", seq_len=32768, chunk=8192),
     "decode_b64": Workload("decode_b64", "decode", batch=64, ctx_min=8192, ctx_max=65536),
@@ -146,6 +148,47 @@ def make_decode(batch: int, ctx_min: int, ctx_max: int, topk: int = 2048, seed: 
                 w=w.contiguous(), q=q.contiguous(), kv=kv.contiguous(), topk=topk,
                 cu_q=cu_q.to(device), cu_k=cu_k.to(torch.int32).to(device),
                 total_q=T, total_k=S, max_len_q=q_per_seq, max_len_k=int(lens_cpu.max()), batch=batch)
+
+
+def to_paged(inp: dict, page_size: int = 64, seed: int = 0, spare_pages: int = 3) -> dict:
+    """The same problem with its key-side caches (k_idx / k_idx8 + k_scale, kv) laid out in
+    pages of ``page_size`` rows placed in a seeded random order, plus the block table
+    [B, max_pages] int32 that maps logical page j of sequence b to its physical page (-1 for
+    unused entries).  ``spare_pages`` unused pages (filled with noise) are mixed in, so no
+    sequence's pages are contiguous by accident.  Values are copied, never changed."""
+    cu_k = inp["cu_k"].cpu().tolist()
+    B = len(cu_k) - 1
+    lens = [cu_k[b + 1] - cu_k[b] for b in range(B)]
+    npages = [(n + page_size - 1) // page_size for n in lens]
+    max_pages = max(1, max(npages))
+    total = sum(npages) + spare_pages
+    g = torch.Generator().manual_seed(seed)
+    perm = torch.randperm(total, generator=g)
+    table = torch.full((B, max_pages), -1, dtype=torch.int32)
+    j = 0
+    for b in range(B):
+        for pg in range(npages[b]):
+            table[b, pg] = int(perm[j])
+            j += 1
+    out = dict(inp)
+    dev = inp["cu_k"].device
+    for name in ("k_idx", "k_idx8", "k_scale", "kv"):
+        if name not in inp:
+            continue
+        src = inp[name]
+        shape = (total * page_size,) + tuple(src.shape[1:])
+        dst = torch.zeros(shape, dtype=src.dtype, device=src.device)
+        if src.dtype == torch.float32:
+            dst.normal_(generator=torch.Generator(device=src.device).manual_seed(seed + 1))
+        for b in range(B):
+            for pg in range(npages[b]):
+                r0 = cu_k[b] + pg * page_size
+                n = min(page_size, cu_k[b + 1] - r0)
+                d0 = int(table[b, pg]) * page_size
+                dst[d0:d0 + n] = src[r0:r0 + n]
+        out[name] = dst.contiguous()
+    out.update(block_table=table.to(dev), page_size=page_size, max_pages=max_pages, phys_k=total * page_size)
+    return out
 
 
 def make_workload(name: str, seed: int = 0, device="cpu", with_latent: bool = True, **overrides):

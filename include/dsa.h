@@ -24,6 +24,10 @@
  *        pos(t) = len_k(b) - len_q(b) + (t - cu_q[b])
  *    and sees keys 0..pos(t) of its own sequence ("preceding tokens", the token
  *    itself included).  Key indices are positions within the sequence.
+ *  - Paged key caches ("DeepSeek-V3.2" (miles docs) §5.3: the sparse-attention KV cache
+ *    is paged, 64 tokens per page): with a block table, key position s of sequence b is
+ *    the row block_table[b * max_pages + s / 64] * 64 + s % 64 of k_idx, k_scale and kv,
+ *    and cu_k only gives the sequence lengths (len_k(b) = cu_k[b+1] - cu_k[b]).
  *  - Errors: argument, shape and alignment checks run on the host before anything
  *    is launched and return DSA_ERR_INVALID_ARG / DSA_ERR_UNSUPPORTED without side
  *    effects.  A failed launch returns DSA_ERR_CUDA.  Device-side bounded waits that
@@ -40,7 +44,7 @@
 extern "C" {
 #endif
 
-#define DSA_ABI_VERSION 1
+#define DSA_ABI_VERSION 2
 
 /* Same object as cudaStream_t; NULL = the legacy default stream. */
 typedef struct CUstream_st *dsa_stream_t;
@@ -80,6 +84,13 @@ typedef struct dsa_problem {
     int32_t topk;           /* index_topk, e.g. 2048 */
     dsa_dtype_t idx_dtype;  /* indexer inputs: DSA_BF16 or DSA_E4M3 (per-token scales) */
     float sm_scale;         /* attention softmax scale, 1/sqrt(192) for DeepSeek-V3.2 */
+    /* Paged key caches (NULL: packed rows, cu_k gives the row offsets).  With a table,
+     * cu_q / cu_k are required, page_size must be 64, total_k is the number of physical
+     * rows (pages x 64) of k_idx / kv, and every len_k(b) <= max_pages * 64; entries past
+     * a sequence's last page are not read. */
+    const int32_t *block_table;  /* device [B, max_pages] int32 physical page numbers */
+    int32_t page_size;           /* 64 */
+    int32_t max_pages;           /* row stride of block_table */
 } dsa_problem_t;
 
 /*
@@ -138,6 +149,28 @@ dsa_status_t dsa_sparse_mla_fwd(const dsa_problem_t *p, const void *q, const voi
                                 const int32_t *idx, void *out, float *lse, dsa_stream_t stream);
 
 /*
+ * Dense ("masked MHA") form of the same attention, for short sequences ("DeepSeek-V3.2
+ * tech report summary", §1 DSA, short-sequence optimisation: in short prefill, DSA is
+ * simulated by masked MHA, which is more efficient there):
+ *   z[t,h,s]   = sm_scale * q[t,h,:] . kv[kbase(b)+s, :]   for the keys 0 <= s <= pos(t)
+ *   out, lse   as in dsa_sparse_mla_fwd, over those keys
+ * restricted to the keys listed in idx[t, :] when idx is not NULL (each listed visible key
+ * counts once; -1, future and out-of-range entries are ignored).  With idx = NULL every
+ * causal key attends.  For an index row without repeated keys (every dsa_topk row) the
+ * result equals dsa_sparse_mla_fwd on that row.  The keys are read as contiguous tiles, so
+ * the work grows with pos(t) + 1 rather than with topk.
+ *   idx : [T, topk] int32 or NULL; with idx, max_len_k <= 16384 (else DSA_ERR_UNSUPPORTED)
+ * Packed caches only (a block table returns DSA_ERR_UNSUPPORTED).
+ * dsa_forward uses this form (with idx = NULL, skipping the indexer and the top-k) whenever
+ * max_len_k <= topk: every visible key is then selected, and the output is bit-identical
+ * to the gathered form.  Above that, up to max_len_k <= 4096 (the short-sequence threshold
+ * of this build), dsa_forward runs the indexer and the top-k and then this form restricted
+ * to the selected keys; longer problems use dsa_sparse_mla_fwd.
+ */
+dsa_status_t dsa_dense_mla_fwd(const dsa_problem_t *p, const void *q, const void *kv,
+                               const int32_t *idx, void *out, float *lse, dsa_stream_t stream);
+
+/*
  * Bytes of workspace dsa_forward needs for this problem when it processes the
  * queries in chunks of `chunk_q` rows (0 = one chunk of max(T, 1) rows).
  */
@@ -146,7 +179,8 @@ size_t dsa_forward_workspace_size(const dsa_problem_t *p, int32_t chunk_q);
 /*
  * The whole path: for each chunk of chunk_q query rows, indexer scores into the
  * workspace, top-k into idx_out (or the workspace when idx_out is NULL), then the
- * sparse MLA for all rows.  Same tensors and rules as the three calls above; the
+ * attention over the selected keys for all rows (gathered form, or the dense form for
+ * short sequences: see dsa_dense_mla_fwd).  Same tensors and rules as the three calls above; the
  * full T x S score matrix is never materialised (at most chunk_q x max_len_k).
  *   idx_out   : [T, topk] int32 or NULL
  *   workspace : device, >= dsa_forward_workspace_size(p, chunk_q) bytes, 256-byte aligned

@@ -48,12 +48,30 @@ def _load() -> ctypes.CDLL:
         lib.dsa_oracle_e4m3_value.argtypes = [ctypes.c_uint8]
         lib.dsa_oracle_e4m3_value.restype = f64
         lib.dsa_oracle_num_threads.restype = i32
+        lib.dsa_oracle_set_pages.argtypes = [P, i32, i32]
         _lib = lib
     return _lib
 
 
 def num_threads() -> int:
     return int(_load().dsa_oracle_num_threads())
+
+
+class _Pages:
+    """Key rows through a block table (paged caches) for the duration of one call."""
+
+    def __init__(self, block_table, page_size: int):
+        self.table = None if block_table is None else _np(block_table, np.int32)
+        self.page = page_size
+
+    def __enter__(self):
+        if self.table is not None:
+            _load().dsa_oracle_set_pages(_ptr(self.table), self.table.shape[1], self.page)
+        return self
+
+    def __exit__(self, *exc):
+        _load().dsa_oracle_set_pages(None, 0, 0)
+        return False
 
 
 # ---------------------------------------------------------------- marshalling
@@ -93,12 +111,15 @@ def _rows(rows, total_q: int) -> np.ndarray:
 
 # ---------------------------------------------------------------- public calls
 
-def indexer(q_rows, w_rows, k, rows=None, cu_q=None, cu_k=None, ld: Optional[int] = None) -> np.ndarray:
+def indexer(q_rows, w_rows, k, rows=None, cu_q=None, cu_k=None, ld: Optional[int] = None,
+            block_table=None, page_size: int = 64) -> np.ndarray:
     """Index scores I[r, s] for the listed query rows (fp64; -inf where s > pos(t)).
 
     q_rows [R, H, D], w_rows [R, H] are the listed rows' query vectors and weights;
     k [S_total, D].  Without ``cu_q``/``cu_k`` the problem is one sequence with
-    queries = keys (plain prefill).
+    queries = keys (plain prefill).  With ``block_table`` [B, max_pages] the keys are
+    paged: key s of sequence b is row table[b, s // page_size] * page_size + s % page_size
+    of k (``cu_k`` then only gives the sequence lengths).
     """
     q = _np(q_rows, np.float64)
     w = _np(w_rows, np.float64)
@@ -111,13 +132,14 @@ def indexer(q_rows, w_rows, k, rows=None, cu_q=None, cu_k=None, ld: Optional[int
     if ld is None:
         ld = int(np.max(np.diff(cuk))) if batch > 0 else 0
     out = np.empty((R, ld), dtype=np.float64)
-    _load().dsa_oracle_indexer(R, _ptr(rr), _ptr(q), _ptr(w), _ptr(kk), H, D, batch,
-                               _ptr(cuq), _ptr(cuk), _ptr(out), ld)
+    with _Pages(block_table, page_size):
+        _load().dsa_oracle_indexer(R, _ptr(rr), _ptr(q), _ptr(w), _ptr(kk), H, D, batch,
+                                   _ptr(cuq), _ptr(cuk), _ptr(out), ld)
     return out
 
 
 def indexer_fp8(q8_rows, q_scale_rows, w_rows, k8, k_scale, rows=None, cu_q=None, cu_k=None,
-                ld: Optional[int] = None) -> np.ndarray:
+                ld: Optional[int] = None, block_table=None, page_size: int = 64) -> np.ndarray:
     """FP8 (e4m3 codes + per-token fp32 scales) variant of :func:`indexer`."""
     q8 = _np(q8_rows, np.uint8)
     qs = _np(q_scale_rows, np.float64)
@@ -132,8 +154,9 @@ def indexer_fp8(q8_rows, q_scale_rows, w_rows, k8, k_scale, rows=None, cu_q=None
     if ld is None:
         ld = int(np.max(np.diff(cuk))) if batch > 0 else 0
     out = np.empty((R, ld), dtype=np.float64)
-    _load().dsa_oracle_indexer_fp8(R, _ptr(rr), _ptr(q8), _ptr(qs), _ptr(w), _ptr(k8a), _ptr(ks),
-                                   H, D, batch, _ptr(cuq), _ptr(cuk), _ptr(out), ld)
+    with _Pages(block_table, page_size):
+        _load().dsa_oracle_indexer_fp8(R, _ptr(rr), _ptr(q8), _ptr(qs), _ptr(w), _ptr(k8a), _ptr(ks),
+                                       H, D, batch, _ptr(cuq), _ptr(cuk), _ptr(out), ld)
     return out
 
 
@@ -156,7 +179,8 @@ def topk(scores, k: int, rows=None, cu_q=None, cu_k=None) -> np.ndarray:
     return out
 
 
-def sparse_mla(q_rows, kv, idx_rows, scale: float, d_v: int = 512, rows=None, cu_q=None, cu_k=None):
+def sparse_mla(q_rows, kv, idx_rows, scale: float, d_v: int = 512, rows=None, cu_q=None, cu_k=None,
+               block_table=None, page_size: int = 64):
     """Sparse MLA (MQA mode) for the listed rows: returns (o [R,H,d_v], lse [R,H]) in fp64."""
     q = _np(q_rows, np.float64)
     kva = _np(kv, np.float64)
@@ -169,19 +193,22 @@ def sparse_mla(q_rows, kv, idx_rows, scale: float, d_v: int = 512, rows=None, cu
     batch = len(cuk) - 1
     o = np.empty((R, H, d_v), dtype=np.float64)
     lse = np.empty((R, H), dtype=np.float64)
-    _load().dsa_oracle_sparse_mla(R, _ptr(rr), _ptr(q), _ptr(ix), k, _ptr(kva), H, Dqk, d_v,
-                                  float(scale), batch, _ptr(cuq), _ptr(cuk), _ptr(o), _ptr(lse))
+    with _Pages(block_table, page_size):
+        _load().dsa_oracle_sparse_mla(R, _ptr(rr), _ptr(q), _ptr(ix), k, _ptr(kva), H, Dqk, d_v,
+                                      float(scale), batch, _ptr(cuq), _ptr(cuk), _ptr(o), _ptr(lse))
     return o, lse
 
 
 def forward(q_idx_rows, w_rows, k_idx, q_rows, kv, topk_k: int, scale: float, d_v: int = 512,
-            rows=None, cu_q=None, cu_k=None):
+            rows=None, cu_q=None, cu_k=None, block_table=None, page_size: int = 64):
     """The whole path for the listed rows, all in fp64: indexer -> top-k -> sparse MLA.
 
     Returns (scores, idx, o, lse)."""
-    sc = indexer(q_idx_rows, w_rows, k_idx, rows=rows, cu_q=cu_q, cu_k=cu_k)
+    sc = indexer(q_idx_rows, w_rows, k_idx, rows=rows, cu_q=cu_q, cu_k=cu_k, block_table=block_table,
+                 page_size=page_size)
     ix = topk(sc, topk_k, rows=rows, cu_q=cu_q, cu_k=cu_k)
-    o, lse = sparse_mla(q_rows, kv, ix, scale, d_v=d_v, rows=rows, cu_q=cu_q, cu_k=cu_k)
+    o, lse = sparse_mla(q_rows, kv, ix, scale, d_v=d_v, rows=rows, cu_q=cu_q, cu_k=cu_k, block_table=block_table,
+                        page_size=page_size)
     return sc, ix, o, lse
 
 

@@ -34,6 +34,10 @@
  *    latent, lse = natural-log log-sum-exp of z.  A listed index counts once per
  *    occurrence.  A row with no valid index gives o = 0 and lse = -inf.
  *  - FP8 indexer: q = e4m3(q8) * q_scale[t], k = e4m3(k8) * k_scale[s] (per token).
+ *  - Paged caches ("DeepSeek-V3.2" (miles docs) §5.3: the KV cache is paged, 64 tokens per
+ *    page): when a block table is set, key position s of sequence b is the row
+ *    table[b * max_pages + s / page_size] * page_size + s % page_size of the key arrays
+ *    (k, k8 and k_scale, kv); otherwise it is the row cu_k[b] + s.
  *
  * Every function here runs the definition directly, one output element at a time,
  * with OpenMP over query rows.  No blocking, fusion or reordering.
@@ -49,9 +53,19 @@
 
 /* --- ragged-batch bookkeeping (reading stated above) ----------------------- */
 
+/* Block table of the paged layout (NULL: packed rows), set by dsa_oracle_set_pages. */
+static const int32_t *g_table = NULL;
+static int g_max_pages = 0, g_page = 0;
+
+void dsa_oracle_set_pages(const int32_t *table, int max_pages, int page_size) {
+    g_table = table;
+    g_max_pages = max_pages;
+    g_page = page_size;
+}
+
 /* For global query row t, find its sequence b, key-row base and position. */
 static int row_info(int64_t t, int batch, const int32_t *cu_q, const int32_t *cu_k,
-                    int64_t *kbase, int64_t *len_k, int64_t *pos) {
+                    int64_t *kbase, int64_t *len_k, int64_t *pos, int64_t *seq) {
     for (int b = 0; b < batch; ++b) {
         if (t >= cu_q[b] && t < cu_q[b + 1]) {
             int64_t lq = (int64_t)cu_q[b + 1] - cu_q[b];
@@ -59,10 +73,17 @@ static int row_info(int64_t t, int batch, const int32_t *cu_q, const int32_t *cu
             *kbase = cu_k[b];
             *len_k = lk;
             *pos = lk - lq + (t - cu_q[b]);
+            *seq = b;
             return 1;
         }
     }
     return 0;
+}
+
+/* Row of the key arrays that holds key position s of sequence b. */
+static int64_t key_row(int64_t b, int64_t kbase, int64_t s) {
+    if (g_table == NULL) return kbase + s;
+    return (int64_t)g_table[b * g_max_pages + s / g_page] * g_page + s % g_page;
 }
 
 int dsa_oracle_num_threads(void) {
@@ -90,14 +111,14 @@ void dsa_oracle_indexer(int n_rows, const int64_t *rows, const double *q_rows,
                         double *out, int64_t ld) {
 #pragma omp parallel for schedule(dynamic, 1)
     for (int r = 0; r < n_rows; ++r) {
-        int64_t kbase = 0, len_k = 0, pos = -1;
+        int64_t kbase = 0, len_k = 0, pos = -1, seq = 0;
         double *orow = out + (int64_t)r * ld;
         for (int64_t s = 0; s < ld; ++s) orow[s] = -INFINITY;
-        if (!row_info(rows[r], batch, cu_q, cu_k, &kbase, &len_k, &pos)) continue;
+        if (!row_info(rows[r], batch, cu_q, cu_k, &kbase, &len_k, &pos, &seq)) continue;
         const double *qr = q_rows + (int64_t)r * H * D;
         const double *wr = w_rows + (int64_t)r * H;
         for (int64_t s = 0; s <= pos && s < len_k; ++s) {
-            const double *ks = k + (kbase + s) * D;
+            const double *ks = k + key_row(seq, kbase, s) * D;
             double score = 0.0;
             for (int j = 0; j < H; ++j) {
                 double dot = 0.0;
@@ -141,16 +162,16 @@ void dsa_oracle_indexer_fp8(int n_rows, const int64_t *rows, const uint8_t *q8_r
                             double *out, int64_t ld) {
 #pragma omp parallel for schedule(dynamic, 1)
     for (int r = 0; r < n_rows; ++r) {
-        int64_t kbase = 0, len_k = 0, pos = -1;
+        int64_t kbase = 0, len_k = 0, pos = -1, seq = 0;
         double *orow = out + (int64_t)r * ld;
         for (int64_t s = 0; s < ld; ++s) orow[s] = -INFINITY;
-        if (!row_info(rows[r], batch, cu_q, cu_k, &kbase, &len_k, &pos)) continue;
+        if (!row_info(rows[r], batch, cu_q, cu_k, &kbase, &len_k, &pos, &seq)) continue;
         const uint8_t *qr = q8_rows + (int64_t)r * H * D;
         const double *wr = w_rows + (int64_t)r * H;
         double qs = qs_rows[r];
         for (int64_t s = 0; s <= pos && s < len_k; ++s) {
-            const uint8_t *ks = k8 + (kbase + s) * D;
-            double kscale = k_scale[kbase + s];
+            const uint8_t *ks = k8 + key_row(seq, kbase, s) * D;
+            double kscale = k_scale[key_row(seq, kbase, s)];
             double score = 0.0;
             for (int j = 0; j < H; ++j) {
                 double dot = 0.0;
@@ -197,10 +218,10 @@ void dsa_oracle_topk(int n_rows, const int64_t *rows, const double *scores, int6
                      int32_t *idx) {
 #pragma omp parallel for schedule(dynamic, 1)
     for (int r = 0; r < n_rows; ++r) {
-        int64_t kbase = 0, len_k = 0, pos = -1;
+        int64_t kbase = 0, len_k = 0, pos = -1, seq = 0;
         int32_t *irow = idx + (int64_t)r * k;
         for (int j = 0; j < k; ++j) irow[j] = -1;
-        if (!row_info(rows[r], batch, cu_q, cu_k, &kbase, &len_k, &pos)) continue;
+        if (!row_info(rows[r], batch, cu_q, cu_k, &kbase, &len_k, &pos, &seq)) continue;
         int64_t n = pos + 1;
         if (n > len_k) n = len_k;
         if (n <= 0) continue;
@@ -238,12 +259,12 @@ void dsa_oracle_sparse_mla(int n_rows, const int64_t *rows, const double *q_rows
                            double *lse) {
 #pragma omp parallel for schedule(dynamic, 1)
     for (int r = 0; r < n_rows; ++r) {
-        int64_t kbase = 0, len_k = 0, pos = -1;
+        int64_t kbase = 0, len_k = 0, pos = -1, seq = 0;
         double *orow = o + (int64_t)r * H * Dv;
         double *lrow = lse + (int64_t)r * H;
         memset(orow, 0, sizeof(double) * (size_t)H * Dv);
         for (int h = 0; h < H; ++h) lrow[h] = -INFINITY;
-        if (!row_info(rows[r], batch, cu_q, cu_k, &kbase, &len_k, &pos)) continue;
+        if (!row_info(rows[r], batch, cu_q, cu_k, &kbase, &len_k, &pos, &seq)) continue;
         const int32_t *irow = idx_rows + (int64_t)r * k;
         double *z = (double *)malloc(sizeof(double) * (size_t)k);
         for (int h = 0; h < H; ++h) {
@@ -255,7 +276,7 @@ void dsa_oracle_sparse_mla(int n_rows, const int64_t *rows, const double *q_rows
                     z[i] = -INFINITY;
                     continue;
                 }
-                const double *row = kv + (kbase + s) * Dqk;
+                const double *row = kv + key_row(seq, kbase, s) * Dqk;
                 double dot = 0.0;
                 for (int d = 0; d < Dqk; ++d) dot += qh[d] * row[d];
                 z[i] = scale * dot;
@@ -269,7 +290,7 @@ void dsa_oracle_sparse_mla(int n_rows, const int64_t *rows, const double *q_rows
             for (int i = 0; i < k; ++i) {
                 if (z[i] == -INFINITY) continue;
                 double p = exp(z[i] - m) / denom;
-                const double *row = kv + (kbase + irow[i]) * Dqk;
+                const double *row = kv + key_row(seq, kbase, irow[i]) * Dqk;
                 for (int e = 0; e < Dv; ++e) oh[e] += p * row[e];
             }
             lrow[h] = m + log(denom);

@@ -27,7 +27,7 @@ def test_library_exports_every_declared_entry_point():
     for name in declared:
         assert hasattr(lib, name), name
     assert set(declared) == set(_native.EXPORTED)
-    assert lib.dsa_abi_version() == 1
+    assert lib.dsa_abi_version() == 2
 
 
 def test_status_strings():
@@ -64,6 +64,14 @@ def test_unsupported_shapes_are_reported():
     for kw in (dict(n_heads=64), dict(d_qk=192), dict(n_idx_heads=32), dict(idx_dim=64), dict(topk=4096)):
         p = _problem(**kw)
         assert lib.dsa_sparse_mla_fwd(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, None) == 2, kw
+
+
+def test_dense_form_with_index_rows_limits_the_key_count():
+    lib = dsa.load()
+    p = _problem(total_q=64, total_k=20000, max_len_q=64, max_len_k=20000, topk=64)
+    assert lib.dsa_dense_mla_fwd(ctypes.byref(p), FAKE, FAKE, FAKE, FAKE, FAKE, None) == 2
+    p = _problem()
+    assert lib.dsa_dense_mla_fwd(ctypes.byref(p), None, FAKE, None, FAKE, FAKE, None) == 1   # q missing
 
 
 def test_workspace_query_and_too_small_workspace():

@@ -398,3 +398,142 @@ def test_bounded_wait_gives_up_reports_and_clears():
     inp = dsa_synth.make_workload("pr_ref_256", seed=0, device=DEV)
     _check_forward_rows(inp, np.arange(0, 256, 17))
     dsa.dsa_check_device_errors()
+
+
+# ------------------------------------------------- dense (masked MHA) form
+
+def _all_causal_idx(inp, k):
+    """Index rows listing every visible key in order (what the top-k returns when pos + 1 <= k)."""
+    T = inp["total_q"]
+    pos = _positions(inp, np.arange(T))
+    idx = np.full((T, k), -1, dtype=np.int32)
+    for t in range(T):
+        n = min(k, int(pos[t]) + 1)
+        idx[t, :n] = np.arange(n)
+    return idx
+
+
+def _oracle_mla(inp, idx_np):
+    return oracle.sparse_mla(inp["q"].cpu(), inp["kv"].cpu(), idx_np, SCALE, rows=np.arange(inp["total_q"]),
+                             cu_q=inp["cu_q"].cpu().numpy(), cu_k=inp["cu_k"].cpu().numpy())
+
+
+def _assert_mla_close(out, lse, o_ref, lse_ref):
+    assert np.max(np.abs(out.cpu().double().numpy() - o_ref)) <= O_ATOL
+    ls = lse.cpu().double().numpy()
+    fin = np.isfinite(lse_ref)
+    assert np.array_equal(fin, np.isfinite(ls))
+    assert np.max(np.abs(ls[fin] - lse_ref[fin]), initial=0.0) <= LSE_ATOL
+
+
+@pytest.mark.parametrize("L,std", [(300, 1.0), (700, 1 / 24)])
+def test_dense_mla_over_all_causal_keys(L, std):
+    # idx = NULL: every key 0..pos(t) attends -- the oracle's sparse attention over index rows
+    # listing all causal keys (which the pins tie to textbook dense causal attention)
+    inp = dsa_synth.make_prefill(L, topk=L, seed=L + 1, device=DEV, latent_std=std)
+    p = dsa.problem_from_inputs(inp)
+    out = torch.empty((L, 128, 512), dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty((L, 128), dtype=torch.float32, device=DEV)
+    dsa.dsa_dense_mla_fwd(p, inp["q"], inp["kv"], None, out, lse)
+    _assert_mla_close(out, lse, *_oracle_mla(inp, _all_causal_idx(inp, L)))
+
+
+def test_dense_mla_masked_by_index_rows_equals_sparse_attention():
+    # index rows with distinct keys plus ignored entries (a future key, -3): the dense form
+    # restricted to them computes the same attention as the gathered form
+    L, k = 1000, 128
+    inp = dsa_synth.make_prefill(L, topk=k, seed=31, device=DEV)
+    idx_np = _random_idx(inp, k, seed=31)
+    p = dsa.problem_from_inputs(inp)
+    out = torch.empty((L, 128, 512), dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty((L, 128), dtype=torch.float32, device=DEV)
+    dsa.dsa_dense_mla_fwd(p, inp["q"], inp["kv"], torch.from_numpy(idx_np).to(DEV), out, lse)
+    _assert_mla_close(out, lse, *_oracle_mla(inp, idx_np))
+
+
+def test_dense_mla_ragged_decode_masked():
+    inp = dsa_synth.make_decode(5, 300, 3000, topk=256, seed=32, device=DEV)
+    idx_np = _random_idx(inp, 256, seed=32)
+    T = inp["total_q"]
+    p = dsa.problem_from_inputs(inp)
+    out = torch.empty((T, 128, 512), dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty((T, 128), dtype=torch.float32, device=DEV)
+    dsa.dsa_dense_mla_fwd(p, inp["q"], inp["kv"], torch.from_numpy(idx_np).to(DEV), out, lse)
+    _assert_mla_close(out, lse, *_oracle_mla(inp, idx_np))
+
+
+def test_forward_short_sequence_takes_the_dense_path_bit_identically():
+    # max_len_k <= topk: every visible key is selected, so dsa_forward skips the indexer and
+    # the top-k; the result must equal the explicit indexer -> top-k -> gathered path bit for bit
+    L, k = 200, 256
+    inp = dsa_synth.make_prefill(L, topk=k, seed=33, device=DEV)
+    idx_f, out_f, lse_f = _run_forward(inp)
+    p = dsa.problem_from_inputs(inp)
+    sc = _gpu_scores(inp, p)
+    idx = torch.empty((L, k), dtype=torch.int32, device=DEV)
+    dsa.dsa_topk(p, sc, idx)
+    out = torch.empty_like(out_f)
+    lse = torch.empty_like(lse_f)
+    dsa.dsa_sparse_mla_fwd(p, inp["q"], inp["kv"], idx, out, lse)
+    assert torch.equal(idx_f, idx)
+    assert torch.equal(out_f, out) and torch.equal(lse_f, lse)
+    np.testing.assert_array_equal(idx.cpu().numpy(), _all_causal_idx(inp, k))
+    _check_forward_rows(inp, np.arange(0, L, 7))
+
+
+# ------------------------------------------------------- paged key caches
+
+def _paged(inp, seed):
+    pg = dsa_synth.to_paged(inp, page_size=64, seed=seed)
+    assert pg["block_table"].device.type == "cuda"
+    return pg
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_indexer_paged_cache_equals_packed(fp8):
+    inp = dsa_synth.make_decode(5, 150, 1500, topk=64, seed=51, device=DEV, q_per_seq=3)
+    if fp8:
+        q8, qs = dsa_synth.quantize_e4m3_per_token(inp["q_idx"].float())
+        k8, ks = dsa_synth.quantize_e4m3_per_token(inp["k_idx"].float())
+        inp = {kk: v for kk, v in inp.items() if kk not in ("q_idx", "k_idx")}
+        inp.update(q_idx8=q8, q_scale=qs, k_idx8=k8, k_scale=ks)
+    pg = _paged(inp, seed=52)
+    a = _gpu_scores(inp, dsa.problem_from_inputs(inp))
+    b = _gpu_scores(pg, dsa.problem_from_inputs(pg))
+    rows = np.arange(inp["total_q"])
+    pos = _positions(inp, rows)
+    for r in rows:
+        n = int(pos[r]) + 1
+        assert torch.equal(a[r, :n], b[r, :n])
+
+
+def _forward_paged_vs_packed(inp, seed, rows):
+    pg = _paged(inp, seed)
+    idx_a, out_a, lse_a = _run_forward(inp)
+    idx_b, out_b, lse_b = _run_forward(pg)
+    assert torch.equal(idx_a, idx_b)
+    assert torch.equal(out_a, out_b) and torch.equal(lse_a, lse_b)
+    # and against the oracle reading the paged layout through the same block table
+    cu_q = pg["cu_q"].cpu().numpy()
+    cu_k = pg["cu_k"].cpu().numpy()
+    table = pg["block_table"].cpu().numpy()
+    gidx = _host_rows(idx_b, rows).numpy()
+    o_ref, lse_ref = oracle.sparse_mla(_host_rows(pg["q"], rows), pg["kv"].cpu(), gidx, SCALE, rows=rows, cu_q=cu_q,
+                                       cu_k=cu_k, block_table=table)
+    assert np.max(np.abs(_host_rows(out_b, rows).double().numpy() - o_ref)) <= O_ATOL
+    assert np.max(np.abs(_host_rows(lse_b, rows).double().numpy() - lse_ref)) <= LSE_ATOL
+    sc_ref = oracle.indexer(_host_rows(pg["q_idx"], rows), _host_rows(pg["w"], rows), pg["k_idx"].cpu(), rows=rows,
+                            cu_q=cu_q, cu_k=cu_k, ld=pg["max_len_k"], block_table=table)
+    bound = _bound_rows(inp, rows)
+    recall, wrong = recall_excluding_near_ties(gidx, sc_ref, bound, _positions(inp, rows), inp["topk"])
+    assert recall >= RECALL_MIN and wrong == 0, (recall, wrong)
+
+
+def test_forward_paged_decode_small():
+    inp = dsa_synth.make_decode(6, 500, 5000, topk=512, seed=53, device=DEV)
+    _forward_paged_vs_packed(inp, seed=54, rows=np.arange(6))
+
+
+def test_forward_paged_decode_b64_full_size():
+    inp = dsa_synth.make_workload("decode_b64", seed=0, device=DEV)
+    _forward_paged_vs_packed(inp, seed=55, rows=np.array([0, 17, 40, 63]))

@@ -378,3 +378,44 @@ def test_decode_rows_equal_last_prefill_rows():
         np.testing.assert_array_equal(sc[b, :Lb], sc_p[0])
         np.testing.assert_array_equal(ix[b], ix_p[0])
         np.testing.assert_array_equal(o[b], o_p[0])
+
+
+# ------------------------------------------------------------------ paged caches
+
+def test_paged_layout_gives_the_packed_results_exactly():
+    # Paged caches ("DeepSeek-V3.2" miles docs §5.3: KV cache pages of 64 tokens): reading the
+    # keys through a shuffled block table must give bit for bit what the packed rows give, for
+    # every oracle function (the same fp64 operations on the same values).
+    import dsa_synth
+
+    inp = dsa_synth.make_decode(4, 90, 400, topk=32, seed=41, q_per_seq=3)
+    pg = dsa_synth.to_paged(inp, page_size=64, seed=5)
+    assert int(pg["block_table"][0, 1]) != int(pg["block_table"][0, 0]) + 1 or \
+        int(pg["block_table"][1, 0]) != int(pg["block_table"][0, -1]) + 1      # really shuffled
+    kw = dict(cu_q=inp["cu_q"], cu_k=inp["cu_k"])
+    T = inp["total_q"]
+    sc = oracle.indexer(inp["q_idx"], inp["w"], inp["k_idx"], **kw)
+    sc_p = oracle.indexer(inp["q_idx"], inp["w"], pg["k_idx"], block_table=pg["block_table"], **kw)
+    np.testing.assert_array_equal(sc, sc_p)
+    ix = oracle.topk(sc, 32, **kw)
+    o, lse = oracle.sparse_mla(inp["q"], inp["kv"], ix, 0.3, **kw)
+    o_p, lse_p = oracle.sparse_mla(inp["q"], pg["kv"], ix, 0.3, block_table=pg["block_table"], **kw)
+    np.testing.assert_array_equal(o, o_p)
+    np.testing.assert_array_equal(lse, lse_p)
+    full = oracle.forward(inp["q_idx"], inp["w"], pg["k_idx"], inp["q"], pg["kv"], 32, 0.3,
+                          block_table=pg["block_table"], **kw)
+    np.testing.assert_array_equal(full[1], ix)
+    # FP8 keys with per-token scales travel with their rows
+    q8, qs = dsa_synth.quantize_e4m3_per_token(inp["q_idx"].float())
+    k8, ks = dsa_synth.quantize_e4m3_per_token(inp["k_idx"].float())
+    f8 = dict(inp, k_idx8=k8, k_scale=ks)
+    pg8 = dsa_synth.to_paged(f8, page_size=64, seed=6)
+    a = oracle.indexer_fp8(q8, qs, inp["w"], k8, ks, **kw)
+    b = oracle.indexer_fp8(q8, qs, inp["w"], pg8["k_idx8"], pg8["k_scale"], block_table=pg8["block_table"], **kw)
+    np.testing.assert_array_equal(a, b)
+    # and the table really is consulted: a table pointing at the wrong pages changes the scores
+    bad = pg["block_table"].clone()
+    bad[0, 0], bad[0, 1] = bad[0, 1].clone(), bad[0, 0].clone()
+    sc_bad = oracle.indexer(inp["q_idx"], inp["w"], pg["k_idx"], block_table=bad, **kw)
+    assert not np.array_equal(sc_bad[:3], sc[:3])
+    assert T == 12
