@@ -228,8 +228,10 @@ dsa_status_t mla_launch(const dsa_problem_t *p, const void *q, const void *kv, c
         dsa::mla::sparse_mla_pair_kernel<true><<<grid, dsa::mla::PairCfg::THREADS, dsa::mla::PairCfg::SMEM, stream>>>(
             tq, to, tkv, P, kvb, idx, ob, lse);
     } else {
+        // kv: [S rows, 576] gathered 4 rows x 64 dims at a time (one-row boxes)
+        if (!make_tmap_rows(&tkv, kv, false, 576, (uint64_t)(p->total_k > 0 ? p->total_k : 1), 1)) return DSA_ERR_CUDA;
         dsa::mla::sparse_mla_pair_kernel<false><<<grid, dsa::mla::PairCfg::THREADS, dsa::mla::PairCfg::SMEM, stream>>>(
-            tq, to, tq, P, kvb, idx, ob, lse);
+            tq, to, tkv, P, kvb, idx, ob, lse);
     }
     return launch_status();
 }

@@ -35,12 +35,13 @@
 //         64-dim value atoms 4 i + 2 c + {0, 1}.
 // Both CTAs lay the ring out identically (same positions, same slots); the even CTA
 // issues every MMA once both CTAs' operands have landed and commits to the barriers of
-// both.  Gathers are 16-byte cp.async (one warp instruction moves 4 rows x 128 bytes),
-// whose issue rate is about 20 GB/s per warp, so seven loader warps take the ring
-// positions in turn, one slot each; a loader signals the even CTA's barrier of its slot
-// itself once its copies have landed (wait, proxy fence, cluster-scope arrive), and the
-// softmax warps of both CTAs signal the even CTA's P^T barrier the same way, so no
-// thread relays the odd CTA's state.
+// both.  Rows are gathered by TMA (tile::gather4: 4 rows x 128 bytes per instruction, the
+// 128-byte swizzle applied by the copy engine), each lane of a loader warp issuing one
+// instruction of an atom; the 2-SM form completes the bytes of both CTAs on the even
+// CTA's barrier of the slot (one expect-tx by the even CTA), so neither CTA relays the
+// other's ring state.  Seven loader warps take the ring positions in turn, one slot each.
+// The softmax warps of both CTAs signal the even CTA's P^T barrier with cluster-scope
+// arrivals after their stores.
 // Dense mode (DENSE = true, the short-sequence "masked MHA" form of the same attention):
 // slot s of block b is key 256 b + s itself, keys 0 .. pos(t) in order, restricted to the
 // keys listed in idx when idx is given (a bitmask built in shared memory; each listed key
@@ -49,9 +50,10 @@
 // visible keys listed in order the two modes run the same MMAs on the same operands.
 //
 // Warp roles (16 warps per CTA): 0-6 gather (0 also issues the q TMA and allocates tensor
-// memory), 7 issues the MMAs (even CTA), 8-15 scan the index row, then run the softmax
-// and the epilogue: warp w owns TMEM lane quarter w % 4 and head half (w - 8) / 4.  The
-// first two warpgroups give registers to the last two (setmaxnreg).
+// memory; in dense mode only warp 0 loads, one tile per atom), 7 issues the MMAs (even
+// CTA), 8-15 scan the index row, then run the softmax and the epilogue: warp w owns TMEM
+// lane quarter w % 4 and head half (w - 8) / 4.  The first two warpgroups give registers
+// to the last two (setmaxnreg).
 #pragma once
 
 #include "dsa_common.cuh"
@@ -113,47 +115,6 @@ __device__ __forceinline__ int pv_value_atom(int c, int p, int m) {
     const int s1 = (s0 + 1) % PairCfg::NSLOT;
     const bool lo_first = s0 < s1;
     return 4 * i + 2 * c + (lo_first ? e : 1 - e);
-}
-
-// Index entries of slots s0 + 32 (lane / 8) + i, i < 32, of the row (-1 past its end).
-__device__ __forceinline__ void pair_fetch(const int32_t *irow, int K, int s0, int lane, int (&e)[32]) {
-    const int s = s0 + (lane >> 3) * 32;
-    if ((K & 3) == 0 && s + 31 < K) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int4 x = __ldg(reinterpret_cast<const int4 *>(irow + s) + i);
-            e[4 * i] = x.x; e[4 * i + 1] = x.y; e[4 * i + 2] = x.z; e[4 * i + 3] = x.w;
-        }
-    } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) e[i] = s + i < K ? __ldg(irow + s + i) : -1;
-    }
-}
-
-// One atom (32 copy instructions, lane l: 16-byte chunk l % 8 of rows 32 (l / 8) + i)
-// into a ring slot, committed as one cp.async group of the lane.
-__device__ __forceinline__ void pair_gather_atom(const char *kv_bytes, const int (&rows)[32], int a, uint32_t slot,
-                                                 int lane) {
-    using namespace sm100;
-    const int ch = lane & 7;
-    const int r0 = (lane >> 3) * 32;
-    const char *src = kv_bytes + a * 128 + ch * 16;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        const int r = r0 + i;
-        cp_async16(slot + r * 128 + ((ch ^ (r & 7)) << 4), src + (int64_t)rows[i] * 1152);
-    }
-    asm volatile("cp.async.commit_group;" ::: "memory");
-}
-
-// The warp's last atom has landed (all its lanes' copies): make it visible to the tensor
-// core and count it on the even CTA's barrier of its slot.
-__device__ __forceinline__ void pair_signal_atom(uint32_t lead_bar, int lane) {
-    using namespace sm100;
-    cp_async_wait<0>();
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) mbar_arrive_cluster(lead_bar);
 }
 
 // Lane l ends with the reduction (max or sum) over the 32 lanes of element l of v.
@@ -222,8 +183,7 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     if (tid == 0 && !misaligned) {
         for (int s = 0; s < C::NSLOT; ++s) {
             mbar_init(empty(s), 1);
-            mbar_init(pfull(s), DENSE ? 1 : 2);   // sparse: the loader warp of this position in each
-                                                  // CTA; dense: the even CTA's expect-tx for both
+            mbar_init(pfull(s), 1);       // the even CTA's expect-tx for both CTAs' bytes
         }
         mbar_init(q_full, 1);
         mbar_init(q_peer, 1);
@@ -251,17 +211,6 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     const char *kv_bytes = reinterpret_cast<const char *>(kv);
     const int lw = warp;                                     // loader warps 0 .. NLOAD-1
     const bool loader = warp < C::NLOAD;
-    int rows[32];
-    if (!DENSE && loader && !misaligned) {
-        // the first ring positions (QK_0 atoms 0 .. NSLOT-1 of this CTA's keys) are gathered
-        // while the row is scanned
-        __syncwarp();
-        named_bar(3, 32 * C::NLOAD);
-        pair_fetch(irow, K, 128 * cr, lane, rows);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) rows[i] = key_row(P, ri, pair_visible(rows[i], ri) ? rows[i] : 0);
-        for (int pp = lw; pp < C::NSLOT; pp += C::NLOAD) pair_gather_atom(kv_bytes, rows, pp, ring_s + pp * C::ATOM, lane);
-    }
     if (DENSE && warp >= C::SOFT0) {
         // last visible key; the bitmask of the listed keys (keys 0 .. last)
         const int part = warp - C::SOFT0;
@@ -344,15 +293,11 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             if (!ok) abort_pair();
         }
     } else if (loader) {
-        // ------------------------------------------------ gather loaders
+        // ------------------------------------------------ row gathers (TMA, 4 rows per lane)
         bool ok = true;
-        int p = 0, cached = -1;                              // cached: slot base of `rows`
+        int p = 0;
         const uint32_t lead_pfull = mapa_shared(pfull(0), 0);
-        int pend = -1;                                       // slot of this warp's atom in flight
-        if (!misaligned) {
-            cached = 128 * cr;
-            if (lw < C::NSLOT) pend = lw;                    // gathered during the scan
-        }
+        if (lw == 0 && lane == 0) prefetch_tmap(&tm_kv);
         for (int g = 0; ok && g < 2 * nblocks; ++g) {
             bool qk;
             int b;
@@ -360,33 +305,33 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             const int natoms = qk ? C::NATOM : 8;
             for (int m = 0; m < natoms; ++m) {
                 const int pp = p + m;
-                if (pp % C::NLOAD != lw || pp < C::NSLOT) continue;
-                if (pend >= 0) {                             // first: the landed atom (no cycle with the slot wait)
-                    pair_signal_atom(lead_pfull + 8u * pend, lane);
-                    pend = -1;
-                }
+                if (pp % C::NLOAD != lw) continue;
                 const int h = qk ? cr : ((m >> 1) & 1);
-                const int s0 = C::BLK * b + 128 * h;
-                if (s0 != cached) {
-                    pair_fetch(irow, K, s0, lane, rows);
+                const int s0 = C::BLK * b + 128 * h + 4 * lane;   // this lane's 4 slots
+                int e[4];
+                if ((K & 3) == 0 && s0 + 3 < K) {
+                    const int4 x = __ldg(reinterpret_cast<const int4 *>(irow + s0));
+                    e[0] = x.x; e[1] = x.y; e[2] = x.z; e[3] = x.w;
+                } else {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) rows[i] = key_row(P, ri, pair_visible(rows[i], ri) ? rows[i] : 0);
-                    cached = s0;
+                    for (int u = 0; u < 4; ++u) e[u] = s0 + u < K ? __ldg(irow + s0 + u) : -1;
                 }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) e[u] = key_row(P, ri, pair_visible(e[u], ri) ? e[u] : 0);
                 const int a = qk ? m : pv_value_atom(cr, p, m);
                 const int slot = pp % C::NSLOT;
                 bool okw = true;
-                if (lane == 0) okw = mbar_wait(empty(slot), ((pp / C::NSLOT) - 1) & 1);
+                if (lane == 0) {
+                    if (pp >= C::NSLOT) okw = mbar_wait(empty(slot), ((pp / C::NSLOT) - 1) & 1);
+                    if (okw && cr == 0) mbar_expect_tx(pfull(slot), 2 * C::ATOM);   // both CTAs' rows
+                }
                 if (!__shfl_sync(0xffffffffu, okw, 0) || misc[1]) { ok = false; break; }
-                pair_gather_atom(kv_bytes, rows, a, ring_s + slot * C::ATOM, lane);
-                pend = slot;
+                tma_gather4_pair(ring_s + slot * C::ATOM + 512 * lane, &tm_kv, lead_pfull + 8u * slot, 64 * a, e[0],
+                                 e[1], e[2], e[3]);
             }
             p += natoms;
         }
-        if (pend >= 0 && ok && nblocks > 0) pair_signal_atom(lead_pfull + 8u * pend, lane);
         if (!ok && lane == 0) abort_pair();
-        cp_async_wait<0>();
-        if (warp == 0 && lane == 0 && !misaligned) mbar_wait(q_full, 0);   // q landed before exit
     } else if (warp == 7 && lane == 0 && cr == 0 && nblocks > 0) {
         // ------------------------------------------------ MMA issuer (even CTA)
         const uint32_t idesc_qk = idesc_bf16(256, 128);
@@ -461,6 +406,7 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         if (mbar_wait(q_full, 0)) mbar_arrive_cluster(mapa_shared(q_peer, 0));
         else abort_pair();
     }
+    if (warp == 0 && lane == 0 && !misaligned) mbar_wait(q_full, 0);   // q landed before exit
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::REG_HIGH));
         // ------------------------------------------------ softmax + epilogue
