@@ -8,9 +8,11 @@ calls and nothing else.
 from ._native import (  # noqa: F401
     DSA_BF16,
     DSA_E4M3,
+    DSA_E4M3_UE8M0,
     EXPORTED,
     DsaError,
     DsaProblem,
+    dsa_cache_write,
     dsa_check_device_errors,
     dsa_dense_mla_fwd,
     dsa_forward,
@@ -29,8 +31,8 @@ from ._native import (  # noqa: F401
 )
 
 __all__ = [
-    "DSA_BF16", "DSA_E4M3", "DsaError", "DsaProblem", "dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_fwd",
-    "dsa_dense_mla_fwd",
+    "DSA_BF16", "DSA_E4M3", "DSA_E4M3_UE8M0", "DsaError", "DsaProblem", "dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_fwd",
+    "dsa_dense_mla_fwd", "dsa_cache_write",
     "dsa_forward_workspace_size", "dsa_forward", "dsa_forward_noalloc", "dsa_forward_noalloc_scratch_bytes",
     "dsa_check_device_errors", "dsa_selftest_bounded_wait", "make_problem",
     "problem_from_inputs", "scores_ld", "load", "library_path",

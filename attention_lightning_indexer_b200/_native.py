@@ -17,6 +17,7 @@ from . import build as _build
 
 DSA_BF16 = 0
 DSA_E4M3 = 1
+DSA_E4M3_UE8M0 = 2
 
 _STATUS = {
     0: "DSA_OK",
@@ -37,6 +38,7 @@ EXPORTED = (
     "dsa_forward_noalloc",
     "dsa_forward_noalloc_scratch_bytes",
     "dsa_check_device_errors",
+    "dsa_cache_write",
     "dsa_selftest_bounded_wait",
     "dsa_status_string",
     "dsa_abi_version",
@@ -105,12 +107,13 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.dsa_forward_noalloc_scratch_bytes.restype = sz
     lib.dsa_check_device_errors.argtypes = [P]
     lib.dsa_selftest_bounded_wait.argtypes = [ctypes.c_uint32, P]
+    lib.dsa_cache_write.argtypes = [i32, P, P, P, P, P, P, P, P, ctypes.c_float, P, P, P]
     lib.dsa_status_string.argtypes = [ctypes.c_int]
     lib.dsa_status_string.restype = ctypes.c_char_p
     lib.dsa_abi_version.restype = i32
     for name in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_dense_mla_fwd", "dsa_forward",
                  "dsa_forward_noalloc",
-                 "dsa_check_device_errors", "dsa_selftest_bounded_wait"):
+                 "dsa_check_device_errors", "dsa_selftest_bounded_wait", "dsa_cache_write"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -156,12 +159,14 @@ def make_problem(batch: int, total_q: int, total_k: int, max_len_q: int, max_len
 def problem_from_inputs(inp: dict, sm_scale: float = 1.0 / 192 ** 0.5) -> DsaProblem:
     """dsa_problem_t for a dict produced by the seeded input generators (tensors on the GPU)."""
     fp8 = "q_idx8" in inp
+    blocks = "q_scale_ue8m0" in inp
     paged = "block_table" in inp
     cu_q = inp.get("cu_q") if inp["batch"] > 1 or paged else None
     cu_k = inp.get("cu_k") if inp["batch"] > 1 or paged else None
     total_k = inp["phys_k"] if paged else inp["total_k"]
     return make_problem(inp["batch"], inp["total_q"], total_k, inp["max_len_q"], inp["max_len_k"],
-                        inp["topk"], cu_q=cu_q, cu_k=cu_k, idx_dtype=DSA_E4M3 if fp8 else DSA_BF16,
+                        inp["topk"], cu_q=cu_q, cu_k=cu_k,
+                        idx_dtype=(DSA_E4M3_UE8M0 if blocks else DSA_E4M3) if fp8 else DSA_BF16,
                         sm_scale=sm_scale, block_table=inp.get("block_table"), page_size=inp.get("page_size", 64))
 
 
@@ -230,6 +235,15 @@ def dsa_forward_noalloc_scratch_bytes() -> int:
 
 def dsa_check_device_errors(stream=None) -> None:
     _check(load().dsa_check_device_errors(_stream(stream)), "dsa_check_device_errors")
+
+
+def dsa_cache_write(k_idx_raw, kv_raw, positions, rows, k_norm_w, k_norm_b, kv_norm_w, inv_freq, k_idx_cache,
+                    kv_cache, eps: float = 1e-6, stream=None) -> None:
+    """Indexer-key and latent cache rows of new tokens (norms + RoPE; see include/dsa.h)."""
+    lib = load()
+    _check(lib.dsa_cache_write(int(positions.numel()), _ptr(k_idx_raw), _ptr(kv_raw), _ptr(positions), _ptr(rows),
+                               _ptr(k_norm_w), _ptr(k_norm_b), _ptr(kv_norm_w), _ptr(inv_freq), eps,
+                               _ptr(k_idx_cache), _ptr(kv_cache), _stream(stream)), "dsa_cache_write")
 
 
 def dsa_selftest_bounded_wait(limit_us: int = 1000, stream=None) -> None:

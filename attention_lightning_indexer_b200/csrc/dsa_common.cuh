@@ -19,7 +19,16 @@ struct Problem {
     float sm_scale;
     const int32_t *block_table;   // nullptr: packed rows; else [batch, max_pages] pages of 64 keys
     int max_pages;
+    int ue8m0;                    // FP8 indexer scales: 0 fp32 per token, 1 ue8m0 per 128-element block
 };
+
+// Value 2^(e - 127) of a ue8m0 scale byte, built exactly from its bits (e = 0 is the
+// subnormal 2^-127, e = 255 is NaN).
+__device__ __forceinline__ float ue8m0_to_float(uint32_t e) {
+    if (e == 0u) return __uint_as_float(0x00400000u);
+    if (e == 255u) return __uint_as_float(0x7fc00000u);
+    return __uint_as_float(e << 23);
+}
 
 // Sequence facts for one global query row t (the boundary's ragged reading: the
 // queries of a sequence are its last len_q tokens).

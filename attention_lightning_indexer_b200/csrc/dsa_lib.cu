@@ -8,6 +8,7 @@
 #include <string.h>
 
 #include "../../include/dsa.h"
+#include "cache_write.cuh"
 #include "dsa_common.cuh"
 #include "indexer_tc.cuh"
 #include "sparse_mla_pair.cuh"
@@ -33,7 +34,8 @@ dsa_status_t check_problem(const dsa_problem_t *p) {
     if (p->n_idx_heads != 64 || p->idx_dim != 128 || p->n_heads != 128 || p->d_qk != 576 || p->d_v != 512)
         return DSA_ERR_UNSUPPORTED;
     if (p->topk > 2048) return DSA_ERR_UNSUPPORTED;
-    if (p->idx_dtype != DSA_BF16 && p->idx_dtype != DSA_E4M3) return DSA_ERR_UNSUPPORTED;
+    if (p->idx_dtype != DSA_BF16 && p->idx_dtype != DSA_E4M3 && p->idx_dtype != DSA_E4M3_UE8M0)
+        return DSA_ERR_UNSUPPORTED;
     if (!(p->sm_scale > 0.0f)) return DSA_ERR_INVALID_ARG;
     if (p->block_table != nullptr) {
         if (p->cu_q == nullptr || p->max_pages < 1) return DSA_ERR_INVALID_ARG;
@@ -56,6 +58,7 @@ Problem to_dev(const dsa_problem_t *p) {
     P.sm_scale = p->sm_scale;
     P.block_table = p->block_table;
     P.max_pages = p->block_table != nullptr ? p->max_pages : 0;
+    P.ue8m0 = p->idx_dtype == DSA_E4M3_UE8M0 ? 1 : 0;
     return P;
 }
 
@@ -149,8 +152,8 @@ dsa_status_t set_smem_attrs() {
 }
 
 template <int QG, bool FP8>
-dsa_status_t indexer_tc_launch(const dsa_problem_t *p, const void *q_idx, const float *q_scale, const void *k_idx,
-                               const float *k_scale, const float *w, float *scores, int64_t ld, int row_begin,
+dsa_status_t indexer_tc_launch(const dsa_problem_t *p, const void *q_idx, const void *q_scale, const void *k_idx,
+                               const void *k_scale, const float *w, float *scores, int64_t ld, int row_begin,
                                int row_count, cudaStream_t stream) {
     using C = dsa::indexer::TcCfg<QG, FP8>;
     CUtensorMap tq, tk;
@@ -171,11 +174,11 @@ dsa_status_t indexer_tc_launch(const dsa_problem_t *p, const void *q_idx, const 
     return launch_status();
 }
 
-dsa_status_t indexer_launch(const dsa_problem_t *p, const void *q_idx, const float *q_scale, const void *k_idx,
-                            const float *k_scale, const float *w, float *scores, int64_t ld, int row_begin,
+dsa_status_t indexer_launch(const dsa_problem_t *p, const void *q_idx, const void *q_scale, const void *k_idx,
+                            const void *k_scale, const float *w, float *scores, int64_t ld, int row_begin,
                             int row_count, cudaStream_t stream) {
     if (row_count == 0 || p->max_len_k == 0 || p->total_k == 0) return DSA_OK;
-    const bool fp8 = p->idx_dtype == DSA_E4M3;
+    const bool fp8 = p->idx_dtype != DSA_BF16;
     // One sequence: groups of 8 consecutive queries share each key tile.  Ragged batches
     // (decode): one query per CTA, its key range split across CTAs.
     if (p->cu_q == nullptr)
@@ -286,8 +289,8 @@ const char *dsa_status_string(dsa_status_t s) {
 
 int32_t dsa_abi_version(void) { return DSA_ABI_VERSION; }
 
-dsa_status_t dsa_indexer_scores(const dsa_problem_t *p, const void *q_idx, const float *q_scale, const void *k_idx,
-                                const float *k_scale, const float *w, float *scores, int64_t ld_scores,
+dsa_status_t dsa_indexer_scores(const dsa_problem_t *p, const void *q_idx, const void *q_scale, const void *k_idx,
+                                const void *k_scale, const float *w, float *scores, int64_t ld_scores,
                                 int32_t row_begin, int32_t row_count, dsa_stream_t stream) {
     dsa_status_t st = check_problem(p);
     if (st != DSA_OK) return st;
@@ -296,7 +299,7 @@ dsa_status_t dsa_indexer_scores(const dsa_problem_t *p, const void *q_idx, const
     if (row_count > 0) {
         if (!q_idx || !k_idx || !w || !scores) return DSA_ERR_INVALID_ARG;
         if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(w) || !aligned16(scores)) return DSA_ERR_INVALID_ARG;
-        if (p->idx_dtype == DSA_E4M3 && (!q_scale || !k_scale)) return DSA_ERR_INVALID_ARG;
+        if (p->idx_dtype != DSA_BF16 && (!q_scale || !k_scale)) return DSA_ERR_INVALID_ARG;
     }
     if ((st = set_smem_attrs()) != DSA_OK) return st;
     return indexer_launch(p, q_idx, q_scale, k_idx, k_scale, w, scores, ld_scores, row_begin, row_count,
@@ -352,8 +355,8 @@ size_t dsa_forward_workspace_size(const dsa_problem_t *p, int32_t chunk_q) {
     return scores + idx;
 }
 
-dsa_status_t dsa_forward(const dsa_problem_t *p, const void *q_idx, const float *q_scale, const void *k_idx,
-                         const float *k_scale, const float *w, const void *q, const void *kv, int32_t chunk_q,
+dsa_status_t dsa_forward(const dsa_problem_t *p, const void *q_idx, const void *q_scale, const void *k_idx,
+                         const void *k_scale, const float *w, const void *q, const void *kv, int32_t chunk_q,
                          int32_t *idx_out, void *out, float *lse, void *workspace, size_t workspace_bytes,
                          dsa_stream_t stream) {
     dsa_status_t st = check_problem(p);
@@ -364,7 +367,7 @@ dsa_status_t dsa_forward(const dsa_problem_t *p, const void *q_idx, const float 
     if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(w) || !aligned16(q) || !aligned16(kv) ||
         !aligned16(out) || !aligned16(lse) || (idx_out && !aligned16(idx_out)))
         return DSA_ERR_INVALID_ARG;
-    if (p->idx_dtype == DSA_E4M3 && (!q_scale || !k_scale)) return DSA_ERR_INVALID_ARG;
+    if (p->idx_dtype != DSA_BF16 && (!q_scale || !k_scale)) return DSA_ERR_INVALID_ARG;
     const size_t need = dsa_forward_workspace_size(p, chunk_q);
     if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return DSA_ERR_WORKSPACE;
@@ -393,6 +396,22 @@ dsa_status_t dsa_forward(const dsa_problem_t *p, const void *q_idx, const float 
         if (st != DSA_OK) return st;
     }
     return mla_launch(p, q, kv, idx, out, lse, s, dense_for(p));
+}
+
+dsa_status_t dsa_cache_write(int32_t n_tokens, const void *k_idx_raw, const void *kv_raw, const int32_t *positions,
+                             const int32_t *rows, const float *k_norm_w, const float *k_norm_b, const float *kv_norm_w,
+                             const float *inv_freq, float eps, void *k_idx_cache, void *kv_cache, dsa_stream_t stream) {
+    if (n_tokens < 0 || !(eps >= 0.0f)) return DSA_ERR_INVALID_ARG;
+    if (n_tokens == 0) return DSA_OK;
+    const void *ptrs[] = {k_idx_raw, kv_raw, positions, rows, k_norm_w, k_norm_b, kv_norm_w, inv_freq, k_idx_cache, kv_cache};
+    for (const void *q : ptrs)
+        if (q == nullptr || !aligned16(q)) return DSA_ERR_INVALID_ARG;
+    const unsigned grid = (unsigned)((n_tokens + dsa::cache::WARPS - 1) / dsa::cache::WARPS);
+    dsa::cache::cache_write_kernel<<<grid, 32 * dsa::cache::WARPS, 0, (cudaStream_t)stream>>>(
+        n_tokens, reinterpret_cast<const __nv_bfloat16 *>(k_idx_raw), reinterpret_cast<const __nv_bfloat16 *>(kv_raw),
+        positions, rows, k_norm_w, k_norm_b, kv_norm_w, inv_freq, eps, reinterpret_cast<__nv_bfloat16 *>(k_idx_cache),
+        reinterpret_cast<__nv_bfloat16 *>(kv_cache));
+    return launch_status();
 }
 
 dsa_status_t dsa_selftest_bounded_wait(uint32_t limit_us, dsa_stream_t stream) {
@@ -455,8 +474,8 @@ dsa_status_t noalloc_scratch(float **scratch) {
 
 }  // namespace
 
-extern "C" dsa_status_t dsa_forward_noalloc(const dsa_problem_t *p, const void *q_idx, const float *q_scale,
-                                            const void *k_idx, const float *k_scale, const float *w, const void *q,
+extern "C" dsa_status_t dsa_forward_noalloc(const dsa_problem_t *p, const void *q_idx, const void *q_scale,
+                                            const void *k_idx, const void *k_scale, const float *w, const void *q,
                                             const void *kv, int32_t *idx_out, void *out, float *lse,
                                             dsa_stream_t stream) {
     dsa_status_t st = check_problem(p);
@@ -466,7 +485,7 @@ extern "C" dsa_status_t dsa_forward_noalloc(const dsa_problem_t *p, const void *
     if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(w) || !aligned16(q) || !aligned16(kv) ||
         !aligned16(idx_out) || !aligned16(out) || !aligned16(lse))
         return DSA_ERR_INVALID_ARG;
-    if (p->idx_dtype == DSA_E4M3 && (!q_scale || !k_scale)) return DSA_ERR_INVALID_ARG;
+    if (p->idx_dtype != DSA_BF16 && (!q_scale || !k_scale)) return DSA_ERR_INVALID_ARG;
     // rows of scores that fit in the fixed scratch; a single row must fit
     const int64_t ld = scores_ld(p);
     const int64_t rows_fit = (int64_t)(NOALLOC_SCRATCH_BYTES / ((size_t)ld * sizeof(float)));

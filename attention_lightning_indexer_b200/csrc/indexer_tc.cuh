@@ -14,8 +14,10 @@
 //    and sums w[t,j] * ReLU(.) over the 64 heads of a query in registers -- no shuffles;
 //  * the fp32 score row is written coalesced (128 consecutive keys per query); keys past
 //    pos(t) are never written, tiles past the group's last position are never loaded.
-// FP8: kind::f8f6f4 MMA on e4m3 codes; since the per-token scales are positive,
-// ReLU(a*b*x) = a*b*ReLU(x) and the scales multiply the finished sum.
+// FP8: kind::f8f6f4 MMA on e4m3 codes; since the scales are positive, ReLU(a*b*x) =
+// a*b*ReLU(x): per-token scales multiply the finished sum; with ue8m0 block scales (one
+// per head of a query token, one per key token) the query scale of head j joins w[t,j]
+// when the weights are staged and the key scale multiplies the sum.
 //
 // Warp roles (12 warps): 0 TMA producer, 1 MMA issuer, 2 TMEM allocator, 3 idle,
 // 4-7 epilogue for accumulator buffer 0, 8-11 epilogue for buffer 1.
@@ -61,7 +63,7 @@ struct TcCfg {
 template <int QG, bool FP8>
 __global__ void __launch_bounds__(384, 1)
 indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k, Problem P,
-                  const float *__restrict__ q_scale, const float *__restrict__ k_scale, const float *__restrict__ w,
+                  const void *__restrict__ q_scale, const void *__restrict__ k_scale, const float *__restrict__ w,
                   float *__restrict__ scores, int64_t ld, int row_begin, int row_count, int nsplit) {
     using C = TcCfg<QG, FP8>;
     using namespace sm100;
@@ -130,7 +132,10 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (warp == 2) tmem_alloc(sbase + C::OFF_MISC, C::TMEM_COLS);
     for (int i = tid; i < C::QROWS; i += C::THREADS) {
         const int q = i / 64;
-        w_s[i] = q < qcount ? __ldg(w + (int64_t)(t0 + q) * 64 + (i % 64)) : 0.f;
+        float wv = q < qcount ? __ldg(w + (int64_t)(t0 + q) * 64 + (i % 64)) : 0.f;
+        if (FP8 && P.ue8m0 && q < qcount)
+            wv *= ue8m0_to_float(__ldg(reinterpret_cast<const uint8_t *>(q_scale) + (int64_t)(t0 + q) * 64 + (i % 64)));
+        w_s[i] = wv;
     }
     tc_fence_before();
     __syncthreads();
@@ -238,14 +243,18 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (lane == 0) mbar_arrive(acc_empty(g));
             const int key = key0 + j * C::BM + row;
             float ks = 1.f;
-            if (FP8 && key < nkeys_total) ks = __ldg(k_scale + key_row(P, rk, key));
+            if (FP8 && key < nkeys_total) {
+                const int kr = key_row(P, rk, key);
+                ks = P.ue8m0 ? ue8m0_to_float(__ldg(reinterpret_cast<const uint8_t *>(k_scale) + kr))
+                             : __ldg(reinterpret_cast<const float *>(k_scale) + kr);
+            }
 #pragma unroll
             for (int qi = 0; qi < C::QPI; ++qi) {
                 const int q = h * C::QPI + qi;
                 if (q < qcount && key <= pos0 + q && key < nkeys_total) {
                     const int t = t0 + q;
                     float v = res[qi];
-                    if (FP8) v *= __ldg(q_scale + t) * ks;
+                    if (FP8) v *= (P.ue8m0 ? 1.0f : __ldg(reinterpret_cast<const float *>(q_scale) + t)) * ks;
                     scores[(int64_t)(t - row_begin) * ld + key] = v;
                 }
             }

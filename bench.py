@@ -197,8 +197,10 @@ def _tokens(inp):
 
 def _forward_args(inp):
     fp8 = "q_idx8" in inp
+    blocks = "q_scale_ue8m0" in inp
     return dict(q_idx=inp["q_idx8"] if fp8 else inp["q_idx"], k_idx=inp["k_idx8"] if fp8 else inp["k_idx"],
-                q_scale=inp.get("q_scale"), k_scale=inp.get("k_scale"))
+                q_scale=inp["q_scale_ue8m0"] if blocks else inp.get("q_scale"),
+                k_scale=inp["k_scale_ue8m0"] if blocks else inp.get("k_scale"))
 
 
 def run_ours(args, ws, rank, local, dist):
@@ -631,6 +633,8 @@ def run_kernel(args, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     wl = dsa_synth.WORKLOADS[args.workload]
+    if args.kernel == "cache_write":
+        return _run_cache_write(args, dsa, dev)
     need_latent = args.kernel in ("sparse_mla", "dense_mla")
     inp = dsa_synth.make_workload(args.workload, seed=args.seed, device=dev, with_latent=need_latent)
     p = dsa.problem_from_inputs(inp)
@@ -687,6 +691,42 @@ def run_kernel(args, local):
                       "ms_per_launch": ms}), flush=True)
 
 
+def _run_cache_write(args, dsa, dev):
+    """The key-cache write of the workload's tokens (all of them), HBM-bound: per token 256 B +
+    1152 B read and written."""
+    inp = dsa_synth.make_workload(args.workload, seed=args.seed, device=dev, with_latent=True)
+    n = inp["total_k"]
+    g = torch.Generator(device=dev).manual_seed(args.seed)
+    k_raw = torch.randn(n, 128, generator=g, device=dev).to(torch.bfloat16)
+    kv_raw = inp["kv"]
+    pos = torch.arange(n, dtype=torch.int32, device=dev)
+    rows = torch.arange(n, dtype=torch.int32, device=dev)
+    ln_w, ln_b = torch.ones(128, device=dev), torch.zeros(128, device=dev)
+    rms_w = torch.ones(512, device=dev)
+    inv_freq = torch.rand(32, generator=g, device=dev)
+    kc = torch.empty(n, 128, dtype=torch.bfloat16, device=dev)
+    kvc = torch.empty(n, 576, dtype=torch.bfloat16, device=dev)
+    fn = lambda: dsa.dsa_cache_write(k_raw, kv_raw, pos, rows, ln_w, ln_b, rms_w, inv_freq, kc, kvc)  # noqa: E731
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        fn()
+    ts = []
+    for _ in range(args.steps):
+        flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        b.synchronize()
+        ts.append(a.elapsed_time(b))
+    dsa.dsa_check_device_errors()
+    ms = statistics.median(ts)
+    nbytes = n * (2 * (128 + 576) * 2 + 8)
+    print(json.dumps({"kernel": "cache_write", "workload": args.workload, "tokens": n, "ms_per_launch": ms,
+                      "gbs": nbytes / ms / 1e6, "peak_gbs": _peaks()["hbm_gbs"]}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -702,7 +742,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode_b64 secondary measurement")
     ap.add_argument("--e2e-chunk", type=int, default=2048, help="query rows per pipelined chunk of the e2e step")
-    ap.add_argument("--kernel", choices=("indexer", "topk", "sparse_mla", "dense_mla"), default=None,
+    ap.add_argument("--kernel", choices=("indexer", "topk", "sparse_mla", "dense_mla", "cache_write"), default=None,
                     help="time one kernel on a bounded slice (for profilers) instead of the full step")
     ap.add_argument("--rows", type=int, default=0, help="query rows for --kernel (default: one chunk)")
     args = ap.parse_args()

@@ -91,9 +91,28 @@ def quantize_e4m3_per_token(x: torch.Tensor):
     return codes.contiguous(), scale.contiguous()
 
 
+def quantize_e4m3_ue8m0_blocks(x: torch.Tensor):
+    """Block-scaled e4m3 codes: one scale per 128-element block along the last dimension,
+    a power of two stored as a ue8m0 byte (exponent + 127), the smallest power of two not
+    below amax / 448 (so no code saturates); codes = round-to-nearest-even(x / scale).
+    For q_I [T, H, 128] a block is one head of one token, for k_I [S, 128] one token.
+    Returns (codes uint8 like x, scale bytes uint8 [..., blocks])."""
+    assert x.shape[-1] % 128 == 0
+    blocks = x.float().reshape(*x.shape[:-1], x.shape[-1] // 128, 128)
+    amax = blocks.abs().amax(dim=-1)
+    e = torch.ceil(torch.log2(torch.clamp(amax / E4M3_MAX, min=2.0 ** -126))).clamp_(-127, 127)
+    scale = torch.exp2(e)
+    y = (blocks / scale[..., None]).clamp_(-E4M3_MAX, E4M3_MAX)
+    codes = y.to(torch.float8_e4m3fn).view(torch.uint8).reshape(x.shape)
+    sbytes = (e + 127).to(torch.uint8)
+    if x.shape[-1] == 128:
+        sbytes = sbytes[..., 0]
+    return codes.contiguous(), sbytes.contiguous()
+
+
 def make_prefill(L: int, topk: int = 2048, seed: int = 0, device="cpu", structured_keys: bool = True,
                  latent_std: float = 1.0, fp8_indexer: bool = False, T: Optional[int] = None,
-                 with_latent: bool = True):
+                 with_latent: bool = True, fp8_blocks: bool = False):
     """One sequence of L tokens.  T (default L) queries are the last T tokens.
 
     ``with_latent=False`` skips the last draws (q, kv) and leaves the indexer inputs
@@ -115,7 +134,10 @@ def make_prefill(L: int, topk: int = 2048, seed: int = 0, device="cpu", structur
                cu_q=torch.tensor([0, T], dtype=torch.int32, device=device),
                cu_k=torch.tensor([0, L], dtype=torch.int32, device=device),
                total_q=T, total_k=L, max_len_q=T, max_len_k=L, batch=1)
-    if fp8_indexer:
+    if fp8_blocks:
+        out["q_idx8"], out["q_scale_ue8m0"] = quantize_e4m3_ue8m0_blocks(q_idx)
+        out["k_idx8"], out["k_scale_ue8m0"] = quantize_e4m3_ue8m0_blocks(k_idx)
+    elif fp8_indexer:
         out["q_idx8"], out["q_scale"] = quantize_e4m3_per_token(q_idx)
         out["k_idx8"], out["k_scale"] = quantize_e4m3_per_token(k_idx)
     else:

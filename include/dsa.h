@@ -60,7 +60,10 @@ typedef enum dsa_status {
 
 typedef enum dsa_dtype {
     DSA_BF16 = 0,
-    DSA_E4M3 = 1
+    DSA_E4M3 = 1,        /* e4m3 codes, fp32 scale per token (q_scale [T], k_scale [S]) */
+    DSA_E4M3_UE8M0 = 2   /* e4m3 codes, power-of-two scales per 128-element block as ue8m0
+                            bytes (value 2^(e - 127)): q_scale uint8 [T, H_I] (one block per
+                            head of a token), k_scale uint8 [S] (one block per key token) */
 } dsa_dtype_t;
 
 /*
@@ -82,7 +85,7 @@ typedef struct dsa_problem {
     int32_t d_qk;           /* 576 = 512 latent + 64 RoPE */
     int32_t d_v;            /* 512 */
     int32_t topk;           /* index_topk, e.g. 2048 */
-    dsa_dtype_t idx_dtype;  /* indexer inputs: DSA_BF16 or DSA_E4M3 (per-token scales) */
+    dsa_dtype_t idx_dtype;  /* indexer inputs: DSA_BF16, DSA_E4M3 or DSA_E4M3_UE8M0 */
     float sm_scale;         /* attention softmax scale, 1/sqrt(192) for DeepSeek-V3.2 */
     /* Paged key caches (NULL: packed rows, cu_k gives the row offsets).  With a table,
      * cu_q / cu_k are required, page_size must be 64, total_k is the number of physical
@@ -99,20 +102,22 @@ typedef struct dsa_problem {
  *     scores[r, s] = sum_j w[t,j] * ReLU( sum_d q_idx[t,j,d] * k_idx[kbase(b)+s, d] )
  * for query rows t = row_begin + r, 0 <= r < row_count, and 0 <= s <= pos(t).
  * Entries with s > pos(t) are left unspecified (callers must not read them).
- *   q_idx   : [T, H_I, d_I]  bf16, or e4m3 codes when idx_dtype == DSA_E4M3
- *   q_scale : [T]  fp32 per-query-token scale (e4m3 only; NULL for bf16)
+ *   q_idx   : [T, H_I, d_I]  bf16, or e4m3 codes (DSA_E4M3, DSA_E4M3_UE8M0)
+ *   q_scale : DSA_E4M3: fp32 [T] per query token; DSA_E4M3_UE8M0: uint8 [T, H_I] ue8m0
+ *             block scales (one per head of a token); NULL for bf16
  *   k_idx   : [S, d_I]       bf16 or e4m3 codes
- *   k_scale : [S]  fp32 per-key-token scale (e4m3 only; NULL for bf16)
+ *   k_scale : DSA_E4M3: fp32 [S]; DSA_E4M3_UE8M0: uint8 [S] ue8m0; NULL for bf16
  *   w       : [T, H_I] fp32
  *   scores  : [row_count, ld_scores] fp32, ld_scores >= max_len_k, ld_scores % 4 == 0
  * Accumulation is fp32 (tensor cores); the e4m3 scales are applied in fp32.
  * The e4m3 scales must be finite and > 0: the kernel multiplies them into the finished
- * head sum, which equals the definition only because ReLU(a*x) = a*ReLU(x) for a > 0
- * (a non-positive scale gives unspecified scores; they live in device memory, so the
- * host cannot check them).
+ * head sum (a per-head block scale into that head's weight), which equals the definition
+ * only because ReLU(a*x) = a*ReLU(x) for a > 0 (a non-positive fp32 scale gives
+ * unspecified scores; they live in device memory, so the host cannot check them; ue8m0
+ * scales are positive by construction, 0xFF is NaN).
  */
-dsa_status_t dsa_indexer_scores(const dsa_problem_t *p, const void *q_idx, const float *q_scale,
-                                const void *k_idx, const float *k_scale, const float *w,
+dsa_status_t dsa_indexer_scores(const dsa_problem_t *p, const void *q_idx, const void *q_scale,
+                                const void *k_idx, const void *k_scale, const float *w,
                                 float *scores, int64_t ld_scores, int32_t row_begin,
                                 int32_t row_count, dsa_stream_t stream);
 
@@ -185,8 +190,8 @@ size_t dsa_forward_workspace_size(const dsa_problem_t *p, int32_t chunk_q);
  *   idx_out   : [T, topk] int32 or NULL
  *   workspace : device, >= dsa_forward_workspace_size(p, chunk_q) bytes, 256-byte aligned
  */
-dsa_status_t dsa_forward(const dsa_problem_t *p, const void *q_idx, const float *q_scale,
-                         const void *k_idx, const float *k_scale, const float *w, const void *q,
+dsa_status_t dsa_forward(const dsa_problem_t *p, const void *q_idx, const void *q_scale,
+                         const void *k_idx, const void *k_scale, const float *w, const void *q,
                          const void *kv, int32_t chunk_q, int32_t *idx_out, void *out, float *lse,
                          void *workspace, size_t workspace_bytes, dsa_stream_t stream);
 
@@ -208,8 +213,8 @@ dsa_status_t dsa_forward(const dsa_problem_t *p, const void *q_idx, const float 
  * stream capture).  All calls share the array: calls that overlap on the GPU race on it.
  * Nothing is allocated or freed by this call.
  */
-dsa_status_t dsa_forward_noalloc(const dsa_problem_t *p, const void *q_idx, const float *q_scale,
-                                 const void *k_idx, const float *k_scale, const float *w, const void *q,
+dsa_status_t dsa_forward_noalloc(const dsa_problem_t *p, const void *q_idx, const void *q_scale,
+                                 const void *k_idx, const void *k_scale, const float *w, const void *q,
                                  const void *kv, int32_t *idx_out, void *out, float *lse, dsa_stream_t stream);
 
 /* Size in bytes of the fixed scratch array used by dsa_forward_noalloc. */
@@ -221,6 +226,31 @@ size_t dsa_forward_noalloc_scratch_bytes(void);
  * DSA_ERR_DEVICE_TIMEOUT, or DSA_ERR_CUDA if the synchronisation itself failed.
  */
 dsa_status_t dsa_check_device_errors(dsa_stream_t stream);
+
+/*
+ * Key-cache write: the rows the path reads, made from the projections of n new tokens
+ * ("DeepSeek-V3.2-Exp" README, 2025-11-17 note: the indexer's RoPE input is
+ * non-interleaved, MLA's RoPE input interleaved; "Model techniques map -- DeepSeek-V3.2":
+ * the indexer key passes through k_norm, the latent through kv_a_layernorm, RoPE acts on
+ * the 64 RoPE dims):
+ *   k_idx_cache[rows[t]] = RoPE_ni(LayerNorm(k_idx_raw[t]) * k_norm_w + k_norm_b)
+ *                          (LayerNorm over the 128 dims; RoPE on dims 0..63, pairs (i, i + 32))
+ *   kv_cache[rows[t], 0:512]   = kv_raw[t, 0:512] / sqrt(mean(kv_raw[t, 0:512]^2) + eps) * kv_norm_w
+ *   kv_cache[rows[t], 512:576] = RoPE_il(kv_raw[t, 512:576])   (pairs (512 + 2i, 513 + 2i))
+ * where RoPE turns pair i (i < 32) by the angle positions[t] * inv_freq[i] (evaluated in
+ * fp64).  Readings where the pages are silent: k_norm is a LayerNorm with weight and bias,
+ * the indexer's RoPE dims are its first 64, the frequencies are the caller's (any scaled
+ * schedule, e.g. YaRN, is computed once when the model is set up).  Arithmetic in fp32,
+ * outputs rounded to bf16.
+ *   k_idx_raw : [n, 128] bf16      kv_raw : [n, 576] bf16      positions, rows : [n] int32
+ *   k_norm_w, k_norm_b : [128] fp32   kv_norm_w : [512] fp32   inv_freq : [32] fp32
+ *   k_idx_cache : bf16 [.., 128]   kv_cache : bf16 [.., 576]   (rows[t]: the destination
+ *   row, packed or through a block table; distinct rows, no two tokens write the same row)
+ */
+dsa_status_t dsa_cache_write(int32_t n_tokens, const void *k_idx_raw, const void *kv_raw,
+                             const int32_t *positions, const int32_t *rows, const float *k_norm_w,
+                             const float *k_norm_b, const float *kv_norm_w, const float *inv_freq,
+                             float eps, void *k_idx_cache, void *kv_cache, dsa_stream_t stream);
 
 /*
  * Self-test of the device-side failure path (no counterpart on the pages): launches one

@@ -42,13 +42,16 @@ def _load() -> ctypes.CDLL:
         P = ctypes.c_void_p
         i32, i64, f64 = ctypes.c_int, ctypes.c_int64, ctypes.c_double
         lib.dsa_oracle_indexer.argtypes = [i32, P, P, P, P, i32, i32, i32, P, P, P, i64]
-        lib.dsa_oracle_indexer_fp8.argtypes = [i32, P, P, P, P, P, P, i32, i32, i32, P, P, P, i64]
+        lib.dsa_oracle_indexer_fp8.argtypes = [i32, P, P, P, i32, P, P, P, i32, i32, i32, P, P, P, i64]
+        lib.dsa_oracle_ue8m0_value.argtypes = [ctypes.c_uint8]
+        lib.dsa_oracle_ue8m0_value.restype = f64
         lib.dsa_oracle_topk.argtypes = [i32, P, P, i64, i32, i32, P, P, P]
         lib.dsa_oracle_sparse_mla.argtypes = [i32, P, P, P, i32, P, i32, i32, i32, f64, i32, P, P, P, P]
         lib.dsa_oracle_e4m3_value.argtypes = [ctypes.c_uint8]
         lib.dsa_oracle_e4m3_value.restype = f64
         lib.dsa_oracle_num_threads.restype = i32
         lib.dsa_oracle_set_pages.argtypes = [P, i32, i32]
+        lib.dsa_oracle_cache_write.argtypes = [i32, P, P, P, P, P, P, P, f64, P, P]
         _lib = lib
     return _lib
 
@@ -140,9 +143,11 @@ def indexer(q_rows, w_rows, k, rows=None, cu_q=None, cu_k=None, ld: Optional[int
 
 def indexer_fp8(q8_rows, q_scale_rows, w_rows, k8, k_scale, rows=None, cu_q=None, cu_k=None,
                 ld: Optional[int] = None, block_table=None, page_size: int = 64) -> np.ndarray:
-    """FP8 (e4m3 codes + per-token fp32 scales) variant of :func:`indexer`."""
+    """FP8 variant of :func:`indexer`: e4m3 codes with per-token fp32 scales
+    (q_scale_rows [R], k_scale [S]) or per-(token, head) q scales (q_scale_rows [R, H])."""
     q8 = _np(q8_rows, np.uint8)
     qs = _np(q_scale_rows, np.float64)
+    per_head = 1 if qs.ndim == 2 else 0
     w = _np(w_rows, np.float64)
     k8a = _np(k8, np.uint8)
     ks = _np(k_scale, np.float64)
@@ -155,9 +160,25 @@ def indexer_fp8(q8_rows, q_scale_rows, w_rows, k8, k_scale, rows=None, cu_q=None
         ld = int(np.max(np.diff(cuk))) if batch > 0 else 0
     out = np.empty((R, ld), dtype=np.float64)
     with _Pages(block_table, page_size):
-        _load().dsa_oracle_indexer_fp8(R, _ptr(rr), _ptr(q8), _ptr(qs), _ptr(w), _ptr(k8a), _ptr(ks),
+        _load().dsa_oracle_indexer_fp8(R, _ptr(rr), _ptr(q8), _ptr(qs), per_head, _ptr(w), _ptr(k8a), _ptr(ks),
                                        H, D, batch, _ptr(cuq), _ptr(cuk), _ptr(out), ld)
     return out
+
+
+def ue8m0_value(code: int) -> float:
+    return float(_load().dsa_oracle_ue8m0_value(int(code) & 0xFF))
+
+
+def ue8m0_decode(codes) -> np.ndarray:
+    """Scale bytes (ue8m0, any shape) to fp64 values through the oracle's decoder."""
+    c = _np(codes, np.uint8)
+    table = np.array([ue8m0_value(i) for i in range(256)], dtype=np.float64)
+    return table[c]
+
+
+def indexer_fp8_block(q8_rows, q_scale_codes_rows, w_rows, k8, k_scale_codes, **kw) -> np.ndarray:
+    """FP8 indexer with ue8m0 block scales: q_scale_codes_rows [R, H], k_scale_codes [S] bytes."""
+    return indexer_fp8(q8_rows, ue8m0_decode(q_scale_codes_rows), w_rows, k8, ue8m0_decode(k_scale_codes), **kw)
 
 
 def e4m3_value(code: int) -> float:
@@ -221,3 +242,18 @@ def positions(rows: Sequence[int], cu_q, cu_k) -> np.ndarray:
         b = int(np.searchsorted(cuq, t, side="right") - 1)
         out.append((cuk[b + 1] - cuk[b]) - (cuq[b + 1] - cuq[b]) + (t - cuq[b]))
     return np.array(out, dtype=np.int64)
+
+
+def cache_write(k_raw, kv_raw, positions, ln_w, ln_b, rms_w, inv_freq, eps: float):
+    """Indexer key and latent rows of new tokens (k_norm + non-interleaved RoPE; RMSNorm +
+    interleaved RoPE on the latent's RoPE dims): returns (k [n, 128], kv [n, 576]) in fp64."""
+    kr = _np(k_raw, np.float64)
+    zr = _np(kv_raw, np.float64)
+    n = kr.shape[0]
+    ps = _np(positions, np.int32)
+    out_k = np.empty((n, 128), dtype=np.float64)
+    out_kv = np.empty((n, 576), dtype=np.float64)
+    _load().dsa_oracle_cache_write(n, _ptr(kr), _ptr(zr), _ptr(ps), _ptr(_np(ln_w, np.float64)),
+                                   _ptr(_np(ln_b, np.float64)), _ptr(_np(rms_w, np.float64)),
+                                   _ptr(_np(inv_freq, np.float64)), float(eps), _ptr(out_k), _ptr(out_kv))
+    return out_k, out_kv

@@ -33,7 +33,11 @@
  *    the valid listed indices (0 <= idx <= pos(t)), value = first d_v dims of the
  *    latent, lse = natural-log log-sum-exp of z.  A listed index counts once per
  *    occurrence.  A row with no valid index gives o = 0 and lse = -inf.
- *  - FP8 indexer: q = e4m3(q8) * q_scale[t], k = e4m3(k8) * k_scale[s] (per token).
+ *  - FP8 indexer: q = e4m3(q8) * q_scale[t], k = e4m3(k8) * k_scale[s] (per token), or
+ *    with block scales (128-element blocks as in the checkpoint format of "DeepSeek-V3.2"
+ *    (miles docs) §1; a block of q_I is one head of one token, a block of k_I one token):
+ *    q = e4m3(q8) * q_scale[t,j], k = e4m3(k8) * k_scale[s], the scales given as ue8m0
+ *    bytes (8-bit exponents, value 2^(e - 127)).
  *  - Paged caches ("DeepSeek-V3.2" (miles docs) §5.3: the KV cache is paged, 64 tokens per
  *    page): when a block table is set, key position s of sequence b is the row
  *    table[b * max_pages + s / page_size] * page_size + s % page_size of the key arrays
@@ -148,15 +152,23 @@ double dsa_oracle_e4m3_value(uint8_t code) {
     return sign ? -v : v;
 }
 
+/* ue8m0 (an 8-bit unsigned exponent, no sign or mantissa): 2^(e - 127); 0xFF is NaN. */
+double dsa_oracle_ue8m0_value(uint8_t code) {
+    if (code == 0xFF) return NAN;
+    return ldexp(1.0, (int)code - 127);
+}
+
 /*
  * FP8 indexer (section ① of [R], "supports FP8"): the same sum as
- * dsa_oracle_indexer with q[t,j,d] = e4m3(q8) * q_scale[t] and
- * k[s,d] = e4m3(k8) * k_scale[s], decoded here in fp64.
- *   q8_rows : [n_rows, H, D] codes of the listed rows;  qs_rows : [n_rows]
+ * dsa_oracle_indexer with q[t,j,d] = e4m3(q8) * q_scale and
+ * k[s,d] = e4m3(k8) * k_scale[s], decoded here in fp64.  The q scale is per token
+ * (qs_per_head = 0: qs_rows [n_rows]) or per (token, head) block (qs_per_head = 1:
+ * qs_rows [n_rows, H]).
+ *   q8_rows : [n_rows, H, D] codes of the listed rows
  *   k8      : [total_k, D] codes;  k_scale : [total_k]
  */
 void dsa_oracle_indexer_fp8(int n_rows, const int64_t *rows, const uint8_t *q8_rows,
-                            const double *qs_rows, const double *w_rows,
+                            const double *qs_rows, int qs_per_head, const double *w_rows,
                             const uint8_t *k8, const double *k_scale, int H, int D,
                             int batch, const int32_t *cu_q, const int32_t *cu_k,
                             double *out, int64_t ld) {
@@ -168,13 +180,13 @@ void dsa_oracle_indexer_fp8(int n_rows, const int64_t *rows, const uint8_t *q8_r
         if (!row_info(rows[r], batch, cu_q, cu_k, &kbase, &len_k, &pos, &seq)) continue;
         const uint8_t *qr = q8_rows + (int64_t)r * H * D;
         const double *wr = w_rows + (int64_t)r * H;
-        double qs = qs_rows[r];
         for (int64_t s = 0; s <= pos && s < len_k; ++s) {
             const uint8_t *ks = k8 + key_row(seq, kbase, s) * D;
             double kscale = k_scale[key_row(seq, kbase, s)];
             double score = 0.0;
             for (int j = 0; j < H; ++j) {
                 double dot = 0.0;
+                double qs = qs_per_head ? qs_rows[(int64_t)r * H + j] : qs_rows[r];
                 for (int d = 0; d < D; ++d) {
                     double qv = dsa_oracle_e4m3_value(qr[(int64_t)j * D + d]) * qs;
                     double kv = dsa_oracle_e4m3_value(ks[d]) * kscale;
@@ -296,5 +308,57 @@ void dsa_oracle_sparse_mla(int n_rows, const int64_t *rows, const double *q_rows
             lrow[h] = m + log(denom);
         }
         free(z);
+    }
+}
+
+/* --- upstream producer: the key-cache write --------------------------------- */
+
+/*
+ * The rows the path reads, made from the projections of new tokens ("DeepSeek-V3.2-Exp"
+ * README, 2025-11-17 note: the indexer's RoPE takes its input in the non-interleaved
+ * layout, MLA's RoPE in the interleaved one; "Model techniques map -- DeepSeek-V3.2": the
+ * indexer's key passes through k_norm, the latent through kv_a_layernorm, RoPE acts on
+ * the 64 RoPE dims only).  Readings: k_norm is a LayerNorm (mean and variance over the
+ * 128 dims, affine weight and bias), kv_a_layernorm an RMSNorm over the 512 KV-LoRA dims
+ * (weight), eps given; the indexer's RoPE dims are its first 64 (pairs (i, i + 32),
+ * non-interleaved), the latent's are dims 512..575 (pairs (512 + 2i, 513 + 2i),
+ * interleaved); both rotate pair i by the angle pos * inv_freq[i], i < 32.
+ *   k_raw [n, 128], kv_raw [n, 576], pos [n], ln_w/ln_b [128], rms_w [512], inv_freq [32]
+ *   out_k [n, 128], out_kv [n, 576]
+ */
+void dsa_oracle_cache_write(int n, const double *k_raw, const double *kv_raw, const int32_t *pos,
+                            const double *ln_w, const double *ln_b, const double *rms_w,
+                            const double *inv_freq, double eps, double *out_k, double *out_kv) {
+#pragma omp parallel for schedule(static)
+    for (int t = 0; t < n; ++t) {
+        const double *x = k_raw + (int64_t)t * 128;
+        double *y = out_k + (int64_t)t * 128;
+        double mean = 0.0, var = 0.0;
+        for (int d = 0; d < 128; ++d) mean += x[d];
+        mean /= 128.0;
+        for (int d = 0; d < 128; ++d) var += (x[d] - mean) * (x[d] - mean);
+        var /= 128.0;
+        const double inv = 1.0 / sqrt(var + eps);
+        for (int d = 0; d < 128; ++d) y[d] = (x[d] - mean) * inv * ln_w[d] + ln_b[d];
+        for (int i = 0; i < 32; ++i) {          /* non-interleaved: (i, i + 32) */
+            const double a = (double)pos[t] * inv_freq[i];
+            const double c = cos(a), s = sin(a);
+            const double u = y[i], v = y[i + 32];
+            y[i] = u * c - v * s;
+            y[i + 32] = v * c + u * s;
+        }
+        const double *z = kv_raw + (int64_t)t * 576;
+        double *o = out_kv + (int64_t)t * 576;
+        double ms = 0.0;
+        for (int d = 0; d < 512; ++d) ms += z[d] * z[d];
+        const double rinv = 1.0 / sqrt(ms / 512.0 + eps);
+        for (int d = 0; d < 512; ++d) o[d] = z[d] * rinv * rms_w[d];
+        for (int i = 0; i < 32; ++i) {          /* interleaved: (512 + 2i, 513 + 2i) */
+            const double a = (double)pos[t] * inv_freq[i];
+            const double c = cos(a), s = sin(a);
+            const double u = z[512 + 2 * i], v = z[513 + 2 * i];
+            o[512 + 2 * i] = u * c - v * s;
+            o[513 + 2 * i] = v * c + u * s;
+        }
     }
 }

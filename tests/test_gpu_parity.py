@@ -121,9 +121,20 @@ def _host_rows(t, rows):
     return t[torch.as_tensor(np.asarray(rows), device=t.device)].cpu()
 
 
+def _scales(inp):
+    """(q_scale, k_scale) device tensors of an FP8 input set (fp32 per token or ue8m0 blocks)."""
+    if "q_scale_ue8m0" in inp:
+        return inp["q_scale_ue8m0"], inp["k_scale_ue8m0"]
+    return inp.get("q_scale"), inp.get("k_scale")
+
+
 def _oracle_scores(inp, rows):
     cu_q = inp["cu_q"].cpu().numpy()
     cu_k = inp["cu_k"].cpu().numpy()
+    if "q_scale_ue8m0" in inp:
+        return oracle.indexer_fp8_block(_host_rows(inp["q_idx8"], rows), _host_rows(inp["q_scale_ue8m0"], rows),
+                                        _host_rows(inp["w"], rows), inp["k_idx8"].cpu(), inp["k_scale_ue8m0"].cpu(),
+                                        rows=rows, cu_q=cu_q, cu_k=cu_k, ld=inp["max_len_k"])
     if "q_idx8" in inp:
         qr = _host_rows(inp["q_idx8"], rows)
         qs = _host_rows(inp["q_scale"], rows)
@@ -138,17 +149,24 @@ def _bound_rows(inp, rows):
     """Per listed row, the score tolerance scale of its visible keys 0..pos(t)."""
     pos = _positions(inp, rows)
     kb = _kbase(inp, rows)
+    blocks = "q_scale_ue8m0" in inp
     if "q_idx8" in inp:
         q_sel = _host_rows(inp["q_idx8"], rows)
-        qs_sel = _host_rows(inp["q_scale"], rows)
-        k_all = fp8_to_f64(inp["k_idx8"].cpu()) * inp["k_scale"].cpu().double()[:, None]
+        if blocks:
+            qs_sel = _host_rows(inp["q_scale_ue8m0"], rows).view(torch.float8_e8m0fnu).double()
+            k_all = fp8_to_f64(inp["k_idx8"].cpu()) * inp["k_scale_ue8m0"].cpu().view(torch.float8_e8m0fnu).double()[:, None]
+        else:
+            qs_sel = _host_rows(inp["q_scale"], rows)
+            k_all = fp8_to_f64(inp["k_idx8"].cpu()) * inp["k_scale"].cpu().double()[:, None]
     else:
         q_sel = _host_rows(inp["q_idx"], rows)
         k_all = inp["k_idx"].cpu()
     w_sel = _host_rows(inp["w"], rows)
     out = []
     for i, t in enumerate(rows):
-        if "q_idx8" in inp:
+        if "q_idx8" in inp and blocks:
+            qr = fp8_to_f64(q_sel[i]) * qs_sel[i][:, None]
+        elif "q_idx8" in inp:
             qr = fp8_to_f64(q_sel[i]) * float(qs_sel[i])
         else:
             qr = q_sel[i]
@@ -171,8 +189,8 @@ def _gpu_scores(inp, p):
     T = inp["total_q"]
     sc = _scores_buffer(T, inp["max_len_k"])
     if "q_idx8" in inp:
-        dsa.dsa_indexer_scores(p, inp["q_idx8"], inp["k_idx8"], inp["w"], sc, q_scale=inp["q_scale"],
-                               k_scale=inp["k_scale"])
+        qs, ks = _scales(inp)
+        dsa.dsa_indexer_scores(p, inp["q_idx8"], inp["k_idx8"], inp["w"], sc, q_scale=qs, k_scale=ks)
     else:
         dsa.dsa_indexer_scores(p, inp["q_idx"], inp["k_idx"], inp["w"], sc)
     return sc
@@ -195,6 +213,18 @@ def test_indexer_bf16_all_rows(L, seed):
 def test_indexer_fp8_all_rows():
     inp = dsa_synth.make_prefill(700, topk=64, seed=3, device=DEV, fp8_indexer=True)
     _check_indexer(inp, np.arange(700))
+
+
+def test_indexer_fp8_ue8m0_block_scales_all_rows():
+    # e4m3 codes with power-of-two scales per 128-element block (per head of a query token,
+    # per key token), given as ue8m0 bytes
+    inp = dsa_synth.make_prefill(700, topk=64, seed=34, device=DEV, fp8_blocks=True)
+    _check_indexer(inp, np.arange(700))
+
+
+def test_forward_fp8_ue8m0_block_scales():
+    inp = dsa_synth.make_prefill(5000, topk=512, seed=35, device=DEV, fp8_blocks=True)
+    _check_forward_rows(inp, sample_rows(5000, 512, n_rand=24, seed=35, edge=6), chunk=1024)
 
 
 def test_indexer_ragged_batch_several_queries_per_sequence():
@@ -301,9 +331,9 @@ def _run_forward(inp, chunk=0, want_idx=True):
     lse = torch.empty((T, 128), dtype=torch.float32, device=DEV)
     idx = torch.empty((T, inp["topk"]), dtype=torch.int32, device=DEV) if want_idx else None
     fp8 = "q_idx8" in inp
+    qs, ks = _scales(inp)
     dsa.dsa_forward(p, inp["q_idx8"] if fp8 else inp["q_idx"], inp["k_idx8"] if fp8 else inp["k_idx"], inp["w"],
-                    inp["q"], inp["kv"], out, lse, ws, chunk_q=chunk, idx_out=idx,
-                    q_scale=inp.get("q_scale"), k_scale=inp.get("k_scale"))
+                    inp["q"], inp["kv"], out, lse, ws, chunk_q=chunk, idx_out=idx, q_scale=qs, k_scale=ks)
     return idx, out, lse
 
 
@@ -537,3 +567,34 @@ def test_forward_paged_decode_small():
 def test_forward_paged_decode_b64_full_size():
     inp = dsa_synth.make_workload("decode_b64", seed=0, device=DEV)
     _forward_paged_vs_packed(inp, seed=55, rows=np.array([0, 17, 40, 63]))
+
+
+# ------------------------------------------------------ key-cache write producer
+
+def test_cache_write_rows_against_oracle():
+    # new tokens at positions up to 163,839 written to scattered cache rows (as through a
+    # block table); rows that are not written keep their sentinel; tolerance: one bf16
+    # rounding (2^-9 relative) of an fp32 computation, doubled
+    n, cap = 777, 4096
+    g = torch.Generator(device=DEV).manual_seed(81)
+    k_raw = (torch.randn(n, 128, generator=g, device=DEV) * 2 + 0.5).to(torch.bfloat16)
+    kv_raw = torch.randn(n, 576, generator=g, device=DEV).to(torch.bfloat16)
+    pos = torch.randint(0, 163840, (n,), generator=g, device=DEV, dtype=torch.int32)
+    pos[:3] = torch.tensor([0, 1, 163839], dtype=torch.int32, device=DEV)
+    rows = torch.randperm(cap, generator=g, device=DEV)[:n].to(torch.int32)
+    ln_w = torch.rand(128, generator=g, device=DEV) + 0.5
+    ln_b = torch.randn(128, generator=g, device=DEV) * 0.1
+    rms_w = torch.rand(512, generator=g, device=DEV) + 0.5
+    inv_freq = torch.rand(32, generator=g, device=DEV) * 0.9 + 0.01
+    kc = torch.full((cap, 128), 7.0, dtype=torch.bfloat16, device=DEV)
+    kvc = torch.full((cap, 576), 7.0, dtype=torch.bfloat16, device=DEV)
+    dsa.dsa_cache_write(k_raw, kv_raw, pos, rows, ln_w, ln_b, rms_w, inv_freq, kc, kvc, eps=1e-6)
+    ref_k, ref_kv = oracle.cache_write(k_raw.cpu(), kv_raw.cpu(), pos.cpu(), ln_w.cpu(), ln_b.cpu(), rms_w.cpu(),
+                                       inv_freq.cpu(), 1e-6)
+    r = rows.long().cpu()
+    got_k = kc.cpu()[r].double().numpy()
+    got_kv = kvc.cpu()[r].double().numpy()
+    assert np.all(np.abs(got_k - ref_k) <= 2.0 ** -8 * np.abs(ref_k) + 1e-4)
+    assert np.all(np.abs(got_kv - ref_kv) <= 2.0 ** -8 * np.abs(ref_kv) + 1e-4)
+    untouched = np.setdiff1d(np.arange(cap), r.numpy())
+    assert torch.all(kc.cpu()[untouched] == 7.0) and torch.all(kvc.cpu()[untouched] == 7.0)

@@ -419,3 +419,94 @@ def test_paged_layout_gives_the_packed_results_exactly():
     sc_bad = oracle.indexer(inp["q_idx"], inp["w"], pg["k_idx"], block_table=bad, **kw)
     assert not np.array_equal(sc_bad[:3], sc[:3])
     assert T == 12
+
+
+# ------------------------------------------------- FP8 with ue8m0 block scales
+
+def test_ue8m0_decoder_matches_library_cast():
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    lib = codes.view(torch.float8_e8m0fnu).to(torch.float64).numpy()
+    ours = np.array([oracle.ue8m0_value(i) for i in range(256)])
+    assert np.isnan(ours[255]) and np.isnan(lib[255])
+    np.testing.assert_array_equal(ours[:255], lib[:255])
+
+
+def test_block_scaled_fp8_indexer_equals_float_indexer_on_dequantised_inputs():
+    # 128-element blocks: one per (token, head) of q_I, one per token of k_I; scales 2^(e-127)
+    import dsa_synth
+
+    g = torch.Generator().manual_seed(61)
+    T, H, D = 40, 5, 128
+    q = torch.randn(T, H, D, generator=g) * torch.rand(T, H, 1, generator=g).mul(6).exp2()
+    k = torch.randn(T, D, generator=g) * 3.0
+    w = torch.randn(T, H, generator=g)
+    q8, qe = dsa_synth.quantize_e4m3_ue8m0_blocks(q)
+    k8, ke = dsa_synth.quantize_e4m3_ue8m0_blocks(k)
+    assert qe.shape == (T, H) and ke.shape == (T,)
+    got = oracle.indexer_fp8_block(q8, qe, w, k8, ke)
+    lib_q = q8.view(torch.float8_e4m3fn).double() * qe.view(torch.float8_e8m0fnu).double()[:, :, None]
+    lib_k = k8.view(torch.float8_e4m3fn).double() * ke.view(torch.float8_e8m0fnu).double()[:, None]
+    ref = oracle.indexer(lib_q, w, lib_k)
+    tri = np.tril(np.ones((T, T), dtype=bool))
+    np.testing.assert_allclose(got[tri], ref[tri], rtol=1e-12, atol=1e-12)
+    # each head's own scale: raising head 2's exponent by one doubles the score of a row that
+    # weights only head 2 (positive homogeneity of ReLU), and leaves head 3's row unchanged
+    w1 = torch.zeros(T, H)
+    w1[:, 2] = 1.0
+    qe2 = qe.clone()
+    qe2[:, 2] += 1
+    a = oracle.indexer_fp8_block(q8, qe, w1, k8, ke)
+    b = oracle.indexer_fp8_block(q8, qe2, w1, k8, ke)
+    np.testing.assert_array_equal(b[tri], 2.0 * a[tri])
+    w3 = torch.zeros(T, H)
+    w3[:, 3] = 1.0
+    np.testing.assert_array_equal(oracle.indexer_fp8_block(q8, qe2, w3, k8, ke)[tri],
+                                  oracle.indexer_fp8_block(q8, qe, w3, k8, ke)[tri])
+
+
+# ------------------------------------------------------ key-cache write producer
+
+def _cache_inputs(n, seed, positions):
+    g = torch.Generator().manual_seed(seed)
+    k = torch.randn(n, 128, generator=g, dtype=torch.float64) * 2 + 0.5
+    kv = torch.randn(n, 576, generator=g, dtype=torch.float64)
+    ln_w = torch.rand(128, generator=g, dtype=torch.float64) + 0.5
+    ln_b = torch.randn(128, generator=g, dtype=torch.float64) * 0.1
+    rms_w = torch.rand(512, generator=g, dtype=torch.float64) + 0.5
+    inv_freq = torch.rand(32, generator=g, dtype=torch.float64) * 0.9 + 0.01
+    pos = torch.tensor(positions, dtype=torch.int32)
+    return k, kv, pos, ln_w, ln_b, rms_w, inv_freq
+
+
+def test_cache_write_norms_match_library_at_position_zero():
+    # position 0 rotates by nothing: the rows are torch's layer_norm / rms_norm
+    eps = 1e-6
+    k, kv, _, ln_w, ln_b, rms_w, inv_freq = _cache_inputs(6, 71, [0] * 6)
+    ok, okv = oracle.cache_write(k, kv, torch.zeros(6, dtype=torch.int32), ln_w, ln_b, rms_w, inv_freq, eps)
+    ref_k = torch.nn.functional.layer_norm(k, (128,), ln_w, ln_b, eps).numpy()
+    ref_z = torch.nn.functional.rms_norm(kv[:, :512], (512,), rms_w, eps).numpy()
+    np.testing.assert_allclose(ok, ref_k, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(okv[:, :512], ref_z, rtol=1e-12, atol=1e-12)
+    np.testing.assert_array_equal(okv[:, 512:], kv[:, 512:].numpy())
+
+
+def test_cache_write_rope_layouts_are_complex_rotations():
+    # RoPE rotates pair i by pos * inv_freq[i] (multiplication by e^{i theta}); the indexer's
+    # pairs are (i, i + 32) of its first 64 dims (non-interleaved), the latent's are
+    # (512 + 2i, 513 + 2i) (interleaved)
+    eps = 1e-6
+    positions = [1, 7, 100, 4095, 65536, 163839]
+    k, kv, pos, ln_w, ln_b, rms_w, inv_freq = _cache_inputs(len(positions), 72, positions)
+    ok, okv = oracle.cache_write(k, kv, pos, ln_w, ln_b, rms_w, inv_freq, eps)
+    theta = pos.double()[:, None] * inv_freq[None, :]
+    rot = torch.polar(torch.ones_like(theta), theta)
+    normed = torch.nn.functional.layer_norm(k, (128,), ln_w, ln_b, eps)
+    zi = torch.complex(normed[:, :32], normed[:, 32:64]) * rot
+    np.testing.assert_allclose(ok[:, :32], zi.real.numpy(), rtol=1e-9, atol=1e-9)
+    np.testing.assert_allclose(ok[:, 32:64], zi.imag.numpy(), rtol=1e-9, atol=1e-9)
+    np.testing.assert_allclose(ok[:, 64:], normed[:, 64:].numpy(), rtol=1e-12, atol=1e-12)
+    zl = torch.view_as_complex(kv[:, 512:].reshape(-1, 32, 2).contiguous()) * rot
+    np.testing.assert_allclose(okv[:, 512:], torch.view_as_real(zl).reshape(-1, 64).numpy(), rtol=1e-9, atol=1e-9)
+    # the two layouts really differ: rotating the latent's dims non-interleaved would not match
+    wrong = torch.complex(kv[:, 512:544], kv[:, 544:576]) * rot
+    assert not np.allclose(okv[:, 512:544], wrong.real.numpy(), atol=1e-6)
