@@ -22,6 +22,7 @@ from ._native import (  # noqa: F401
     dsa_indexer_scores,
     dsa_sparse_mla_fwd,
     dsa_selftest_bounded_wait,
+    dsa_set_debug_checks,
     dsa_topk,
     library_path,
     load,
@@ -34,6 +35,6 @@ __all__ = [
     "DSA_BF16", "DSA_E4M3", "DSA_E4M3_UE8M0", "DsaError", "DsaProblem", "dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_fwd",
     "dsa_dense_mla_fwd", "dsa_cache_write",
     "dsa_forward_workspace_size", "dsa_forward", "dsa_forward_noalloc", "dsa_forward_noalloc_scratch_bytes",
-    "dsa_check_device_errors", "dsa_selftest_bounded_wait", "make_problem",
+    "dsa_check_device_errors", "dsa_selftest_bounded_wait", "dsa_set_debug_checks", "make_problem",
     "problem_from_inputs", "scores_ld", "load", "library_path",
 ]

@@ -26,6 +26,7 @@ _STATUS = {
     3: "DSA_ERR_WORKSPACE",
     4: "DSA_ERR_CUDA",
     5: "DSA_ERR_DEVICE_TIMEOUT",
+    6: "DSA_ERR_DEVICE_BOUNDS",
 }
 
 EXPORTED = (
@@ -39,6 +40,7 @@ EXPORTED = (
     "dsa_forward_noalloc_scratch_bytes",
     "dsa_check_device_errors",
     "dsa_cache_write",
+    "dsa_set_debug_checks",
     "dsa_selftest_bounded_wait",
     "dsa_status_string",
     "dsa_abi_version",
@@ -108,6 +110,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.dsa_check_device_errors.argtypes = [P]
     lib.dsa_selftest_bounded_wait.argtypes = [ctypes.c_uint32, P]
     lib.dsa_cache_write.argtypes = [i32, P, P, P, P, P, P, P, P, ctypes.c_float, P, P, P]
+    lib.dsa_set_debug_checks.argtypes = [i32]
+    lib.dsa_set_debug_checks.restype = None
     lib.dsa_status_string.argtypes = [ctypes.c_int]
     lib.dsa_status_string.restype = ctypes.c_char_p
     lib.dsa_abi_version.restype = i32
@@ -244,6 +248,11 @@ def dsa_cache_write(k_idx_raw, kv_raw, positions, rows, k_norm_w, k_norm_b, kv_n
     _check(lib.dsa_cache_write(int(positions.numel()), _ptr(k_idx_raw), _ptr(kv_raw), _ptr(positions), _ptr(rows),
                                _ptr(k_norm_w), _ptr(k_norm_b), _ptr(kv_norm_w), _ptr(inv_freq), eps,
                                _ptr(k_idx_cache), _ptr(kv_cache), _stream(stream)), "dsa_cache_write")
+
+
+def dsa_set_debug_checks(enable: bool) -> None:
+    """Per-row input checks in every kernel (see include/dsa.h)."""
+    load().dsa_set_debug_checks(1 if enable else 0)
 
 
 def dsa_selftest_bounded_wait(limit_us: int = 1000, stream=None) -> None:

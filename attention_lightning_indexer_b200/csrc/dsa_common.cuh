@@ -20,6 +20,7 @@ struct Problem {
     const int32_t *block_table;   // nullptr: packed rows; else [batch, max_pages] pages of 64 keys
     int max_pages;
     int ue8m0;                    // FP8 indexer scales: 0 fp32 per token, 1 ue8m0 per 128-element block
+    int debug;                    // check each row's sequence facts against the sizes (see row_ok)
 };
 
 // Value 2^(e - 127) of a ue8m0 scale byte, built exactly from its bits (e = 0 is the
@@ -85,5 +86,27 @@ __device__ __forceinline__ int visible_keys(const RowInfo &r) {
 __device__ unsigned int g_error_flag;
 
 __device__ __forceinline__ void raise_error(unsigned int code) { atomicOr(&g_error_flag, code); }
+
+constexpr unsigned ERR_BOUNDS = 4u;   // a debug-mode check found an inconsistent input
+
+// Debug mode: the row's sequence must lie inside the key arrays (cu_q / cu_k consistent with
+// total_k and max_len_k, block-table pages inside total_k).  A row that fails is counted
+// in the error flag and treated by every kernel as having no keys, so no access leaves
+// the arrays.  Always true outside debug mode.
+__device__ __forceinline__ bool row_ok(const Problem &P, const RowInfo &r) {
+    if (!P.debug) return true;
+    bool ok = r.len_k >= 1 && r.pos >= 0 && r.pos < r.len_k && r.len_k <= P.max_len_k;
+    if (P.block_table == nullptr) {
+        ok = ok && r.kbase >= 0 && (int64_t)r.kbase + r.len_k <= P.total_k;
+    } else if (ok) {
+        const int32_t *tab = P.block_table + (int64_t)r.seq * P.max_pages;
+        for (int pg = 0; pg < ((r.len_k + 63) >> 6) && ok; ++pg) {
+            const int e = __ldg(tab + pg);
+            ok = e >= 0 && ((int64_t)e + 1) * 64 <= P.total_k;
+        }
+    }
+    if (!ok) raise_error(ERR_BOUNDS);
+    return ok;
+}
 
 }  // namespace dsa

@@ -18,6 +18,8 @@ namespace {
 
 using dsa::Problem;
 
+int g_debug_checks = 0;   // dsa_set_debug_checks
+
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 dsa_status_t check_problem(const dsa_problem_t *p) {
@@ -59,6 +61,7 @@ Problem to_dev(const dsa_problem_t *p) {
     P.block_table = p->block_table;
     P.max_pages = p->block_table != nullptr ? p->max_pages : 0;
     P.ue8m0 = p->idx_dtype == DSA_E4M3_UE8M0 ? 1 : 0;
+    P.debug = g_debug_checks;
     return P;
 }
 
@@ -283,6 +286,7 @@ const char *dsa_status_string(dsa_status_t s) {
         case DSA_ERR_WORKSPACE: return "workspace missing or too small";
         case DSA_ERR_CUDA: return "CUDA launch or runtime error";
         case DSA_ERR_DEVICE_TIMEOUT: return "a device-side bounded wait gave up";
+        case DSA_ERR_DEVICE_BOUNDS: return "a debug-mode device check found an inconsistent input (row skipped)";
     }
     return "unknown status";
 }
@@ -425,8 +429,11 @@ dsa_status_t dsa_check_device_errors(dsa_stream_t stream) {
     unsigned int flag = 0, zero = 0;
     if (cudaMemcpyFromSymbol(&flag, dsa::g_error_flag, sizeof(flag)) != cudaSuccess) return DSA_ERR_CUDA;
     if (flag != 0 && cudaMemcpyToSymbol(dsa::g_error_flag, &zero, sizeof(zero)) != cudaSuccess) return DSA_ERR_CUDA;
-    return flag ? DSA_ERR_DEVICE_TIMEOUT : DSA_OK;
+    if (flag & (dsa::sm100::ERR_WAIT_TIMEOUT | dsa::sm100::ERR_SMEM_ALIGN)) return DSA_ERR_DEVICE_TIMEOUT;
+    return flag ? DSA_ERR_DEVICE_BOUNDS : DSA_OK;
 }
+
+void dsa_set_debug_checks(int32_t enable) { g_debug_checks = enable != 0; }
 
 }  // extern "C"
 

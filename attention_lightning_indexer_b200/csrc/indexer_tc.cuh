@@ -52,7 +52,7 @@ struct TcCfg {
     static constexpr int OFF_K = Q_BYTES;
     static constexpr int OFF_W = OFF_K + STAGES * KTILE_BYTES;
     static constexpr int OFF_BAR = OFF_W + QROWS * 4;
-    static constexpr int NBARS = 1 + 2 * STAGES + 4;
+    static constexpr int NBARS = 1 + 2 * STAGES + 4 + 1;   // ... + drain
     static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
     static constexpr int SMEM = OFF_MISC + 16;
     static constexpr int THREADS = 384;
@@ -84,7 +84,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         kbase = ri.kbase;
         pos0 = ri.pos;
         key0 = 0;
-        nkeys_total = min(ri.pos + qcount, ri.len_k);          // visible keys of the last query
+        nkeys_total = row_ok(P, ri) ? min(ri.pos + qcount, ri.len_k) : 0;   // visible keys of the last query
     } else {
         const int r = (int)blockIdx.x / nsplit, split = (int)blockIdx.x % nsplit;
         t0 = row_begin + r;
@@ -94,7 +94,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         kbase = ri.kbase;
         pos0 = ri.pos;
         key0 = split * C::SPLIT_KEYS;
-        nkeys_total = min(visible_keys(ri), key0 + C::SPLIT_KEYS);
+        nkeys_total = row_ok(P, ri) ? min(visible_keys(ri), key0 + C::SPLIT_KEYS) : 0;
     }
     if (nkeys_total <= key0) return;                          // uniform for the whole CTA
     const int ntiles = (nkeys_total - key0 + C::BM - 1) / C::BM;
@@ -114,6 +114,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     auto k_empty = [&](int s) { return bar0 + 8u * (1 + C::STAGES + s); };
     auto acc_full = [&](int b) { return bar0 + 8u * (1 + 2 * C::STAGES + b); };
     auto acc_empty = [&](int b) { return bar0 + 8u * (1 + 2 * C::STAGES + 2 + b); };
+    const uint32_t drain = bar0 + 8u * (1 + 2 * C::STAGES + 4);
     volatile uint32_t *misc = reinterpret_cast<volatile uint32_t *>(smem + C::OFF_MISC);  // [0] tmem base, [1] abort
 
     if (tid == 0) {
@@ -126,6 +127,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             mbar_init(acc_full(b), 1);
             mbar_init(acc_empty(b), 4);
         }
+        mbar_init(drain, 1);
         misc[1] = 0;
         fence_barrier_init();
     }
@@ -151,11 +153,13 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             for (int q = 0; q < qcount; ++q)
                 tma_load_2d(q_s + a * C::QATOM_BYTES + q * C::QBOX_BYTES, &tm_q, q_full, a * 128 / C::EB,
                             (t0 + q) * 64);
+        int issued = 0;                                       // key tiles whose loads were issued
         for (int j = 0; j < ntiles; ++j) {
             const int s = j % C::STAGES;
             if (j >= C::STAGES && !mbar_wait(k_empty(s), ((j / C::STAGES) - 1) & 1)) { misc[1] = 1; break; }
             if (misc[1]) break;
             mbar_expect_tx(k_full(s), C::KTILE_BYTES);
+            issued = j + 1;
             const int kk0 = key0 + j * C::BM;
             for (int a = 0; a < C::ATOMS; ++a) {
                 const uint32_t dst = k_s + s * C::KTILE_BYTES + a * C::KATOM_BYTES;
@@ -167,15 +171,21 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 }
             }
         }
-        // drain: the last commits on k_empty must land before the CTA may exit
+        // drain: the last commits on k_empty must land before the CTA may exit; after an
+        // abort, at least every issued load must have landed (no copy into freed memory)
         for (int j = max(0, ntiles - C::STAGES); j < ntiles && !misc[1]; ++j)
             if (!mbar_wait(k_empty(j % C::STAGES), (j / C::STAGES) & 1)) misc[1] = 1;
+        if (misc[1]) {
+            mbar_wait(q_full, 0);
+            for (int j = max(0, issued - C::STAGES); j < issued; ++j) mbar_wait(k_full(j % C::STAGES), (j / C::STAGES) & 1);
+        }
     } else if (warp == 1 && lane == 0) {
         // ------------------------------------------------ MMA issuer
         const uint32_t idesc = FP8 ? idesc_e4m3(C::BM, C::N) : idesc_bf16(C::BM, C::N);
         bool ok = mbar_wait(q_full, 0);
         tc_fence_after();
         int it = 0;
+        bool any = false;                                     // an MMA has been issued
         for (int j = 0; ok && j < ntiles && !misc[1]; ++j) {
             const int s = j % C::STAGES;
             if (!mbar_wait(k_full(s), (j / C::STAGES) & 1)) { ok = false; break; }
@@ -197,12 +207,17 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     else
                         mma_f16(d, desc_sw128(a_addr), desc_sw128(b_addr), idesc, kk > 0 ? 1u : 0u);
                 }
+                any = true;
                 mma_commit(acc_full(b));
             }
             if (!ok) break;
             mma_commit(k_empty(s));
         }
         if (!ok) misc[1] = 1;
+        if (misc[1] && any) {                                 // nothing in flight at dealloc
+            mma_commit(drain);
+            mbar_wait(drain, 0);
+        }
     } else if (warp >= 4) {
         // ------------------------------------------------ epilogue warpgroups
         const int g = (warp - 4) >> 2;            // accumulator buffer handled by this warpgroup
@@ -254,7 +269,11 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 if (q < qcount && key <= pos0 + q && key < nkeys_total) {
                     const int t = t0 + q;
                     float v = res[qi];
-                    if (FP8) v *= (P.ue8m0 ? 1.0f : __ldg(reinterpret_cast<const float *>(q_scale) + t)) * ks;
+                    if (FP8) {
+                        const float qs = P.ue8m0 ? 1.0f : __ldg(reinterpret_cast<const float *>(q_scale) + t);
+                        if (P.debug && !(qs > 0.f && ks > 0.f && qs < INFINITY && ks < INFINITY)) raise_error(ERR_BOUNDS);
+                        v *= qs * ks;
+                    }
                     scores[(int64_t)(t - row_begin) * ld + key] = v;
                 }
             }

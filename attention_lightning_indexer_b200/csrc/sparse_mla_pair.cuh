@@ -150,6 +150,7 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     const int t = T - 1 - (int)(blockIdx.x >> 1);           // heavier (later) tokens first
     const int K = P.topk;
     const RowInfo ri = row_info(P, t);
+    const bool rok = row_ok(P, ri);                          // same in both CTAs
     const int32_t *irow = idx != nullptr ? idx + (int64_t)t * K : nullptr;
     const bool masked = DENSE && idx != nullptr;
 
@@ -256,7 +257,7 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     int last_slot = -1;
 #pragma unroll
     for (int i = 0; i < 8; ++i) last_slot = max(last_slot, reinterpret_cast<int *>(red)[i]);
-    const int nblocks = misaligned ? 0 : (last_slot + C::BLK) / C::BLK;   // 0 when no slot is visible
+    const int nblocks = (misaligned || !rok) ? 0 : (last_slot + C::BLK) / C::BLK;   // 0 when no slot is visible
     __syncthreads();   // red is reused by the softmax warps
     const uint32_t peer_misc1 = mapa_shared(sbase + C::OFF_MISC + 4, (uint32_t)peer);
     auto abort_pair = [&]() {                                // stop both CTAs of the pair

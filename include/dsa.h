@@ -55,7 +55,8 @@ typedef enum dsa_status {
     DSA_ERR_UNSUPPORTED = 2,   /* a shape this build does not implement (see below) */
     DSA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than dsa_forward_workspace_size */
     DSA_ERR_CUDA = 4,          /* a CUDA launch or query failed */
-    DSA_ERR_DEVICE_TIMEOUT = 5 /* a device-side bounded wait gave up (from dsa_check_device_errors) */
+    DSA_ERR_DEVICE_TIMEOUT = 5, /* a device-side bounded wait gave up (from dsa_check_device_errors) */
+    DSA_ERR_DEVICE_BOUNDS = 6   /* a debug-mode device check failed (from dsa_check_device_errors) */
 } dsa_status_t;
 
 typedef enum dsa_dtype {
@@ -222,8 +223,9 @@ size_t dsa_forward_noalloc_scratch_bytes(void);
 
 /*
  * Synchronises `stream`, then reads and clears the device-side error flag of the
- * current device (set by a kernel whose bounded wait gave up).  Returns DSA_OK,
- * DSA_ERR_DEVICE_TIMEOUT, or DSA_ERR_CUDA if the synchronisation itself failed.
+ * current device (set by a kernel whose bounded wait gave up, or by a debug-mode check).
+ * Returns DSA_OK, DSA_ERR_DEVICE_TIMEOUT, DSA_ERR_DEVICE_BOUNDS, or DSA_ERR_CUDA if the
+ * synchronisation itself failed.
  */
 dsa_status_t dsa_check_device_errors(dsa_stream_t stream);
 
@@ -260,6 +262,16 @@ dsa_status_t dsa_cache_write(int32_t n_tokens, const void *k_idx_raw, const void
  * DSA_ERR_DEVICE_TIMEOUT and clears the flag; the device stays usable.
  */
 dsa_status_t dsa_selftest_bounded_wait(uint32_t limit_us, dsa_stream_t stream);
+
+/*
+ * Debug checks (process-wide, for the launches made after the call; off by default): every
+ * kernel checks the sequence facts of each query row against the problem's sizes (cu_q /
+ * cu_k inside total_k and max_len_k, block-table pages inside total_k) and, in the FP8
+ * indexer with fp32 scales, that the scales are finite and > 0.  A failing row is counted
+ * in the device flag (DSA_ERR_DEVICE_BOUNDS from dsa_check_device_errors) and treated as
+ * having no keys, so no access leaves the arrays.  Costs a few loads per row.
+ */
+void dsa_set_debug_checks(int32_t enable);
 
 /* Static English description of a status code (never NULL). */
 const char *dsa_status_string(dsa_status_t s);

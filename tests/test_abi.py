@@ -32,7 +32,7 @@ def test_library_exports_every_declared_entry_point():
 
 def test_status_strings():
     lib = dsa.load()
-    for code in range(6):
+    for code in range(7):
         assert lib.dsa_status_string(code)
     assert lib.dsa_status_string(99) == b"unknown status"
 

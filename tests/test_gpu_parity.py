@@ -598,3 +598,41 @@ def test_cache_write_rows_against_oracle():
     assert np.all(np.abs(got_kv - ref_kv) <= 2.0 ** -8 * np.abs(ref_kv) + 1e-4)
     untouched = np.setdiff1d(np.arange(cap), r.numpy())
     assert torch.all(kc.cpu()[untouched] == 7.0) and torch.all(kvc.cpu()[untouched] == 7.0)
+
+
+# ------------------------------------------------------------ debug checks
+
+def test_debug_checks_flag_and_skip_an_inconsistent_sequence():
+    # The last sequence's key range runs 64 rows past total_k (its length stays within
+    # max_len_k, so even unchecked every access would stay inside the buffers: TMA loads
+    # past the arrays read zeros).  With debug checks on, that row is flagged and skipped
+    # (no keys: idx -1, out 0, lse -inf) while the other rows are unchanged.
+    inp = dsa_synth.make_decode(4, 5000, 6000, topk=256, seed=91, device=DEV)
+    ref = _run_forward(inp)
+    dsa.dsa_check_device_errors()
+    bad = dict(inp)
+    cu_k = inp["cu_k"].clone()
+    cu_k[-1] += 64                                       # only the last sequence grows
+    bad["cu_k"] = cu_k
+    bad["max_len_k"] = inp["max_len_k"] + 64
+    dsa.dsa_set_debug_checks(True)
+    try:
+        idx, out, lse = _run_forward(bad)
+        with pytest.raises(dsa.DsaError) as e:
+            dsa.dsa_check_device_errors()
+        assert e.value.code == 6
+        dsa.dsa_check_device_errors()                    # cleared by the read
+        assert torch.equal(idx[:3], ref[0][:3]) and torch.equal(out[:3], ref[1][:3]) and torch.equal(lse[:3], ref[2][:3])
+        assert torch.all(idx[3] == -1) and torch.all(out[3] == 0) and torch.all(torch.isneginf(lse[3]))
+        _run_forward(inp)                                # a consistent problem passes the checks
+        dsa.dsa_check_device_errors()
+        # FP8 with an fp32 scale that is not > 0
+        f8 = dsa_synth.make_prefill(600, topk=64, seed=92, device=DEV, fp8_indexer=True)
+        f8["k_scale"][17] = 0.0
+        _gpu_scores(f8, dsa.problem_from_inputs(f8))
+        with pytest.raises(dsa.DsaError) as e:
+            dsa.dsa_check_device_errors()
+        assert e.value.code == 6
+    finally:
+        dsa.dsa_set_debug_checks(False)
+        dsa.dsa_check_device_errors()
