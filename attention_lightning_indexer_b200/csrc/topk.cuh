@@ -12,9 +12,9 @@
 // Fast path (one HBM read of the row):
 //   * every 16th float4 of the row is sampled; a radix select on the sample (two 11-bit
 //     digits) gives a key t_lo that about 1.2 k keys of the full row are expected to reach;
-//   * one pass over the row keeps the keys >= t_lo with their indices, each warp in its
-//     own shared-memory segment and in ascending index order (ballot prefix sums, no
-//     atomics);
+//   * one pass over the row (float4 loads, the next chunk in flight while the current one
+//     is filtered) keeps the keys >= t_lo with their indices, each warp in its own
+//     shared-memory segment and in ascending index order (ballot prefix sums, no atomics);
 //   * an exact radix select (11/11/10-bit digits) over these candidates gives the k-th
 //     largest key `thr` and how many keys equal to it are taken (smallest indices first);
 //   * the candidates > thr and the first `need_eq` == thr are written in ascending index
@@ -22,6 +22,11 @@
 // If the sample misjudged (fewer than k candidates, or a warp's segment overflows) the
 // general path runs instead: a full-row radix select with candidate compaction and an
 // ordered final pass over the row (same result, more passes).
+//
+// Every digit pass takes two block barriers: the histograms are double-buffered (a pass
+// clears the other buffer for the next pass while it counts), and the bin holding the
+// target rank is found from 32 group sums kept beside each histogram (two dependent
+// shared-memory loads per lane instead of a walk over 64 bins).
 #pragma once
 
 #include "dsa_common.cuh"
@@ -30,25 +35,28 @@ namespace dsa {
 namespace topk {
 
 constexpr int BINS = 2048;        // 11-bit digits
+constexpr int GROUPS = 32;        // group sums per histogram (one per lane of the bin search)
 constexpr unsigned FULL = 0xffffffffu;
 
 template <int NT>
 struct Cfg {
     static constexpr int THREADS = NT;
     static constexpr int WARPS = NT / 32;
-    static constexpr int SEG = 8192 / WARPS;                  // candidate slots per warp (fast path)
+    static constexpr int SEG = 7168 / WARPS;                  // candidate slots per warp (fast path)
     static constexpr int CAND_CAP = WARPS * SEG * 2;          // general-path candidate indices (same bytes)
     // Dynamic shared memory layout.
-    static constexpr int OFF_HIST = 0;                        // [BINS] u32
-    static constexpr int OFF_SEGK = OFF_HIST + BINS * 4;      // [WARPS][SEG] u32 keys (also: samples)
-    static constexpr int OFF_SEGI = OFF_SEGK + WARPS * SEG * 4;   // [WARPS][SEG] int indices
-    static constexpr int OFF_SCAL = OFF_SEGI + WARPS * SEG * 4;   // scalars, see below
-    // scal: [0..1] select_bin result, [2] candidate count, [3] overflow flag, then three
-    // per-warp arrays A = scal + 8, B = A + WARPS, C = B + WARPS
+    static constexpr int OFF_HIST = 0;                             // [2][BINS] u32
+    static constexpr int OFF_GRP = OFF_HIST + 2 * BINS * 4;        // [2][GROUPS] u32
+    static constexpr int OFF_SEGK = OFF_GRP + 2 * GROUPS * 4;      // [WARPS][SEG] u32 keys
+    static constexpr int OFF_SEGI = OFF_SEGK + WARPS * SEG * 4;    // [WARPS][SEG] int indices
+    // (the samples of the fast path, up to 2 * WARPS * SEG keys, span both arrays)
+    static constexpr int OFF_SCAL = OFF_SEGI + WARPS * SEG * 4;    // scalars, see below
+    // scal: [0..1] and [4..5] digit-pass results (by pass parity), [2] candidate count,
+    // [3] overflow flag, then three per-warp arrays A = scal + 8, B = A + WARPS, C = B + WARPS
     static constexpr int NSCAL = 8 + 3 * WARPS;
     static constexpr int SMEM = OFF_SCAL + NSCAL * 4;
+    static_assert(7168 % WARPS == 0 && NT % 32 == 0, "whole warps, equal segments");
     static_assert(CAND_CAP * 4 == 2 * WARPS * SEG * 4, "general-path candidates reuse both segment arrays");
-    static_assert(NT % 32 == 0 && 2048 % (NT / 32) == 0, "whole warps; select_bin splits 2048 bins over 32 lanes");
 };
 
 __device__ __forceinline__ uint32_t order_key(float f) {
@@ -57,56 +65,101 @@ __device__ __forceinline__ uint32_t order_key(float f) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Warp-aggregated histogram increment; d == BINS means "no key" (lane still participates).
-__device__ __forceinline__ void hist_add(uint32_t *hist, uint32_t d, int lane) {
-    const unsigned peers = __match_any_sync(FULL, d);
-    if (d < (uint32_t)BINS && lane == __ffs(peers) - 1) atomicAdd(&hist[d], (uint32_t)__popc(peers));
+// The float whose key is k (inverse of order_key; key 0x80000000 gives +0.0).  For finite
+// v: order_key(v) >= k  <=>  v >= key_float(k), signed zeros included.
+__device__ __forceinline__ float key_float(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
-// Warp 0: the bin holding the `remaining`-th largest key; writes bin and the count of
-// keys in strictly higher bins to scal[0], scal[1].  Lane L first sums its block of
-// nbins/32 consecutive bins (lane 0 owns the highest; the loop is skewed by the lane so the
-// 32 lanes hit 32 different banks), a warp scan finds the lane whose block holds the
-// target, and the warp then scans that block (per/32 bins per lane) to find the bin.
-__device__ __forceinline__ void select_bin(const uint32_t *hist, int nbins, int remaining, int *scal) {
+// Histogram buffers of parity p.
+template <class C>
+__device__ __forceinline__ uint32_t *hist_of(unsigned char *smem, int p) {
+    return reinterpret_cast<uint32_t *>(smem + C::OFF_HIST) + p * BINS;
+}
+template <class C>
+__device__ __forceinline__ uint32_t *grp_of(unsigned char *smem, int p) {
+    return reinterpret_cast<uint32_t *>(smem + C::OFF_GRP) + p * GROUPS;
+}
+
+// Clears the histogram and group sums of parity p (all threads).
+template <class C>
+__device__ __forceinline__ void clear_hist(unsigned char *smem, int p) {
+    uint4 *h = reinterpret_cast<uint4 *>(hist_of<C>(smem, p));
+    for (int i = threadIdx.x; i < BINS / 4; i += C::THREADS) h[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (threadIdx.x < GROUPS) grp_of<C>(smem, p)[threadIdx.x] = 0u;
+}
+
+// Warp-aggregated count of digit d (d >= NB: no key; the lane still takes part) into the
+// bin and its group (NB / GROUPS consecutive bins).
+template <int NB>
+__device__ __forceinline__ void hist_add(uint32_t *hist, uint32_t *grp, uint32_t d, int lane) {
+    const unsigned peers = __match_any_sync(FULL, d);
+    if (d < (uint32_t)NB && lane == __ffs(peers) - 1) atomicAdd(&hist[d], (uint32_t)__popc(peers));
+    const uint32_t g = d < (uint32_t)NB ? d / (uint32_t)(NB / GROUPS) : (uint32_t)GROUPS;
+    const unsigned gpeers = __match_any_sync(FULL, g);
+    if (g < (uint32_t)GROUPS && lane == __ffs(gpeers) - 1) atomicAdd(&grp[g], (uint32_t)__popc(gpeers));
+}
+
+__device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v, int lane) {
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t x = __shfl_up_sync(FULL, v, off);
+        if (lane >= off) v += x;
+    }
+    return v;
+}
+
+// Warp 0: the bin of an NB-bin histogram holding the `remaining`-th largest key; writes the
+// bin and the count of keys in strictly higher bins to res[0], res[1].  Lane l first takes
+// group 31 - l (highest first), a warp scan finds the group holding the target, then each
+// lane takes Q = NB / 1024 bins of that group (highest first) and a second scan finds the
+// bin.  remaining <= the histogram's total.
+template <int NB>
+__device__ __forceinline__ void select_bin(const uint32_t *hist, const uint32_t *grp, int remaining, int *res) {
+    constexpr int PER = NB / GROUPS;   // bins per group: 64 or 32
+    constexpr int Q = PER / 32;        // bins per lane within the group: 2 or 1
     const int lane = threadIdx.x & 31;
-    const int per = nbins / 32;               // 64 or 32 bins per lane
-    const int top = nbins - 1 - lane * per;   // lane 0 owns the highest bins
-    uint32_t mine = 0;
-    for (int i = 0; i < per; ++i) mine += hist[top - ((i + lane) & (per - 1))];
-    uint32_t incl = mine;
+    const uint32_t rem = (uint32_t)remaining;
+    const uint32_t mine = grp[GROUPS - 1 - lane];
+    const uint32_t incl = warp_incl_scan(mine, lane);
+    const unsigned hit = __ballot_sync(FULL, (incl - mine) < rem && rem <= incl);
+    const int src = hit ? __ffs(hit) - 1 : 0;  // hit == 0 cannot happen; stay in range
+    const uint32_t above_grp = __shfl_sync(FULL, incl - mine, src);
+    const int btop = (GROUPS - src) * PER - 1;  // highest bin of that group
+    uint32_t h[Q];
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const uint32_t v = __shfl_up_sync(FULL, incl, off);
-        if (lane >= off) incl += v;
-    }
-    // the lane whose block holds the target (exactly one: remaining <= total keys)
-    const unsigned hit = __ballot_sync(FULL, (incl - mine) < (uint32_t)remaining && (uint32_t)remaining <= incl);
-    const int src = hit ? __ffs(hit) - 1 : 0;  // hit == 0 cannot happen (remaining <= count); stay in range
-    const uint32_t above_blk = __shfl_sync(FULL, incl - mine, src);
-    const int btop = nbins - 1 - src * per;
-    // that block, highest bin first: lane l holds bins btop - l*q .. btop - l*q - (q-1), q = per/32
-    const int q = per / 32;
-    uint32_t h[2] = {0, 0};
-    for (int j = 0; j < q; ++j) h[j] = hist[btop - lane * q - j];
-    const uint32_t lsum = h[0] + (q > 1 ? h[1] : 0u);
-    uint32_t lincl = lsum;
+    for (int j = 0; j < Q; ++j) h[j] = hist[btop - lane * Q - j];
+    uint32_t lsum = 0;
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const uint32_t v = __shfl_up_sync(FULL, lincl, off);
-        if (lane >= off) lincl += v;
-    }
-    const uint32_t lbefore = above_blk + lincl - lsum;
-    const bool mine_hit = lbefore < (uint32_t)remaining && (uint32_t)remaining <= lbefore + lsum;
-    if (hit != 0 && mine_hit) {
-        if (lbefore + h[0] >= (uint32_t)remaining) {
-            scal[0] = btop - lane * q;
-            scal[1] = (int)lbefore;
-        } else {
-            scal[0] = btop - lane * q - 1;
-            scal[1] = (int)(lbefore + h[0]);
+    for (int j = 0; j < Q; ++j) lsum += h[j];
+    const uint32_t lbefore = above_grp + warp_incl_scan(lsum, lane) - lsum;
+    if (hit != 0 && lbefore < rem && rem <= lbefore + lsum) {
+        uint32_t acc = lbefore;
+#pragma unroll
+        for (int j = 0; j < Q; ++j) {
+            if (acc + h[j] >= rem) {
+                res[0] = btop - lane * Q - j;
+                res[1] = (int)acc;
+                break;
+            }
+            acc += h[j];
         }
     }
+}
+
+// One digit pass.  On entry the buffers of parity `cur` are zero and visible to all
+// threads; this pass clears parity cur ^ 1 for the next one, counts with add(hist, grp),
+// and returns {bin, keys in higher bins} of the `remaining`-th largest.  Two barriers.
+template <class C, int NB, class Add>
+__device__ __forceinline__ int2 digit_pass(unsigned char *smem, int cur, int remaining, Add add) {
+    int *res = reinterpret_cast<int *>(smem + C::OFF_SCAL) + 4 * cur;
+    uint32_t *hist = hist_of<C>(smem, cur), *grp = grp_of<C>(smem, cur);
+    clear_hist<C>(smem, cur ^ 1);
+    add(hist, grp);
+    __syncthreads();
+    if ((threadIdx.x >> 5) == 0) select_bin<NB>(hist, grp, remaining, res);
+    __syncthreads();
+    return make_int2(res[0], res[1]);
 }
 
 __device__ __forceinline__ int warp_sum(int v) {
@@ -116,12 +169,7 @@ __device__ __forceinline__ int warp_sum(int v) {
 }
 
 __device__ __forceinline__ int warp_excl_scan(int v, int lane, int &total) {
-    int incl = v;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const int x = __shfl_up_sync(FULL, incl, off);
-        if (lane >= off) incl += x;
-    }
+    const int incl = (int)warp_incl_scan((uint32_t)v, lane);
     total = __shfl_sync(FULL, incl, 31);
     return incl - v;
 }
@@ -140,71 +188,50 @@ __device__ __forceinline__ void load4(const float *src, int i0, int we, uint32_t
     for (int c = 0; c < 4; ++c) k[c] = i0 + c < we ? order_key(__ldg(src + i0 + c)) : 0u;
 }
 
-// Exact radix selection (11/11/10-bit digits, MSB first) of the `rank`-th largest key among
-// the keys get(j), j < m, for which valid(j) holds.  Returns the key; *above receives the
-// number of keys strictly greater.  All threads call it; uses hist and scal[0..1].
-// With passes == 2 the result is only a lower bound of that key: the smallest key of the
-// 22-bit bin that holds it (enough for a candidate threshold).
-template <class C, class Get>
-__device__ uint32_t radix_select(int m, int rank, Get get, uint32_t *hist, int *scal, int *above, int passes = 3) {
-    constexpr int THREADS = C::THREADS;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    uint32_t prefix = 0, mask = 0;
-    int remaining = rank, above_total = 0;
-    const int m_pad = (m + 31) & ~31;
-    for (int pass = 0; pass < passes; ++pass) {
-        const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-        const int nb = pass == 2 ? 1024 : 2048;
-        for (int i = tid; i < nb; i += THREADS) hist[i] = 0;
-        __syncthreads();
-        for (int j = tid; j < m_pad; j += THREADS) {
-            uint32_t d = (uint32_t)BINS, key = 0;
-            if (j < m && get(j, key) && (key & mask) == prefix) d = (key >> shift) & (uint32_t)(nb - 1);
-            hist_add(hist, d, lane);
-        }
-        __syncthreads();
-        if (warp == 0) select_bin(hist, nb, remaining, scal);
-        __syncthreads();
-        remaining -= scal[1];
-        above_total += scal[1];
-        prefix |= (uint32_t)scal[0] << shift;
-        mask |= (uint32_t)(nb - 1) << shift;
-        __syncthreads();
-    }
-    *above = above_total;
-    return prefix;
+// The lane's 4 consecutive scores i0..i0+3, reading only below we (the rest are 0 and
+// must be masked by the caller).
+__device__ __forceinline__ float4 load4f(const float *src, int i0, int we) {
+    if (i0 + 3 < we) return __ldg(reinterpret_cast<const float4 *>(src + i0));
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (i0 < we) v.x = __ldg(src + i0);
+    if (i0 + 1 < we) v.y = __ldg(src + i0 + 1);
+    if (i0 + 2 < we) v.z = __ldg(src + i0 + 2);
+    return v;
 }
 
-// The same selection when each warp holds its own items: warp w's items are get(j),
-// j < m_w (m_w differs per warp); every warp walks only its own items.
-template <class C, class Get>
-__device__ uint32_t radix_select_per_warp(int m_w, int rank, Get get, uint32_t *hist, int *scal, int *above) {
-    constexpr int THREADS = C::THREADS;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+// Exact radix selection (11/11/10-bit digits, MSB first) of the `rank`-th largest key.
+// for_items(fn) calls fn(key, valid) once per item of the calling thread; the lanes of a
+// warp must make the same number of calls.  Starts on zeroed buffers of parity 0 and
+// leaves parity 0 zeroed after an even number of passes.  Returns the key; *above
+// receives the number of keys strictly greater.  With passes == 2 the result is only a
+// lower bound of that key: the smallest key of the 22-bit bin that holds it.
+template <class C, class ForItems>
+__device__ uint32_t radix_select(int rank, ForItems for_items, unsigned char *smem, int *above, int passes = 3) {
+    const int lane = threadIdx.x & 31;
     uint32_t prefix = 0, mask = 0;
     int remaining = rank, above_total = 0;
-    const int m_pad = (m_w + 31) & ~31;
-    for (int pass = 0; pass < 3; ++pass) {
+    for (int pass = 0; pass < passes; ++pass) {
         const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-        const int nb = pass == 2 ? 1024 : 2048;
-        for (int i = tid; i < nb; i += THREADS) hist[i] = 0;
-        __syncthreads();
-        for (int j = lane; j < m_pad; j += 32) {
-            uint32_t d = (uint32_t)BINS;
-            if (j < m_w) {
-                const uint32_t key = get(j);
-                if ((key & mask) == prefix) d = (key >> shift) & (uint32_t)(nb - 1);
-            }
-            hist_add(hist, d, lane);
+        int2 r;
+        if (pass < 2) {
+            r = digit_pass<C, 2048>(smem, pass & 1, remaining, [&](uint32_t *hist, uint32_t *grp) {
+                for_items([&](uint32_t key, bool valid) {
+                    const bool in = valid && (key & mask) == prefix;
+                    hist_add<2048>(hist, grp, in ? (key >> shift) & 2047u : 2048u, lane);
+                });
+            });
+        } else {
+            r = digit_pass<C, 1024>(smem, pass & 1, remaining, [&](uint32_t *hist, uint32_t *grp) {
+                for_items([&](uint32_t key, bool valid) {
+                    const bool in = valid && (key & mask) == prefix;
+                    hist_add<1024>(hist, grp, in ? key & 1023u : 1024u, lane);
+                });
+            });
         }
-        __syncthreads();
-        if (warp == 0) select_bin(hist, nb, remaining, scal);
-        __syncthreads();
-        remaining -= scal[1];
-        above_total += scal[1];
-        prefix |= (uint32_t)scal[0] << shift;
-        mask |= (uint32_t)(nb - 1) << shift;
-        __syncthreads();
+        remaining -= r.y;
+        above_total += r.y;
+        prefix |= (uint32_t)r.x << shift;
+        mask |= (pass == 2 ? 1023u : 2047u) << shift;
     }
     *above = above_total;
     return prefix;
@@ -245,24 +272,49 @@ __device__ __forceinline__ void ordered_output(const float *src, int wb, int we,
     }
 }
 
+// Appends the scores of one float4 group (indices i0..i0+3 of lane's slot, nv of them
+// valid) that reach f_lo to the warp's segment in index order: lanes in order, then the
+// four components.
+template <int SEG>
+__device__ __forceinline__ void keep_group(const float4 v, int i0, int nv, float f_lo, unsigned lt, int &cnt,
+                                          uint32_t *mk, int *mi) {
+    const bool t0 = nv > 0 && v.x >= f_lo, t1 = nv > 1 && v.y >= f_lo;
+    const bool t2 = nv > 2 && v.z >= f_lo, t3 = nv > 3 && v.w >= f_lo;
+    const unsigned b0 = __ballot_sync(FULL, t0), b1 = __ballot_sync(FULL, t1);
+    const unsigned b2 = __ballot_sync(FULL, t2), b3 = __ballot_sync(FULL, t3);
+    int off = cnt + __popc(b0 & lt) + __popc(b1 & lt) + __popc(b2 & lt) + __popc(b3 & lt);
+    if (t0) {
+        if (off < SEG) { mk[off] = order_key(v.x); mi[off] = i0; }
+        ++off;
+    }
+    if (t1) {
+        if (off < SEG) { mk[off] = order_key(v.y); mi[off] = i0 + 1; }
+        ++off;
+    }
+    if (t2) {
+        if (off < SEG) { mk[off] = order_key(v.z); mi[off] = i0 + 2; }
+        ++off;
+    }
+    if (t3 && off < SEG) { mk[off] = order_key(v.w); mi[off] = i0 + 3; }
+    cnt += __popc(b0) + __popc(b1) + __popc(b2) + __popc(b3);
+}
+
 // Fast path.  Returns false (nothing written) when the sample misjudged the row.
 template <class C>
 __device__ bool select_row_sampled(const float *src, int n, int K, unsigned char *smem, int32_t *out) {
     constexpr int THREADS = C::THREADS, WARPS = C::WARPS, SEG = C::SEG;
-    constexpr int OFF_HIST = C::OFF_HIST, OFF_SEGK = C::OFF_SEGK, OFF_SEGI = C::OFF_SEGI, OFF_SCAL = C::OFF_SCAL;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    uint32_t *hist = reinterpret_cast<uint32_t *>(smem + OFF_HIST);
-    uint32_t *segk = reinterpret_cast<uint32_t *>(smem + OFF_SEGK);
-    int *segi = reinterpret_cast<int *>(smem + OFF_SEGI);
-    int *scal = reinterpret_cast<int *>(smem + OFF_SCAL);
+    uint32_t *segk = reinterpret_cast<uint32_t *>(smem + C::OFF_SEGK);
+    int *segi = reinterpret_cast<int *>(smem + C::OFF_SEGI);
+    int *scal = reinterpret_cast<int *>(smem + C::OFF_SCAL);
     int *seg_cnt = scal + 8, *wgt = scal + 8 + WARPS, *weq = scal + 8 + 2 * WARPS;
     const float4 *s4 = reinterpret_cast<const float4 *>(src);
     const int n4 = n >> 2;
     const int nsamp4 = (n4 + 15) / 16;                       // sampled float4 (every 16th)
     const int ns = 4 * nsamp4;
-    if (ns < 64 || ns > WARPS * SEG) return false;
+    if (ns < 64 || ns > 2 * WARPS * SEG) return false;
 
-    // ---- sample keys into the segment key array (free at this point)
+    // ---- sample keys into the segment arrays (keys, then indices: contiguous, free now)
     for (int m = tid; m < nsamp4; m += THREADS) {
         const float4 v = __ldg(s4 + 16 * m);
         segk[4 * m + 0] = order_key(v.x);
@@ -270,62 +322,70 @@ __device__ bool select_row_sampled(const float *src, int n, int K, unsigned char
         segk[4 * m + 2] = order_key(v.z);
         segk[4 * m + 3] = order_key(v.w);
     }
-    if (tid < WARPS) seg_cnt[tid] = 0;
+    clear_hist<C>(smem, 0);
     if (tid == 0) scal[3] = 0;
     __syncthreads();
     const int target = min(ns, (int)((1.2 * K * (double)ns) / (double)n) + 16);
     int dummy;
     // a lower bound of the sample's target-th key is all the candidate pass needs: two
-    // digit passes (22 bits)
+    // digit passes (22 bits); the samples are last read before the first barrier of the
+    // second pass, so the candidate pass below may overwrite them
+    const int ns_pad = (ns + THREADS - 1) / THREADS * THREADS;
     const uint32_t t_lo = radix_select<C>(
-        ns, target, [&](int j, uint32_t &key) { key = segk[j]; return true; }, hist, scal, &dummy, 2);
-    __syncthreads();   // samples no longer needed
+        target,
+        [&](auto fn) {
+            for (int j = tid; j < ns_pad; j += THREADS) fn(j < ns ? segk[j] : 0u, j < ns);
+        },
+        smem, &dummy, 2);
+    const float f_lo = key_float(t_lo);
 
-    // ---- candidates: keys >= t_lo, per warp in ascending index order
+    // ---- candidates: scores >= f_lo, per warp in ascending index order.  Chunks of 512
+    // scores per warp (4 float4 per lane); the next chunk is loaded before the current one
+    // is filtered.
     const int R = ((n + WARPS * 128 - 1) / (WARPS * 128)) * 128;
-    const int wb = warp * R, we = min(n, wb + R);
+    const int wb = min(n, warp * R), we = min(n, wb + R);
     uint32_t *mk = segk + warp * SEG;
     int *mi = segi + warp * SEG;
     int cnt = 0;
-    bool overflow = false;
     const unsigned lt = (1u << lane) - 1u;
-    for (int base = wb; base < we; base += 512) {
-        // 16 coalesced loads per lane, keys base + 32 j + lane: the order (j, lane) is the
-        // index order, so ballot prefix counts keep the segment sorted by index
-        uint32_t kk[16];
+    float4 v[4];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const int i = base + 32 * j + lane;
-            kk[j] = i < we ? order_key(__ldg(src + i)) : 0u;
+    for (int g = 0; g < 4; ++g) v[g] = load4f(src, wb + 128 * g + 4 * lane, we);
+    for (int base = wb; base < we; base += 512) {
+        float4 nx[4];
+        const int nbase = base + 512;
+        if (nbase < we) {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) nx[g] = load4f(src, nbase + 128 * g + 4 * lane, we);
         }
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const int i = base + 32 * j + lane;
-            const bool take = i < we && kk[j] >= t_lo;
-            const unsigned m = __ballot_sync(FULL, take);
-            if (take) {
-                const int off = cnt + __popc(m & lt);
-                if (off < SEG) {
-                    mk[off] = kk[j];
-                    mi[off] = i;
-                }
-            }
-            cnt += __popc(m);
+        for (int g = 0; g < 4; ++g) {
+            const int i0 = base + 128 * g + 4 * lane;
+            keep_group<SEG>(v[g], i0, min(max(we - i0, 0), 4), f_lo, lt, cnt, mk, mi);
+        }
+        if (nbase < we) {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) v[g] = nx[g];
         }
     }
-    overflow = cnt > SEG;
     if (lane == 0) {
-        seg_cnt[warp] = overflow ? 0 : cnt;
-        if (overflow) scal[3] = 1;
+        seg_cnt[warp] = cnt > SEG ? 0 : cnt;
+        if (cnt > SEG) scal[3] = 1;
     }
     __syncthreads();
     int total = 0;
     for (int w = 0; w < WARPS; ++w) total += seg_cnt[w];
     if (scal[3] != 0 || total < K) return false;   // uniform decision
 
-    // ---- exact k-th largest among the candidates
+    // ---- exact k-th largest among the candidates (each warp walks its own segment)
     int above;
-    const uint32_t thr = radix_select_per_warp<C>(cnt, K, [&](int j) { return mk[j]; }, hist, scal, &above);
+    const int cnt_pad = (cnt + 31) & ~31;
+    const uint32_t thr = radix_select<C>(
+        K,
+        [&](auto fn) {
+            for (int j = lane; j < cnt_pad; j += 32) fn(j < cnt ? mk[j] : 0u, j < cnt);
+        },
+        smem, &above);
     const int need_eq = K - above;                   // >= 1
     const int count_gt = above;
 
@@ -337,7 +397,6 @@ __device__ bool select_row_sampled(const float *src, int n, int K, unsigned char
     }
     cg = warp_sum(cg);
     ce = warp_sum(ce);
-    __syncthreads();
     if (lane == 0) {
         wgt[warp] = cg;
         weq[warp] = ce;
@@ -371,51 +430,41 @@ __device__ bool select_row_sampled(const float *src, int n, int K, unsigned char
 template <class C>
 __device__ void select_row_general(const float *src, int n, int K, unsigned char *smem, int32_t *out) {
     constexpr int THREADS = C::THREADS, WARPS = C::WARPS, CAND_CAP = C::CAND_CAP;
-    constexpr int OFF_HIST = C::OFF_HIST, OFF_SEGK = C::OFF_SEGK, OFF_SCAL = C::OFF_SCAL;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    uint32_t *hist = reinterpret_cast<uint32_t *>(smem + OFF_HIST);
-    int *cand = reinterpret_cast<int *>(smem + OFF_SEGK);   // CAND_CAP entries over both segment arrays
-    int *scal = reinterpret_cast<int *>(smem + OFF_SCAL);
+    int *cand = reinterpret_cast<int *>(smem + C::OFF_SEGK);   // CAND_CAP entries over both segment arrays
+    int *scal = reinterpret_cast<int *>(smem + C::OFF_SCAL);
     // per warp: keys above bin b0, keys in b0 above thr, keys == thr
     int *w_above = scal + 8, *w_gt = scal + 8 + WARPS, *w_eq = scal + 8 + 2 * WARPS;
     const float4 *s4 = reinterpret_cast<const float4 *>(src);
     const int n4 = n >> 2;
     const int R = ((n + WARPS * 128 - 1) / (WARPS * 128)) * 128;
-    const int wb = warp * R, we = min(n, wb + R);
+    const int wb = min(n, warp * R), we = min(n, wb + R);
 
-    __syncthreads();
-    for (int i = tid; i < BINS; i += THREADS) hist[i] = 0;
+    __syncthreads();   // the fast path's last reads of shared memory are done
+    clear_hist<C>(smem, 0);
     for (int i = tid; i < 3 * WARPS; i += THREADS) scal[8 + i] = 0;
     if (tid == 0) scal[2] = 0;
     __syncthreads();
 
-    // ---- pass 1: histogram of bits 31..21 over the whole row
-    for (int base = 0; base < n4; base += THREADS * 4) {
-        float4 v[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int i = base + u * THREADS + tid;
-            v[u] = i < n4 ? __ldg(s4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+    // ---- pass 1: histogram of bits 31..21 over the whole row (float4 body, scalar tail)
+    const int n4_pad = (n4 + THREADS - 1) / THREADS * THREADS;
+    const int tail = n - (n4 << 2);
+    const int2 r0 = digit_pass<C, 2048>(smem, 0, K, [&](uint32_t *hist, uint32_t *grp) {
+        for (int i = tid; i < n4_pad; i += THREADS) {
+            const bool ok = i < n4;
+            const float4 v = ok ? __ldg(s4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+            hist_add<2048>(hist, grp, ok ? order_key(v.x) >> 21 : 2048u, lane);
+            hist_add<2048>(hist, grp, ok ? order_key(v.y) >> 21 : 2048u, lane);
+            hist_add<2048>(hist, grp, ok ? order_key(v.z) >> 21 : 2048u, lane);
+            hist_add<2048>(hist, grp, ok ? order_key(v.w) >> 21 : 2048u, lane);
         }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const bool ok = base + u * THREADS + tid < n4;
-            hist_add(hist, ok ? order_key(v[u].x) >> 21 : (uint32_t)BINS, lane);
-            hist_add(hist, ok ? order_key(v[u].y) >> 21 : (uint32_t)BINS, lane);
-            hist_add(hist, ok ? order_key(v[u].z) >> 21 : (uint32_t)BINS, lane);
-            hist_add(hist, ok ? order_key(v[u].w) >> 21 : (uint32_t)BINS, lane);
+        if (warp == 0) {   // the tail (< 4 keys): the whole warp takes part
+            const bool ok = lane < tail;
+            hist_add<2048>(hist, grp, ok ? order_key(__ldg(src + (n4 << 2) + lane)) >> 21 : 2048u, lane);
         }
-    }
-    {
-        const int tail = n - (n4 << 2);
-        if (tid < tail) atomicAdd(&hist[order_key(__ldg(src + (n4 << 2) + tid)) >> 21], 1u);
-    }
-    __syncthreads();
-    if (warp == 0) select_bin(hist, BINS, K, scal);
-    __syncthreads();
-    const uint32_t b0 = (uint32_t)scal[0];
-    int remaining = K - scal[1];
-    __syncthreads();
+    });
+    const uint32_t b0 = (uint32_t)r0.x;
+    int remaining = K - r0.y;
 
     // ---- pass 2: per-warp count of keys above bin b0, compaction of the keys in b0
     {
@@ -443,31 +492,37 @@ __device__ void select_row_general(const float *src, int n, int K, unsigned char
     const int ncand = scal[2];
     const bool use_cand = ncand <= CAND_CAP;
 
-    // ---- digits 2 and 3 on the candidates (or on the whole row after an overflow)
+    // ---- digits 2 and 3 on the candidates (or on the whole row after an overflow); the
+    // first pass left parity 1 cleared
     uint32_t prefix = b0 << 21, mask = 0xFFE00000u;
-    for (int pass = 1; pass <= 2; ++pass) {
-        const int shift = pass == 1 ? 10 : 0;
-        const int nb = pass == 1 ? 2048 : 1024;
-        for (int i = tid; i < nb; i += THREADS) hist[i] = 0;
-        __syncthreads();
-        const int m = use_cand ? ncand : n;
-        const int m_pad = (m + 31) & ~31;
+    const int m = use_cand ? ncand : n;
+    const int m_pad = (m + THREADS - 1) / THREADS * THREADS;
+    auto key_at = [&](int j) { return order_key(__ldg(src + (use_cand ? cand[j] : j))); };
+    const int2 r1 = digit_pass<C, 2048>(smem, 1, remaining, [&](uint32_t *hist, uint32_t *grp) {
         for (int j = tid; j < m_pad; j += THREADS) {
-            uint32_t d = (uint32_t)BINS;
+            uint32_t d = 2048u;
             if (j < m) {
-                const uint32_t key = order_key(__ldg(src + (use_cand ? cand[j] : j)));
-                if ((key & mask) == prefix) d = (key >> shift) & (uint32_t)(nb - 1);
+                const uint32_t key = key_at(j);
+                if ((key & mask) == prefix) d = (key >> 10) & 2047u;
             }
-            hist_add(hist, d, lane);
+            hist_add<2048>(hist, grp, d, lane);
         }
-        __syncthreads();
-        if (warp == 0) select_bin(hist, nb, remaining, scal);
-        __syncthreads();
-        remaining -= scal[1];
-        prefix |= (uint32_t)scal[0] << shift;
-        mask |= (uint32_t)(nb - 1) << shift;
-        __syncthreads();
-    }
+    });
+    remaining -= r1.y;
+    prefix |= (uint32_t)r1.x << 10;
+    mask |= 2047u << 10;
+    const int2 r2 = digit_pass<C, 1024>(smem, 0, remaining, [&](uint32_t *hist, uint32_t *grp) {
+        for (int j = tid; j < m_pad; j += THREADS) {
+            uint32_t d = 1024u;
+            if (j < m) {
+                const uint32_t key = key_at(j);
+                if ((key & mask) == prefix) d = key & 1023u;
+            }
+            hist_add<1024>(hist, grp, d, lane);
+        }
+    });
+    remaining -= r2.y;
+    prefix |= (uint32_t)r2.x;
     const uint32_t thr = prefix;
     const int need_eq = remaining;       // >= 1
     const int count_gt = K - need_eq;
