@@ -129,8 +129,8 @@ dsa_status_t set_smem_attrs() {
     e = cudaFuncSetAttribute(dsa::topk::topk_rows_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              dsa::topk::Cfg<256>::SMEM);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(dsa::topk::topk_rows_kernel<512>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 dsa::topk::Cfg<512>::SMEM);
+        e = cudaFuncSetAttribute(dsa::topk::topk_rows_kernel<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 dsa::topk::Cfg<1024>::SMEM);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(dsa::mla::sparse_mla_pair_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  dsa::mla::PairCfg::SMEM);
@@ -199,14 +199,14 @@ dsa_status_t topk_launch(const dsa_problem_t *p, const float *scores, int64_t ld
                          int32_t *idx, cudaStream_t stream) {
     if (row_count == 0) return DSA_OK;
     Problem P = to_dev(p);
-    // Fewer rows than SMs (decode): 512 threads per row; otherwise 256 threads, several
+    // Fewer rows than SMs (decode): 1024 threads per row; otherwise 256 threads, several
     // CTAs per SM.  Both produce the same indices in the same order.
     int dev = 0, n_sm = 148;
     if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
         return DSA_ERR_CUDA;
     if (row_count < n_sm)
-        dsa::topk::topk_rows_kernel<512><<<row_count, 512, dsa::topk::Cfg<512>::SMEM, stream>>>(P, scores, ld,
-                                                                                                 row_begin, idx);
+        dsa::topk::topk_rows_kernel<1024><<<row_count, 1024, dsa::topk::Cfg<1024>::SMEM, stream>>>(P, scores, ld,
+                                                                                                    row_begin, idx);
     else
         dsa::topk::topk_rows_kernel<256><<<row_count, 256, dsa::topk::Cfg<256>::SMEM, stream>>>(P, scores, ld,
                                                                                                row_begin, idx);

@@ -6,15 +6,16 @@
 //
 // Scores map to order-preserving 32-bit keys (-0.0 folded onto +0.0), so comparing keys
 // as unsigned integers compares the floats as values.  One CTA per row: 256 threads when
-// there are many rows (several CTAs share an SM), 512 when a launch has fewer rows than
+// there are many rows (several CTAs share an SM), 1024 when a launch has fewer rows than
 // SMs (decode), so a long row is not left to 8 warps.
 //
 // Fast path (one HBM read of the row):
 //   * every 16th float4 of the row is sampled; a radix select on the sample (two 11-bit
 //     digits) gives a key t_lo that about 1.2 k keys of the full row are expected to reach;
 //   * one pass over the row (float4 loads, the next chunk in flight while the current one
-//     is filtered) keeps the keys >= t_lo with their indices, each warp in its own
-//     shared-memory segment and in ascending index order (ballot prefix sums, no atomics);
+//     is filtered) keeps the scores >= t_lo (as raw float bits) with their indices, each
+//     warp in its own shared-memory segment and in ascending index order (ballot prefix
+//     sums, predicated stores, no atomics);
 //   * an exact radix select (11/11/10-bit digits) over these candidates gives the k-th
 //     largest key `thr` and how many keys equal to it are taken (smallest indices first);
 //   * the candidates > thr and the first `need_eq` == thr are written in ascending index
@@ -89,15 +90,24 @@ __device__ __forceinline__ void clear_hist(unsigned char *smem, int p) {
     if (threadIdx.x < GROUPS) grp_of<C>(smem, p)[threadIdx.x] = 0u;
 }
 
-// Warp-aggregated count of digit d (d >= NB: no key; the lane still takes part) into the
-// bin and its group (NB / GROUPS consecutive bins).
+// Count of digit d (d >= NB: no key; the lane still takes part) into the bin and its group
+// (NB / GROUPS consecutive bins).  A warp whose lanes all hold one digit (a run of equal
+// keys) adds 32 with one atomic; otherwise each lane adds its own.
 template <int NB>
 __device__ __forceinline__ void hist_add(uint32_t *hist, uint32_t *grp, uint32_t d, int lane) {
-    const unsigned peers = __match_any_sync(FULL, d);
-    if (d < (uint32_t)NB && lane == __ffs(peers) - 1) atomicAdd(&hist[d], (uint32_t)__popc(peers));
-    const uint32_t g = d < (uint32_t)NB ? d / (uint32_t)(NB / GROUPS) : (uint32_t)GROUPS;
-    const unsigned gpeers = __match_any_sync(FULL, g);
-    if (g < (uint32_t)GROUPS && lane == __ffs(gpeers) - 1) atomicAdd(&grp[g], (uint32_t)__popc(gpeers));
+    constexpr uint32_t PER = NB / GROUPS;
+    const uint32_t d0 = __shfl_sync(FULL, d, 0);
+    if (__all_sync(FULL, d == d0)) {
+        if (lane == 0 && d0 < (uint32_t)NB) {
+            atomicAdd(&hist[d0], 32u);
+            atomicAdd(&grp[d0 / PER], 32u);
+        }
+        return;
+    }
+    if (d < (uint32_t)NB) {
+        atomicAdd(&hist[d], 1u);
+        atomicAdd(&grp[d / PER], 1u);
+    }
 }
 
 __device__ __forceinline__ uint32_t warp_incl_scan(uint32_t v, int lane) {
@@ -272,32 +282,30 @@ __device__ __forceinline__ void ordered_output(const float *src, int wb, int we,
     }
 }
 
-// Appends the scores of one float4 group (indices i0..i0+3 of lane's slot, nv of them
-// valid) that reach f_lo to the warp's segment in index order: lanes in order, then the
-// four components.
-template <int SEG>
-__device__ __forceinline__ void keep_group(const float4 v, int i0, int nv, float f_lo, unsigned lt, int &cnt,
+// Appends the scores of one float4 group (indices i0..i0+3 of the lane's slot, nv of them
+// valid) that reach f_lo, as float bits, to the warp's segment in index order: lanes in
+// order, then the four components.  CHECKED = false: all four valid and the segment has
+// room for 128 more (the caller's warp-uniform test), so the stores need no guard.
+template <bool CHECKED>
+__device__ __forceinline__ void keep_group(const float4 v, int i0, int nv, float f_lo, unsigned lt, int seg, int &cnt,
                                           uint32_t *mk, int *mi) {
-    const bool t0 = nv > 0 && v.x >= f_lo, t1 = nv > 1 && v.y >= f_lo;
-    const bool t2 = nv > 2 && v.z >= f_lo, t3 = nv > 3 && v.w >= f_lo;
+    const bool t0 = (!CHECKED || nv > 0) && v.x >= f_lo, t1 = (!CHECKED || nv > 1) && v.y >= f_lo;
+    const bool t2 = (!CHECKED || nv > 2) && v.z >= f_lo, t3 = (!CHECKED || nv > 3) && v.w >= f_lo;
     const unsigned b0 = __ballot_sync(FULL, t0), b1 = __ballot_sync(FULL, t1);
     const unsigned b2 = __ballot_sync(FULL, t2), b3 = __ballot_sync(FULL, t3);
     int off = cnt + __popc(b0 & lt) + __popc(b1 & lt) + __popc(b2 & lt) + __popc(b3 & lt);
-    if (t0) {
-        if (off < SEG) { mk[off] = order_key(v.x); mi[off] = i0; }
-        ++off;
-    }
-    if (t1) {
-        if (off < SEG) { mk[off] = order_key(v.y); mi[off] = i0 + 1; }
-        ++off;
-    }
-    if (t2) {
-        if (off < SEG) { mk[off] = order_key(v.z); mi[off] = i0 + 2; }
-        ++off;
-    }
-    if (t3 && off < SEG) { mk[off] = order_key(v.w); mi[off] = i0 + 3; }
+    if (t0 && (!CHECKED || off < seg)) { mk[off] = __float_as_uint(v.x); mi[off] = i0; }
+    off += t0;
+    if (t1 && (!CHECKED || off < seg)) { mk[off] = __float_as_uint(v.y); mi[off] = i0 + 1; }
+    off += t1;
+    if (t2 && (!CHECKED || off < seg)) { mk[off] = __float_as_uint(v.z); mi[off] = i0 + 2; }
+    off += t2;
+    if (t3 && (!CHECKED || off < seg)) { mk[off] = __float_as_uint(v.w); mi[off] = i0 + 3; }
     cnt += __popc(b0) + __popc(b1) + __popc(b2) + __popc(b3);
 }
+
+// Key of a candidate stored as float bits.
+__device__ __forceinline__ uint32_t cand_key(uint32_t bits) { return order_key(__uint_as_float(bits)); }
 
 // Fast path.  Returns false (nothing written) when the sample misjudged the row.
 template <class C>
@@ -358,10 +366,14 @@ __device__ bool select_row_sampled(const float *src, int n, int K, unsigned char
 #pragma unroll
             for (int g = 0; g < 4; ++g) nx[g] = load4f(src, nbase + 128 * g + 4 * lane, we);
         }
+        const bool whole = base + 512 <= we;   // warp-uniform
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
             const int i0 = base + 128 * g + 4 * lane;
-            keep_group<SEG>(v[g], i0, min(max(we - i0, 0), 4), f_lo, lt, cnt, mk, mi);
+            if (whole && cnt + 128 <= SEG)
+                keep_group<false>(v[g], i0, 4, f_lo, lt, SEG, cnt, mk, mi);
+            else
+                keep_group<true>(v[g], i0, min(max(we - i0, 0), 4), f_lo, lt, SEG, cnt, mk, mi);
         }
         if (nbase < we) {
 #pragma unroll
@@ -373,8 +385,7 @@ __device__ bool select_row_sampled(const float *src, int n, int K, unsigned char
         if (cnt > SEG) scal[3] = 1;
     }
     __syncthreads();
-    int total = 0;
-    for (int w = 0; w < WARPS; ++w) total += seg_cnt[w];
+    const int total = warp_sum(lane < WARPS ? seg_cnt[lane] : 0);
     if (scal[3] != 0 || total < K) return false;   // uniform decision
 
     // ---- exact k-th largest among the candidates (each warp walks its own segment)
@@ -383,7 +394,7 @@ __device__ bool select_row_sampled(const float *src, int n, int K, unsigned char
     const uint32_t thr = radix_select<C>(
         K,
         [&](auto fn) {
-            for (int j = lane; j < cnt_pad; j += 32) fn(j < cnt ? mk[j] : 0u, j < cnt);
+            for (int j = lane; j < cnt_pad; j += 32) fn(j < cnt ? cand_key(mk[j]) : 0u, j < cnt);
         },
         smem, &above);
     const int need_eq = K - above;                   // >= 1
@@ -392,8 +403,9 @@ __device__ bool select_row_sampled(const float *src, int n, int K, unsigned char
     // ---- per-warp counts of > thr and == thr, then ordered writes
     int cg = 0, ce = 0;
     for (int j = lane; j < cnt; j += 32) {
-        cg += mk[j] > thr;
-        ce += mk[j] == thr;
+        const uint32_t key = cand_key(mk[j]);
+        cg += key > thr;
+        ce += key == thr;
     }
     cg = warp_sum(cg);
     ce = warp_sum(ce);
@@ -402,14 +414,11 @@ __device__ bool select_row_sampled(const float *src, int n, int K, unsigned char
         weq[warp] = ce;
     }
     __syncthreads();
-    int gt_off = 0, eq_off = 0;
-    for (int w2 = 0; w2 < warp; ++w2) {
-        gt_off += wgt[w2];
-        eq_off += weq[w2];
-    }
+    int gt_off = warp_sum(lane < warp ? wgt[lane] : 0);
+    int eq_off = warp_sum(lane < warp ? weq[lane] : 0);
     for (int base = 0; base < cnt; base += 32) {
         const int j = base + lane;
-        const uint32_t key = j < cnt ? mk[j] : 0u;
+        const uint32_t key = j < cnt ? cand_key(mk[j]) : 0u;
         const bool g = j < cnt && key > thr, e = j < cnt && key == thr;
         const unsigned bg = __ballot_sync(FULL, g), be = __ballot_sync(FULL, e);
         if (g) {
@@ -556,11 +565,8 @@ __device__ void select_row_general(const float *src, int n, int K, unsigned char
         }
     }
     __syncthreads();
-    int gt_off = 0, eq_off = 0;
-    for (int w2 = 0; w2 < warp; ++w2) {
-        gt_off += w_above[w2] + w_gt[w2];
-        eq_off += w_eq[w2];
-    }
+    int gt_off = warp_sum(lane < warp ? w_above[lane] + w_gt[lane] : 0);
+    int eq_off = warp_sum(lane < warp ? w_eq[lane] : 0);
     ordered_output(src, wb, we, lane, thr, need_eq, count_gt, K, gt_off, eq_off, out);
 }
 
