@@ -260,9 +260,10 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Key length up to which the fused forward runs the attention in the dense ("masked MHA")
 // form over the selected keys: on B200 its contiguous TMA tile loads beat the row gathers
-// up to here even though it multiplies every causal key (measured 3.79 vs 4.10 ms at 4096
-// keys with index_topk 2048).
-constexpr int DENSE_KV_THRESHOLD = 4096;
+// up to here even though it multiplies every causal key.  Measured with index_topk 2048
+// (dense vs gathered ms per prefill): 1.65 vs 2.01 at 2560 keys, 2.25 vs 2.50 at 3072,
+// 2.93 vs 2.99 at 3584, 3.70 vs 3.49 at 4096.
+constexpr int DENSE_KV_THRESHOLD = 3584;
 
 bool dense_for(const dsa_problem_t *p) { return p->block_table == nullptr && p->max_len_k <= DENSE_KV_THRESHOLD; }
 

@@ -15,9 +15,8 @@
 //  * the fp32 score row is written coalesced (128 consecutive keys per query); keys past
 //    pos(t) are never written, tiles past the group's last position are never loaded.
 // FP8: kind::f8f6f4 MMA on e4m3 codes; since the scales are positive, ReLU(a*b*x) =
-// a*b*ReLU(x): per-token scales multiply the finished sum; with ue8m0 block scales (one
-// per head of a query token, one per key token) the query scale of head j joins w[t,j]
-// when the weights are staged and the key scale multiplies the sum.
+// a*b*ReLU(x): the query's scale (per token, or per head with ue8m0 block scales) joins
+// w[t,j] when the weights are staged, and the key's scale multiplies the finished sum.
 //
 // Warp roles (12 warps): 0 TMA producer, 1 MMA issuer, 2 TMEM allocator, 3 idle,
 // 4-7 epilogue for accumulator buffer 0, 8-11 epilogue for buffer 1.
@@ -135,8 +134,16 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     for (int i = tid; i < C::QROWS; i += C::THREADS) {
         const int q = i / 64;
         float wv = q < qcount ? __ldg(w + (int64_t)(t0 + q) * 64 + (i % 64)) : 0.f;
-        if (FP8 && P.ue8m0 && q < qcount)
-            wv *= ue8m0_to_float(__ldg(reinterpret_cast<const uint8_t *>(q_scale) + (int64_t)(t0 + q) * 64 + (i % 64)));
+        if (FP8 && q < qcount) {   // the query's scale joins its head weights (scales are > 0)
+            float qs;
+            if (P.ue8m0) {
+                qs = ue8m0_to_float(__ldg(reinterpret_cast<const uint8_t *>(q_scale) + (int64_t)(t0 + q) * 64 + (i % 64)));
+            } else {
+                qs = __ldg(reinterpret_cast<const float *>(q_scale) + t0 + q);
+                if (P.debug && !(qs > 0.f && qs < INFINITY)) raise_error(ERR_BOUNDS);
+            }
+            wv *= qs;
+        }
         w_s[i] = wv;
     }
     tc_fence_before();
@@ -226,54 +233,69 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
         for (int it = g; it < nitems; it += 2) {
             const int use = it >> 1;
-            if (misc[1] || !mbar_wait(acc_full(g), use & 1)) { misc[1] = 1; break; }
-            tc_fence_after();
             const int j = it / C::NSUB, h = it % C::NSUB;
-            float res[C::QPI];
-#pragma unroll
-            for (int qi = 0; qi < C::QPI; ++qi) {
-                uint32_t v0[32], v1[32];
-                const uint32_t col = (uint32_t)(g * C::N + qi * 64);
-                tmem_ld32(t_lane + col, v0);
-                tmem_ld32(t_lane + col + 32, v1);
-                tmem_wait_ld();
-                // sum over heads of w * ReLU(x): even heads in the low lane, odd heads in
-                // the high lane of packed fp32 FMAs (each lane rounds like a scalar fmaf)
-                const uint64_t *wq2 = reinterpret_cast<const uint64_t *>(w_s + (h * C::QPI + qi) * 64);
-                uint64_t acc = 0;
-#pragma unroll
-                for (int c = 0; c < 32; c += 2)
-                    fma_f32x2(acc, pack_f32x2(fmaxf(__uint_as_float(v0[c]), 0.f), fmaxf(__uint_as_float(v0[c + 1]), 0.f)),
-                              wq2[c / 2]);
-#pragma unroll
-                for (int c = 0; c < 32; c += 2)
-                    fma_f32x2(acc, pack_f32x2(fmaxf(__uint_as_float(v1[c]), 0.f), fmaxf(__uint_as_float(v1[c + 1]), 0.f)),
-                              wq2[16 + c / 2]);
-                float acc0, acc1;
-                unpack_f32x2(acc, acc0, acc1);
-                res[qi] = acc0 + acc1;
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(acc_empty(g));
             const int key = key0 + j * C::BM + row;
-            float ks = 1.f;
+            float ks = 1.f;   // the key's scale, loaded before the accumulator wait
             if (FP8 && key < nkeys_total) {
                 const int kr = key_row(P, rk, key);
                 ks = P.ue8m0 ? ue8m0_to_float(__ldg(reinterpret_cast<const uint8_t *>(k_scale) + kr))
                              : __ldg(reinterpret_cast<const float *>(k_scale) + kr);
             }
+            if (misc[1] || !mbar_wait(acc_full(g), use & 1)) { misc[1] = 1; break; }
+            tc_fence_after();
+            // The item's accumulator columns are read in 2 * QPI chunks of 32 (query qi, head
+            // half): the load of chunk k + 1 is in flight while chunk k is summed, and the
+            // buffer is released as soon as its last chunk has landed.
+            // Sum over heads of w * ReLU(x) on packed fp32 FMAs: even heads in the low lane,
+            // odd heads in the high lane (every lane rounds like a scalar fmaf).  FP8, whose
+            // MMA leaves the epilogue less time, sums heads 0..31 and 32..63 in two
+            // independent chains added at the end; bf16 keeps one chain in head order.
+            float res[C::QPI];
+            uint32_t va[32], vb[32];
+            uint64_t acc = 0, acc_hi = 0;
+            const uint32_t col0 = t_lane + (uint32_t)(g * C::N);
+            tmem_ld32(col0, va);
+            tmem_wait_ld();
+            tmem_regs_ready(va);
+#pragma unroll
+            for (int k = 0; k < 2 * C::QPI; ++k) {
+                const int qi = k >> 1, half = k & 1;
+                uint32_t(&cur)[32] = half ? vb : va;
+                uint32_t(&nxt)[32] = half ? va : vb;
+                if (k + 1 < 2 * C::QPI) tmem_ld32(col0 + (uint32_t)((k + 1) * 32), nxt);
+                if (half == 0) {
+                    acc = 0;
+                    acc_hi = 0;
+                }
+                const uint64_t *wq2 = reinterpret_cast<const uint64_t *>(w_s + (h * C::QPI + qi) * 64 + half * 32);
+                uint64_t &dst = (FP8 && half) ? acc_hi : acc;
+#pragma unroll
+                for (int c = 0; c < 32; c += 2)
+                    fma_f32x2(dst, pack_f32x2(fmaxf(__uint_as_float(cur[c]), 0.f), fmaxf(__uint_as_float(cur[c + 1]), 0.f)),
+                              wq2[c / 2]);
+                if (half == 1) {
+                    float acc0, acc1, acc2, acc3;
+                    unpack_f32x2(acc, acc0, acc1);
+                    unpack_f32x2(acc_hi, acc2, acc3);
+                    res[qi] = FP8 ? (acc0 + acc1) + (acc2 + acc3) : acc0 + acc1;
+                }
+                if (k + 1 < 2 * C::QPI) {
+                    tmem_wait_ld();
+                    tmem_regs_ready(nxt);
+                    if (k + 2 == 2 * C::QPI) {   // the buffer's last chunk has landed
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(acc_empty(g));
+                    }
+                }
+            }
+            if (FP8 && P.debug && key < nkeys_total && !P.ue8m0 && !(ks > 0.f && ks < INFINITY)) raise_error(ERR_BOUNDS);
 #pragma unroll
             for (int qi = 0; qi < C::QPI; ++qi) {
                 const int q = h * C::QPI + qi;
                 if (q < qcount && key <= pos0 + q && key < nkeys_total) {
                     const int t = t0 + q;
-                    float v = res[qi];
-                    if (FP8) {
-                        const float qs = P.ue8m0 ? 1.0f : __ldg(reinterpret_cast<const float *>(q_scale) + t);
-                        if (P.debug && !(qs > 0.f && ks > 0.f && qs < INFINITY && ks < INFINITY)) raise_error(ERR_BOUNDS);
-                        v *= qs * ks;
-                    }
+                    const float v = FP8 ? res[qi] * ks : res[qi];
                     scores[(int64_t)(t - row_begin) * ld + key] = v;
                 }
             }

@@ -169,7 +169,7 @@ dsa_status_t dsa_sparse_mla_fwd(const dsa_problem_t *p, const void *q, const voi
  * Packed caches only (a block table returns DSA_ERR_UNSUPPORTED).
  * dsa_forward uses this form (with idx = NULL, skipping the indexer and the top-k) whenever
  * max_len_k <= topk: every visible key is then selected, and the output is bit-identical
- * to the gathered form.  Above that, up to max_len_k <= 4096 (the short-sequence threshold
+ * to the gathered form.  Above that, up to max_len_k <= 3584 (the short-sequence threshold
  * of this build), dsa_forward runs the indexer and the top-k and then this form restricted
  * to the selected keys; longer problems use dsa_sparse_mla_fwd.
  */

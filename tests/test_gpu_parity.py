@@ -391,6 +391,15 @@ def test_prefill_4k_full_size_sampled():
     _check_forward_rows(inp, rows, chunk=4096)
 
 
+def test_prefill_3k_forward_takes_the_masked_dense_form():
+    # topk < max_len_k <= the short-sequence threshold: dsa_forward runs the indexer and the
+    # top-k, then the dense form restricted to the selected keys (its key blocks group the
+    # keys differently from the gathered form, so the two agree to rounding, not bit for
+    # bit); checked against the oracle on sampled rows
+    inp = dsa_synth.make_workload("prefill_4k", seed=5, device=DEV, L=3072)
+    _check_forward_rows(inp, sample_rows(3072, 2048, n_rand=12, seed=6, edge=4))
+
+
 def test_prefill_32k_full_size_sampled_bench_config():
     inp = dsa_synth.make_workload("prefill_32k", seed=0, device=DEV)
     rows = sample_rows(32768, 2048, n_rand=12, seed=2, edge=4)
