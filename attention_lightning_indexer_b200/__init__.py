@@ -20,6 +20,8 @@ from ._native import (  # noqa: F401
     dsa_forward_noalloc_scratch_bytes,
     dsa_forward_workspace_size,
     dsa_indexer_scores,
+    dsa_indexer_topk_streaming,
+    dsa_indexer_topk_streaming_workspace_size,
     dsa_sparse_mla_fwd,
     dsa_selftest_bounded_wait,
     dsa_set_debug_checks,
@@ -33,6 +35,7 @@ from ._native import (  # noqa: F401
 
 __all__ = [
     "DSA_BF16", "DSA_E4M3", "DSA_E4M3_UE8M0", "DsaError", "DsaProblem", "dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_fwd",
+    "dsa_indexer_topk_streaming", "dsa_indexer_topk_streaming_workspace_size",
     "dsa_dense_mla_fwd", "dsa_cache_write",
     "dsa_forward_workspace_size", "dsa_forward", "dsa_forward_noalloc", "dsa_forward_noalloc_scratch_bytes",
     "dsa_check_device_errors", "dsa_selftest_bounded_wait", "dsa_set_debug_checks", "make_problem",

@@ -32,6 +32,8 @@ _STATUS = {
 EXPORTED = (
     "dsa_indexer_scores",
     "dsa_topk",
+    "dsa_indexer_topk_streaming_workspace_size",
+    "dsa_indexer_topk_streaming",
     "dsa_sparse_mla_fwd",
     "dsa_dense_mla_fwd",
     "dsa_forward_workspace_size",
@@ -99,6 +101,9 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     pp = ctypes.POINTER(DsaProblem)
     lib.dsa_indexer_scores.argtypes = [pp, P, P, P, P, P, P, i64, i32, i32, P]
     lib.dsa_topk.argtypes = [pp, P, i64, i32, i32, P, P]
+    lib.dsa_indexer_topk_streaming_workspace_size.argtypes = [pp, i32]
+    lib.dsa_indexer_topk_streaming_workspace_size.restype = sz
+    lib.dsa_indexer_topk_streaming.argtypes = [pp, P, P, P, P, P, i32, i32, i32, P, P, sz, P]
     lib.dsa_sparse_mla_fwd.argtypes = [pp, P, P, P, P, P, P]
     lib.dsa_dense_mla_fwd.argtypes = [pp, P, P, P, P, P, P]
     lib.dsa_forward_workspace_size.argtypes = [pp, i32]
@@ -115,7 +120,7 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.dsa_status_string.argtypes = [ctypes.c_int]
     lib.dsa_status_string.restype = ctypes.c_char_p
     lib.dsa_abi_version.restype = i32
-    for name in ("dsa_indexer_scores", "dsa_topk", "dsa_sparse_mla_fwd", "dsa_dense_mla_fwd", "dsa_forward",
+    for name in ("dsa_indexer_scores", "dsa_topk", "dsa_indexer_topk_streaming", "dsa_sparse_mla_fwd", "dsa_dense_mla_fwd", "dsa_forward",
                  "dsa_forward_noalloc",
                  "dsa_check_device_errors", "dsa_selftest_bounded_wait", "dsa_cache_write"):
         getattr(lib, name).restype = ctypes.c_int
@@ -196,6 +201,23 @@ def dsa_topk(p: DsaProblem, scores, idx, row_begin: int = 0, row_count: Optional
         row_count = p.total_q - row_begin
     _check(lib.dsa_topk(ctypes.byref(p), _ptr(scores), scores.stride(0), row_begin, row_count, _ptr(idx),
                         _stream(stream)), "dsa_topk")
+
+
+def dsa_indexer_topk_streaming_workspace_size(p: DsaProblem, chunk_q: int = 0) -> int:
+    return int(load().dsa_indexer_topk_streaming_workspace_size(ctypes.byref(p), chunk_q))
+
+
+def dsa_indexer_topk_streaming(p: DsaProblem, q_idx, k_idx, w, idx, workspace, row_begin: int = 0,
+                               row_count: Optional[int] = None, chunk_q: int = 0, q_scale=None, k_scale=None,
+                               stream=None) -> None:
+    """Indexer and top-k without score rows: the same idx as dsa_indexer_scores + dsa_topk."""
+    lib = load()
+    if row_count is None:
+        row_count = p.total_q - row_begin
+    _check(lib.dsa_indexer_topk_streaming(ctypes.byref(p), _ptr(q_idx), _ptr(q_scale), _ptr(k_idx), _ptr(k_scale),
+                                          _ptr(w), row_begin, row_count, chunk_q, _ptr(idx), _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(), _stream(stream)),
+           "dsa_indexer_topk_streaming")
 
 
 def dsa_sparse_mla_fwd(p: DsaProblem, q, kv, idx, out, lse, stream=None) -> None:

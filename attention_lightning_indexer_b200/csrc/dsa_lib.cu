@@ -11,6 +11,7 @@
 #include "cache_write.cuh"
 #include "dsa_common.cuh"
 #include "indexer_tc.cuh"
+#include "select_stream.cuh"
 #include "sparse_mla_pair.cuh"
 #include "topk.cuh"
 
@@ -120,6 +121,20 @@ inline dsa_status_t launch_status() {
 // device current).
 constexpr int MAX_DEVICES = 64;
 
+// Longest key range the streaming selection takes (the sample of a row must fit the
+// threshold kernel's shared memory); longer problems use the two-pass kernels.
+constexpr int STREAM_MAX_KEYS = dsa::topk::STREAM_MAX_SAMPLES / 128 * (dsa::indexer::SAMPLE_STRIDE * 128);
+
+size_t select_smem(int max_len_k) {
+    return (size_t)dsa::topk::StreamCfg::SMEM + 8u * (size_t)((max_len_k + 31) / 32);
+}
+
+template <int QG, bool FP8, int MODE>
+cudaError_t indexer_attr() {
+    return cudaFuncSetAttribute(dsa::indexer::indexer_tc_kernel<QG, FP8, MODE>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, dsa::indexer::TcCfg<QG, FP8>::SMEM);
+}
+
 dsa_status_t set_smem_attrs() {
     static bool done[MAX_DEVICES] = {};
     int dev = -1;
@@ -137,27 +152,30 @@ dsa_status_t set_smem_attrs() {
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(dsa::mla::sparse_mla_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  dsa::mla::PairCfg::SMEM);
+    if (e == cudaSuccess) e = indexer_attr<8, false, dsa::indexer::SCORES>();
+    if (e == cudaSuccess) e = indexer_attr<8, true, dsa::indexer::SCORES>();
+    if (e == cudaSuccess) e = indexer_attr<8, false, dsa::indexer::SAMPLE>();
+    if (e == cudaSuccess) e = indexer_attr<8, true, dsa::indexer::SAMPLE>();
+    if (e == cudaSuccess) e = indexer_attr<8, false, dsa::indexer::FILTER>();
+    if (e == cudaSuccess) e = indexer_attr<8, true, dsa::indexer::FILTER>();
+    if (e == cudaSuccess) e = indexer_attr<1, false, dsa::indexer::SCORES>();
+    if (e == cudaSuccess) e = indexer_attr<1, true, dsa::indexer::SCORES>();
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(dsa::indexer::indexer_tc_kernel<8, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 dsa::indexer::TcCfg<8, false>::SMEM);
+        e = cudaFuncSetAttribute(dsa::topk::sample_threshold_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 dsa::topk::StreamCfg::SMEM);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(dsa::indexer::indexer_tc_kernel<8, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 dsa::indexer::TcCfg<8, true>::SMEM);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(dsa::indexer::indexer_tc_kernel<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 dsa::indexer::TcCfg<1, false>::SMEM);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(dsa::indexer::indexer_tc_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 dsa::indexer::TcCfg<1, true>::SMEM);
+        e = cudaFuncSetAttribute(dsa::topk::select_candidates_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)select_smem(STREAM_MAX_KEYS));
     if (e != cudaSuccess) return DSA_ERR_CUDA;
     done[dev] = true;
     return DSA_OK;
 }
 
-template <int QG, bool FP8>
+template <int QG, bool FP8, int MODE = dsa::indexer::SCORES>
 dsa_status_t indexer_tc_launch(const dsa_problem_t *p, const void *q_idx, const void *q_scale, const void *k_idx,
                                const void *k_scale, const float *w, float *scores, int64_t ld, int row_begin,
-                               int row_count, cudaStream_t stream) {
+                               int row_count, cudaStream_t stream,
+                               dsa::indexer::StreamArgs sa = dsa::indexer::StreamArgs{}) {
     using C = dsa::indexer::TcCfg<QG, FP8>;
     CUtensorMap tq, tk;
     if (!make_tmap_rows(&tq, q_idx, FP8, 128, (uint64_t)p->total_q * 64, 64)) return DSA_ERR_CUDA;
@@ -172,8 +190,8 @@ dsa_status_t indexer_tc_launch(const dsa_problem_t *p, const void *q_idx, const 
         nsplit = (p->max_len_k + C::SPLIT_KEYS - 1) / C::SPLIT_KEYS;
         grid = (unsigned)row_count * (unsigned)nsplit;
     }
-    dsa::indexer::indexer_tc_kernel<QG, FP8><<<grid, C::THREADS, C::SMEM, stream>>>(
-        tq, tk, P, q_scale, k_scale, w, scores, ld, row_begin, row_count, nsplit);
+    dsa::indexer::indexer_tc_kernel<QG, FP8, MODE><<<grid, C::THREADS, C::SMEM, stream>>>(
+        tq, tk, P, q_scale, k_scale, w, scores, ld, row_begin, row_count, nsplit, sa);
     return launch_status();
 }
 
@@ -196,7 +214,7 @@ dsa_status_t indexer_launch(const dsa_problem_t *p, const void *q_idx, const voi
 }
 
 dsa_status_t topk_launch(const dsa_problem_t *p, const float *scores, int64_t ld, int row_begin, int row_count,
-                         int32_t *idx, cudaStream_t stream) {
+                         int32_t *idx, cudaStream_t stream, const uint8_t *row_mask = nullptr) {
     if (row_count == 0) return DSA_OK;
     Problem P = to_dev(p);
     // Fewer rows than SMs (decode): 1024 threads per row; otherwise 256 threads, several
@@ -206,10 +224,10 @@ dsa_status_t topk_launch(const dsa_problem_t *p, const float *scores, int64_t ld
         return DSA_ERR_CUDA;
     if (row_count < n_sm)
         dsa::topk::topk_rows_kernel<1024><<<row_count, 1024, dsa::topk::Cfg<1024>::SMEM, stream>>>(P, scores, ld,
-                                                                                                    row_begin, idx);
+                                                                                                    row_begin, idx, row_mask);
     else
         dsa::topk::topk_rows_kernel<256><<<row_count, 256, dsa::topk::Cfg<256>::SMEM, stream>>>(P, scores, ld,
-                                                                                               row_begin, idx);
+                                                                                               row_begin, idx, row_mask);
     return launch_status();
 }
 
@@ -273,6 +291,89 @@ int effective_chunk(const dsa_problem_t *p, int32_t chunk_q) {
     int T = p->total_q > 0 ? p->total_q : 1;
     if (chunk_q <= 0 || chunk_q > T) return T;
     return chunk_q;
+}
+
+// ---- streaming indexer -> top-k (no score rows; see select_stream.cuh)
+
+struct StreamWs {
+    float *scores;   // [chunk, ld]: rows the threshold misjudged are redone from full scores
+    float *sample;   // [chunk, lds]
+    float *f_lo;     // [chunk]
+    int *cnt;        // [chunk]
+    uint8_t *flag;   // [chunk]
+    uint2 *cand;     // [chunk, cap]
+    int64_t ld, lds;
+    int cap;
+};
+
+bool streaming_applies(const dsa_problem_t *p) {
+    return p->cu_q == nullptr && p->max_len_k > p->topk && p->max_len_k <= STREAM_MAX_KEYS;
+}
+
+// Bytes of the streaming workspace for chunks of `chunk` rows; fills *ws when base is given.
+size_t stream_layout(const dsa_problem_t *p, int chunk, unsigned char *base, StreamWs *ws) {
+    const int64_t ld = scores_ld(p);
+    const int64_t span = (int64_t)dsa::indexer::SAMPLE_STRIDE * 128;
+    const int64_t lds = ((p->max_len_k + span - 1) / span) * 128;
+    const int cap = dsa::topk::STREAM_CAP;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off = align_up(off + bytes, 256);
+        return base ? base + at : nullptr;
+    };
+    unsigned char *sc = take((size_t)chunk * (size_t)ld * 4);
+    unsigned char *sm = take((size_t)chunk * (size_t)lds * 4);
+    unsigned char *fl = take((size_t)chunk * 4);
+    unsigned char *cn = take((size_t)chunk * 4);
+    unsigned char *fg = take((size_t)chunk);
+    unsigned char *cd = take((size_t)chunk * (size_t)cap * 8);
+    if (ws) {
+        ws->scores = reinterpret_cast<float *>(sc);
+        ws->sample = reinterpret_cast<float *>(sm);
+        ws->f_lo = reinterpret_cast<float *>(fl);
+        ws->cnt = reinterpret_cast<int *>(cn);
+        ws->flag = fg;
+        ws->cand = reinterpret_cast<uint2 *>(cd);
+        ws->ld = ld;
+        ws->lds = lds;
+        ws->cap = cap;
+    }
+    return off;
+}
+
+template <bool FP8>
+dsa_status_t stream_chunk(const dsa_problem_t *p, const void *q_idx, const void *q_scale, const void *k_idx,
+                          const void *k_scale, const float *w, int r0, int rc, int32_t *idx, const StreamWs &ws,
+                          cudaStream_t s) {
+    using namespace dsa::indexer;
+    dsa_status_t st;
+    if (cudaMemsetAsync(ws.cnt, 0, (size_t)rc * 4, s) != cudaSuccess) return DSA_ERR_CUDA;
+    if ((st = indexer_tc_launch<8, FP8, SAMPLE>(p, q_idx, q_scale, k_idx, k_scale, w, ws.sample, ws.lds, r0, rc,
+                                                s)) != DSA_OK)
+        return st;
+    Problem P = to_dev(p);
+    dsa::topk::sample_threshold_kernel<<<rc, dsa::topk::STREAM_NT, dsa::topk::StreamCfg::SMEM, s>>>(
+        P, ws.sample, ws.lds, SAMPLE_STRIDE * 128, r0, ws.f_lo);
+    if ((st = launch_status()) != DSA_OK) return st;
+    StreamArgs fa{};
+    fa.f_lo = ws.f_lo;
+    fa.cnt = ws.cnt;
+    fa.cand = ws.cand;
+    fa.cap = ws.cap;
+    if ((st = indexer_tc_launch<8, FP8, FILTER>(p, q_idx, q_scale, k_idx, k_scale, w, nullptr, 0, r0, rc, s, fa)) !=
+        DSA_OK)
+        return st;
+    dsa::topk::select_candidates_kernel<<<rc, dsa::topk::STREAM_NT, select_smem(p->max_len_k), s>>>(
+        P, ws.cnt, ws.cand, ws.cap, r0, idx, ws.flag);
+    if ((st = launch_status()) != DSA_OK) return st;
+    // rows whose candidates could not decide: full score rows and the two-pass selection
+    StreamArgs ra{};
+    ra.row_mask = ws.flag;
+    if ((st = indexer_tc_launch<8, FP8, SCORES>(p, q_idx, q_scale, k_idx, k_scale, w, ws.scores, ws.ld, r0, rc, s,
+                                                ra)) != DSA_OK)
+        return st;
+    return topk_launch(p, ws.scores, ws.ld, r0, rc, idx, s, ws.flag);
 }
 
 }  // namespace
@@ -401,6 +502,51 @@ dsa_status_t dsa_forward(const dsa_problem_t *p, const void *q_idx, const void *
         if (st != DSA_OK) return st;
     }
     return mla_launch(p, q, kv, idx, out, lse, s, dense_for(p));
+}
+
+size_t dsa_indexer_topk_streaming_workspace_size(const dsa_problem_t *p, int32_t chunk_q) {
+    if (check_problem(p) != DSA_OK) return 0;
+    const int chunk = effective_chunk(p, chunk_q);
+    if (!streaming_applies(p)) return align_up((size_t)chunk * (size_t)scores_ld(p) * sizeof(float), 256);
+    return stream_layout(p, chunk, nullptr, nullptr);
+}
+
+dsa_status_t dsa_indexer_topk_streaming(const dsa_problem_t *p, const void *q_idx, const void *q_scale,
+                                        const void *k_idx, const void *k_scale, const float *w, int32_t row_begin,
+                                        int32_t row_count, int32_t chunk_q, int32_t *idx, void *workspace,
+                                        size_t workspace_bytes, dsa_stream_t stream) {
+    dsa_status_t st = check_problem(p);
+    if (st != DSA_OK) return st;
+    if (row_begin < 0 || row_count < 0 || row_begin + row_count > p->total_q) return DSA_ERR_INVALID_ARG;
+    if (row_count == 0) return DSA_OK;
+    if (!q_idx || !k_idx || !w || !idx) return DSA_ERR_INVALID_ARG;
+    if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(w) || !aligned16(idx)) return DSA_ERR_INVALID_ARG;
+    if (p->idx_dtype != DSA_BF16 && (!q_scale || !k_scale)) return DSA_ERR_INVALID_ARG;
+    const size_t need = dsa_indexer_topk_streaming_workspace_size(p, chunk_q);
+    if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return DSA_ERR_WORKSPACE;
+    if ((st = set_smem_attrs()) != DSA_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    const int chunk = effective_chunk(p, chunk_q);
+    const bool fp8 = p->idx_dtype != DSA_BF16;
+    StreamWs ws{};
+    const bool streaming = streaming_applies(p);
+    if (streaming) stream_layout(p, chunk, static_cast<unsigned char *>(workspace), &ws);
+    for (int r0 = row_begin; r0 < row_begin + row_count; r0 += chunk) {
+        const int rc = row_begin + row_count - r0 < chunk ? row_begin + row_count - r0 : chunk;
+        int32_t *out = idx + (int64_t)(r0 - row_begin) * p->topk;
+        if (streaming) {
+            st = fp8 ? stream_chunk<true>(p, q_idx, q_scale, k_idx, k_scale, w, r0, rc, out, ws, s)
+                     : stream_chunk<false>(p, q_idx, q_scale, k_idx, k_scale, w, r0, rc, out, ws, s);
+        } else {   // ragged batches and very long rows: the two-pass kernels (the same indices)
+            float *scores = static_cast<float *>(workspace);
+            const int64_t ld = scores_ld(p);
+            st = indexer_launch(p, q_idx, q_scale, k_idx, k_scale, w, scores, ld, r0, rc, s);
+            if (st == DSA_OK) st = topk_launch(p, scores, ld, r0, rc, out, s);
+        }
+        if (st != DSA_OK) return st;
+    }
+    return DSA_OK;
 }
 
 dsa_status_t dsa_cache_write(int32_t n_tokens, const void *k_idx_raw, const void *kv_raw, const int32_t *positions,

@@ -20,6 +20,14 @@
 //
 // Warp roles (12 warps): 0 TMA producer, 1 MMA issuer, 2 TMEM allocator, 3 idle,
 // 4-7 epilogue for accumulator buffer 0, 8-11 epilogue for buffer 1.
+//
+// Output modes (the streaming selection of the fused indexer -> top-k):
+//   SCORES   the score rows (optionally only for the groups holding a row of row_mask);
+//   SAMPLE   every SAMPLE_STRIDE-th key tile only, written compactly: sample column
+//            j' * 128 + r holds key j' * SAMPLE_STRIDE * 128 + r;
+//   FILTER   no score rows: each score >= the row's threshold f_lo is appended as (float
+//            bits, key) to the row's candidate list (one atomic per warp and query for the
+//            slots; the order of the list is not defined), the count in cnt.
 #pragma once
 
 #include "dsa_common.cuh"
@@ -27,6 +35,18 @@
 
 namespace dsa {
 namespace indexer {
+
+enum Mode { SCORES = 0, SAMPLE = 1, FILTER = 2 };
+constexpr int SAMPLE_STRIDE = 16;
+
+// Arguments of the streaming modes.
+struct StreamArgs {
+    const uint8_t *row_mask;   // SCORES: score only groups with a nonzero row_mask[t - row_begin] (nullptr: all)
+    const float *f_lo;         // FILTER: per-row threshold
+    int *cnt;                  // FILTER: per-row candidate count (zeroed by the caller)
+    uint2 *cand;               // FILTER: [rows, cap] candidates (float bits, key)
+    int cap;
+};
 
 template <int QG, bool FP8>
 struct TcCfg {
@@ -59,12 +79,14 @@ struct TcCfg {
     static_assert(SMEM <= 232448, "shared memory budget");
 };
 
-template <int QG, bool FP8>
+template <int QG, bool FP8, int MODE>
 __global__ void __launch_bounds__(384, 1)
 indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k, Problem P,
                   const void *__restrict__ q_scale, const void *__restrict__ k_scale, const float *__restrict__ w,
-                  float *__restrict__ scores, int64_t ld, int row_begin, int row_count, int nsplit) {
+                  float *__restrict__ scores, int64_t ld, int row_begin, int row_count, int nsplit, StreamArgs sa) {
     using C = TcCfg<QG, FP8>;
+    static_assert(MODE == SCORES || (QG > 1 && C::NSUB == 2), "streaming modes: one query group per CTA, "
+                                                              "one item half per epilogue warpgroup");
     using namespace sm100;
     extern __shared__ __align__(1024) unsigned char smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -96,7 +118,13 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         nkeys_total = row_ok(P, ri) ? min(visible_keys(ri), key0 + C::SPLIT_KEYS) : 0;
     }
     if (nkeys_total <= key0) return;                          // uniform for the whole CTA
-    const int ntiles = (nkeys_total - key0 + C::BM - 1) / C::BM;
+    if (MODE == SCORES && sa.row_mask != nullptr) {           // uniform: the same rows for every thread
+        bool any = false;
+        for (int q = 0; q < qcount; ++q) any = any || sa.row_mask[t0 + q - row_begin] != 0;
+        if (!any) return;
+    }
+    const int tstride = MODE == SAMPLE ? SAMPLE_STRIDE : 1;  // key tiles advanced per tile processed
+    const int ntiles = ((nkeys_total - key0 + C::BM - 1) / C::BM + tstride - 1) / tstride;
     const int nitems = ntiles * C::NSUB;
 
     const uint32_t sbase = smem_u32(smem);
@@ -167,7 +195,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (misc[1]) break;
             mbar_expect_tx(k_full(s), C::KTILE_BYTES);
             issued = j + 1;
-            const int kk0 = key0 + j * C::BM;
+            const int kk0 = key0 + j * tstride * C::BM;
             for (int a = 0; a < C::ATOMS; ++a) {
                 const uint32_t dst = k_s + s * C::KTILE_BYTES + a * C::KATOM_BYTES;
                 if (P.block_table == nullptr) {
@@ -231,10 +259,16 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const int quarter = warp & 3;             // TMEM lane quarter this warp may access
         const int row = quarter * 32 + lane;      // key row inside the tile
         const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
+        float th[C::QPI];   // FILTER: the thresholds of this warpgroup's queries (h == g)
+#pragma unroll
+        for (int qi = 0; qi < C::QPI; ++qi) {
+            const int q = g * C::QPI + qi;
+            th[qi] = (MODE == FILTER && q < qcount) ? __ldg(sa.f_lo + (t0 + q - row_begin)) : 0.f;
+        }
         for (int it = g; it < nitems; it += 2) {
             const int use = it >> 1;
             const int j = it / C::NSUB, h = it % C::NSUB;
-            const int key = key0 + j * C::BM + row;
+            const int key = key0 + j * tstride * C::BM + row;
             float ks = 1.f;   // the key's scale, loaded before the accumulator wait
             if (FP8 && key < nkeys_total) {
                 const int kr = key_row(P, rk, key);
@@ -290,13 +324,38 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 }
             }
             if (FP8 && P.debug && key < nkeys_total && !P.ue8m0 && !(ks > 0.f && ks < INFINITY)) raise_error(ERR_BOUNDS);
+            if (MODE == FILTER) {
+                // each query is the same for the whole warp: the warp reserves its slots of
+                // the QPI rows with independent atomics (issued together), then stores
+                unsigned m[C::QPI];
+                int base[C::QPI];
 #pragma unroll
-            for (int qi = 0; qi < C::QPI; ++qi) {
-                const int q = h * C::QPI + qi;
-                if (q < qcount && key <= pos0 + q && key < nkeys_total) {
-                    const int t = t0 + q;
-                    const float v = FP8 ? res[qi] * ks : res[qi];
-                    scores[(int64_t)(t - row_begin) * ld + key] = v;
+                for (int qi = 0; qi < C::QPI; ++qi) {
+                    const int q = h * C::QPI + qi;
+                    const bool valid = q < qcount && key <= pos0 + q && key < nkeys_total;
+                    res[qi] = FP8 ? res[qi] * ks : res[qi];
+                    m[qi] = __ballot_sync(0xffffffffu, valid && res[qi] >= th[qi]);
+                    base[qi] = 0;
+                    if (lane == 0 && m[qi] != 0u) base[qi] = atomicAdd(sa.cnt + (t0 + q - row_begin), __popc(m[qi]));
+                }
+#pragma unroll
+                for (int qi = 0; qi < C::QPI; ++qi) {
+                    const int t = t0 + h * C::QPI + qi;
+                    const int b = __shfl_sync(0xffffffffu, base[qi], 0);
+                    const int slot = b + __popc(m[qi] & ((1u << lane) - 1u));
+                    if (((m[qi] >> lane) & 1u) && slot < sa.cap)
+                        sa.cand[(int64_t)(t - row_begin) * sa.cap + slot] = make_uint2(__float_as_uint(res[qi]), (uint32_t)key);
+                }
+            } else {
+#pragma unroll
+                for (int qi = 0; qi < C::QPI; ++qi) {
+                    const int q = h * C::QPI + qi;
+                    if (q < qcount && key <= pos0 + q && key < nkeys_total) {
+                        const int t = t0 + q;
+                        const float v = FP8 ? res[qi] * ks : res[qi];
+                        const int col = MODE == SAMPLE ? j * C::BM + row : key;
+                        scores[(int64_t)(t - row_begin) * ld + col] = v;
+                    }
                 }
             }
         }

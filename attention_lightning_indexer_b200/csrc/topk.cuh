@@ -570,13 +570,16 @@ __device__ void select_row_general(const float *src, int n, int K, unsigned char
     ordered_output(src, wb, we, lane, thr, need_eq, count_gt, K, gt_off, eq_off, out);
 }
 
-// grid = row_count CTAs of NT threads, dynamic shared memory Cfg<NT>::SMEM bytes.
+// grid = row_count CTAs of NT threads, dynamic shared memory Cfg<NT>::SMEM bytes.  With a
+// row_mask only the rows r with row_mask[r] != 0 are selected (the others are untouched).
 template <int NT>
 __global__ void __launch_bounds__(NT, NT >= 512 ? 1 : 3) topk_rows_kernel(Problem P, const float *__restrict__ scores, int64_t ld,
-                                                       int row_begin, int32_t *__restrict__ idx) {
+                                                       int row_begin, int32_t *__restrict__ idx,
+                                                       const uint8_t *__restrict__ row_mask) {
     using C = Cfg<NT>;
     extern __shared__ __align__(16) unsigned char smem[];
     const int r = blockIdx.x;
+    if (row_mask != nullptr && row_mask[r] == 0) return;
     const int K = P.topk;
     int32_t *out = idx + (int64_t)r * K;
     const RowInfo ri = row_info(P, row_begin + r);

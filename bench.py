@@ -43,10 +43,10 @@ FLOP_PER_PAIR_MLA = 128 * (576 + 512) * 2       # per (query, selected key) pair
 # sha256 of the source file it was captured from; reported only while the source is
 # unchanged.
 TRAFFIC = {
-    # ncu capture of the 4096-query prefill launch: 1.142 GB of DRAM traffic (q reads and
-    # out writes, both proportional to the query count; kv rows come from L2), scaled x8 to
-    # the 32768-query launch of the 32K step
-    "sparse_mla": {"bytes_per_launch": 1.14244e9 * 8, "src_sha": "2de55da9dd0e8b6b"},
+    # ncu capture of the 4096-query prefill launch: 1.142 GB of DRAM traffic (643 MB read,
+    # 499 MB written: q reads and out writes, both proportional to the query count; kv rows
+    # come from L2), scaled x8 to the 32768-query launch of the 32K step
+    "sparse_mla": {"bytes_per_launch": 1.142312e9 * 8, "src_sha": "fa50549e97859dac"},
 }
 
 
@@ -644,7 +644,27 @@ def run_kernel(args, local):
     r0 = T - rows
     ld = dsa.scores_ld(inp["max_len_k"])
     stream = torch.cuda.current_stream(dev)
-    if args.kernel in ("indexer", "topk"):
+    if args.kernel in ("indexer_topk", "indexer_topk_streaming"):
+        # the selection of the whole workload in its chunks: two passes through score rows,
+        # or the streaming path (no score rows); the same indices either way
+        ch = args.chunk or wl.chunk or T
+        idx = torch.empty((T, inp["topk"]), dtype=torch.int32, device=dev)
+        if args.kernel == "indexer_topk":
+            scores = torch.empty((min(ch, T), ld), dtype=torch.float32, device=dev)
+
+            def fn():
+                for c0 in range(0, T, ch):
+                    rc = min(ch, T - c0)
+                    dsa.dsa_indexer_scores(p, fa["q_idx"], fa["k_idx"], inp["w"], scores, row_begin=c0, row_count=rc,
+                                           q_scale=fa["q_scale"], k_scale=fa["k_scale"], stream=stream)
+                    dsa.dsa_topk(p, scores, idx[c0:c0 + rc], row_begin=c0, row_count=rc, stream=stream)
+        else:
+            ws_s = torch.empty(dsa.dsa_indexer_topk_streaming_workspace_size(p, ch), dtype=torch.uint8, device=dev)
+            fn = lambda: dsa.dsa_indexer_topk_streaming(p, fa["q_idx"], fa["k_idx"], inp["w"], idx, ws_s,
+                                                        chunk_q=ch, q_scale=fa["q_scale"], k_scale=fa["k_scale"],
+                                                        stream=stream)
+        rows, r0 = T, 0
+    elif args.kernel in ("indexer", "topk"):
         scores = torch.empty((rows, ld), dtype=torch.float32, device=dev)
         idx = torch.empty((rows, inp["topk"]), dtype=torch.int32, device=dev)
         dsa.dsa_indexer_scores(p, fa["q_idx"], fa["k_idx"], inp["w"], scores, row_begin=r0, row_count=rows,
@@ -742,7 +762,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode_b64 secondary measurement")
     ap.add_argument("--e2e-chunk", type=int, default=2048, help="query rows per pipelined chunk of the e2e step")
-    ap.add_argument("--kernel", choices=("indexer", "topk", "sparse_mla", "dense_mla", "cache_write"), default=None,
+    ap.add_argument("--kernel", choices=("indexer", "topk", "indexer_topk", "indexer_topk_streaming", "sparse_mla",
+                                         "dense_mla", "cache_write"), default=None,
                     help="time one kernel on a bounded slice (for profilers) instead of the full step")
     ap.add_argument("--rows", type=int, default=0, help="query rows for --kernel (default: one chunk)")
     args = ap.parse_args()

@@ -137,6 +137,35 @@ dsa_status_t dsa_topk(const dsa_problem_t *p, const float *scores, int64_t ld_sc
                       int32_t row_begin, int32_t row_count, int32_t *idx, dsa_stream_t stream);
 
 /*
+ * Indexer and top-k fused without score rows ("DeepSeek-V3.2 tech report summary", §1 DSA,
+ * ① and ②): idx[r, :] for the rows t = row_begin + r receives exactly what
+ * dsa_indexer_scores followed by dsa_topk would write (the same indices in the same slots),
+ * computed chunk_q rows at a time (0 = all rows at once) as follows.
+ *  1. The indexer scores every 16th tile of 128 keys of each row (a sample).
+ *  2. A per-row threshold is taken from that sample, chosen so that about 1.2 * topk keys
+ *     reach it.
+ *  3. The indexer runs again over all keys and keeps only the scores that reach the
+ *     threshold, as an unordered list of candidates.
+ *  4. The selection runs over the candidates.
+ * A row whose threshold let fewer than topk keys through, or more than the list holds, is
+ * redone from its full score row.  So the result never depends on the threshold, only the
+ * time does.
+ * This path applies to one sequence without cu arrays and max_len_k <= 229376. Ragged
+ * batches and longer rows run the two-pass kernels on the workspace, with the same result.
+ *   idx       : [row_count, topk] int32
+ *   workspace : device, >= dsa_indexer_topk_streaming_workspace_size(p, chunk_q) bytes,
+ *               256-byte aligned (it includes one chunk of score rows for the rows that
+ *               are redone)
+ * Other tensors, scales and errors as dsa_indexer_scores.
+ */
+size_t dsa_indexer_topk_streaming_workspace_size(const dsa_problem_t *p, int32_t chunk_q);
+dsa_status_t dsa_indexer_topk_streaming(const dsa_problem_t *p, const void *q_idx, const void *q_scale,
+                                        const void *k_idx, const void *k_scale, const float *w,
+                                        int32_t row_begin, int32_t row_count, int32_t chunk_q,
+                                        int32_t *idx, void *workspace, size_t workspace_bytes,
+                                        dsa_stream_t stream);
+
+/*
  * Sparse MLA forward in MQA mode ("DeepSeek-V3.2 tech report summary", §1 DSA,
  * MLA-based implementation: each latent KV entry is shared by all query heads;
  * latent = 512 KV-LoRA + 64 RoPE per "Model techniques map -- DeepSeek-V3.2",
