@@ -37,7 +37,7 @@ namespace dsa {
 namespace indexer {
 
 enum Mode { SCORES = 0, SAMPLE = 1, FILTER = 2 };
-constexpr int SAMPLE_STRIDE = 16;
+constexpr int SAMPLE_STRIDE = 32;
 
 // Arguments of the streaming modes.
 struct StreamArgs {

@@ -8,8 +8,9 @@
 // The indexer runs twice on the tensor cores: once over every SAMPLE_STRIDE-th key tile
 // (a sample row per query), once over all tiles writing only the scores that reach a
 // per-row threshold f_lo (an unordered candidate list).  In between,
-// sample_threshold_kernel takes f_lo from the sample (the same two-digit radix estimate
-// as the top-k's fast path: about 1.2 k keys of the row are expected to reach it).
+// sample_threshold_kernel takes f_lo from the sample (the two-digit radix estimate of the
+// top-k's fast path, with a wider margin: about 1.4 k keys of the row are expected to
+// reach it).
 // select_candidates_kernel then selects over the candidates.  This is exact whenever at
 // least k keys reached f_lo and none was dropped: the k-th largest score is then >= f_lo,
 // so every key that can be selected, ties included, is a candidate.  Otherwise the row is
@@ -84,7 +85,9 @@ sample_threshold_kernel(Problem P, const float *__restrict__ sample, int64_t lds
     for (int i = tid; i < ns; i += STREAM_NT) keys[i] = order_key(__ldg(src + i));
     clear_hist<C>(smem, 0);
     __syncthreads();
-    const int target = min(ns, (int)((1.2 * K * (double)ns) / (double)n) + 16);
+    // about 1.4 k keys of the row are expected to reach the threshold: a row that falls
+    // short of k is redone from full scores, which costs more than the extra candidates
+    const int target = min(ns, (int)((1.4 * K * (double)ns) / (double)n) + 8);
     const int ns_pad = (ns + STREAM_NT - 1) / STREAM_NT * STREAM_NT;
     int dummy;
     const uint32_t t_lo = radix_select<C>(

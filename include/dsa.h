@@ -141,8 +141,8 @@ dsa_status_t dsa_topk(const dsa_problem_t *p, const float *scores, int64_t ld_sc
  * ① and ②): idx[r, :] for the rows t = row_begin + r receives exactly what
  * dsa_indexer_scores followed by dsa_topk would write (the same indices in the same slots),
  * computed chunk_q rows at a time (0 = all rows at once) as follows.
- *  1. The indexer scores every 16th tile of 128 keys of each row (a sample).
- *  2. A per-row threshold is taken from that sample, chosen so that about 1.2 * topk keys
+ *  1. The indexer scores every 32nd tile of 128 keys of each row (a sample).
+ *  2. A per-row threshold is taken from that sample, chosen so that about 1.4 * topk keys
  *     reach it.
  *  3. The indexer runs again over all keys and keeps only the scores that reach the
  *     threshold, as an unordered list of candidates.
@@ -150,7 +150,7 @@ dsa_status_t dsa_topk(const dsa_problem_t *p, const float *scores, int64_t ld_sc
  * A row whose threshold let fewer than topk keys through, or more than the list holds, is
  * redone from its full score row.  So the result never depends on the threshold, only the
  * time does.
- * This path applies to one sequence without cu arrays and max_len_k <= 229376. Ragged
+ * This path applies to one sequence without cu arrays and max_len_k <= 458752. Ragged
  * batches and longer rows run the two-pass kernels on the workspace, with the same result.
  *   idx       : [row_count, topk] int32
  *   workspace : device, >= dsa_indexer_topk_streaming_workspace_size(p, chunk_q) bytes,

@@ -15,7 +15,7 @@ import torch
 import attention_lightning_indexer_b200 as dsa
 import dsa_synth
 from gpu_utils import sorted_rows
-from test_gpu_parity import _check_forward_rows, _gpu_scores, _scales
+from test_gpu_parity import _gpu_scores, _scales
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -81,12 +81,12 @@ def test_streaming_all_tied_rows_take_index_order_and_overflow_is_redone():
 
 
 def test_streaming_misjudged_threshold_is_redone():
-    # the sampled tiles (every 16th tile of 128 keys) get keys 8x larger than the rest, so
+    # the sampled tiles (every 32nd tile of 128 keys) get keys 8x larger than the rest, so
     # the sample sets the threshold far too high and fewer than k keys reach it
     L, k = 8192, 1024
     inp = dsa_synth.make_prefill(L, topk=k, seed=55, device=DEV, with_latent=False)
     kk = inp["k_idx"].float()
-    for j in range(0, L, 16 * 128):
+    for j in range(0, L, 32 * 128):
         kk[j:j + 128] *= 8.0
     inp["k_idx"] = kk.to(torch.bfloat16)
     p = dsa.problem_from_inputs(inp)
