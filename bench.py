@@ -45,8 +45,9 @@ FLOP_PER_PAIR_MLA = 128 * (576 + 512) * 2       # per (query, selected key) pair
 TRAFFIC = {
     # ncu capture of the 4096-query prefill launch: 1.142 GB of DRAM traffic (643 MB read,
     # 499 MB written: q reads and out writes, both proportional to the query count; kv rows
-    # come from L2), scaled x8 to the 32768-query launch of the 32K step
-    "sparse_mla": {"bytes_per_launch": 1.142312e9 * 8, "src_sha": "fa50549e97859dac"},
+    # come from L2), scaled x8 to the 32768-query launch of the 32K step (that prefill only:
+    # at 128K the kv rows no longer fit in L2)
+    "sparse_mla": {"bytes_per_launch": 1.142312e9 * 8, "total_q": 32768, "src_sha": "fa50549e97859dac"},
 }
 
 
@@ -401,7 +402,8 @@ def _breakdown(dsa, p, inp, fa, chunk, dev, stream, flush, reps=2, decode=False)
     kd = kernels[dom]
     src = {"indexer": "indexer_tc.cuh", "topk": "topk.cuh", "sparse_mla": "sparse_mla_pair.cuh"}[dom]
     tr = TRAFFIC.get(dom)
-    traffic = tr["bytes_per_launch"] if tr and tr.get("src_sha") == _src_sha(src) else None
+    traffic = (tr["bytes_per_launch"] if tr and tr.get("src_sha") == _src_sha(src) and not decode
+               and inp["total_q"] == tr.get("total_q") and "q_idx8" not in inp else None)
     if dom == "topk" or decode:
         roof = {"bound": "hbm", "achieved": kd["gbs"], "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": kd["gbs"] / pk["hbm_gbs"], "traffic": traffic}
