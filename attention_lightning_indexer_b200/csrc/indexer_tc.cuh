@@ -80,7 +80,7 @@ struct TcCfg {
 };
 
 template <int QG, bool FP8, int MODE>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(384, (QG == 1 && !FP8) ? 2 : 1)
 indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k, Problem P,
                   const void *__restrict__ q_scale, const void *__restrict__ k_scale, const float *__restrict__ w,
                   float *__restrict__ scores, int64_t ld, int row_begin, int row_count, int nsplit, StreamArgs sa) {
