@@ -18,8 +18,11 @@
 // a*b*ReLU(x): the query's scale (per token, or per head with ue8m0 block scales) joins
 // w[t,j] when the weights are staged, and the key's scale multiplies the finished sum.
 //
-// Warp roles (12 warps): 0 TMA producer, 1 MMA issuer, 2 TMEM allocator, 3 idle,
-// 4-7 epilogue for accumulator buffer 0, 8-11 epilogue for buffer 1.
+// Warp roles: 0 TMA producer, 1 MMA issuer, 2 TMEM allocator, 3 idle; then the epilogue
+// warpgroups.  bf16 and decode: 4-7 for accumulator buffer 0, 8-11 for buffer 1 (12 warps).
+// FP8 query groups: 4-7 and 12-15 for buffer 0 and 8-11 and 16-19 for buffer 1, each
+// warpgroup summing two of the item's four queries (20 warps; setmaxnreg moves registers
+// from the first warpgroup to the epilogue).
 //
 // Output modes (the streaming selection of the fused indexer -> top-k):
 //   SCORES   the score rows (optionally only for the groups holding a row of row_mask);
@@ -74,13 +77,23 @@ struct TcCfg {
     static constexpr int NBARS = 1 + 2 * STAGES + 4 + 1;   // ... + drain
     static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
     static constexpr int SMEM = OFF_MISC + 16;
-    static constexpr int THREADS = 384;
+    // Epilogue warpgroups: two (one per accumulator buffer, each summing the buffer's QPI
+    // queries), or for FP8 query groups four (two per buffer, QPI / 2 queries each): the
+    // e4m3 MMA leaves the epilogue half the time, and more warps hide its latencies.
+    static constexpr int EPI_WG = (FP8 && QG > 1) ? 4 : 2;
+    static constexpr int EPI_SPLIT = EPI_WG / 2;            // warpgroups per accumulator buffer
+    static constexpr int QPW = QPI / EPI_SPLIT;             // queries per warpgroup per item
+    static constexpr int THREADS = 128 * (1 + EPI_WG);
+    // register split when EPI_WG == 4 (setmaxnreg): 128 x REG_LOW + 512 x REG_HIGH must not
+    // exceed 640 x the registers a thread is launched with (96)
+    static constexpr int REG_LOW = 56, REG_HIGH = 104;
     static constexpr int SPLIT_KEYS = 4096;                 // key range of one CTA when QG == 1
+    static_assert(EPI_WG == 2 || 128 * REG_LOW + 512 * REG_HIGH <= 640 * 96, "register split");
     static_assert(SMEM <= 232448, "shared memory budget");
 };
 
 template <int QG, bool FP8, int MODE>
-__global__ void __launch_bounds__(384, (QG == 1 && !FP8) ? 2 : 1)
+__global__ void __launch_bounds__(TcCfg<QG, FP8>::THREADS, (QG == 1 && !FP8) ? 2 : 1)
 indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k, Problem P,
                   const void *__restrict__ q_scale, const void *__restrict__ k_scale, const float *__restrict__ w,
                   float *__restrict__ scores, int64_t ld, int row_begin, int row_count, int nsplit, StreamArgs sa) {
@@ -152,7 +165,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(acc_full(b), 1);
-            mbar_init(acc_empty(b), 4);
+            mbar_init(acc_empty(b), 4 * C::EPI_SPLIT);
         }
         mbar_init(drain, 1);
         misc[1] = 0;
@@ -179,6 +192,9 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     tc_fence_after();
     const uint32_t tmem = misc[0];
 
+    if (warp < 4) {
+    // with four epilogue warpgroups the first warpgroup gives registers to the epilogue
+    if (C::EPI_WG == 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REG_LOW));
     if (warp == 0 && lane == 0) {
         // ------------------------------------------------ TMA producer
         prefetch_tmap(&tm_q);
@@ -253,16 +269,22 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             mma_commit(drain);
             mbar_wait(drain, 0);
         }
-    } else if (warp >= 4) {
+    }
+    } else {
+        if (C::EPI_WG == 4) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::REG_HIGH));
         // ------------------------------------------------ epilogue warpgroups
-        const int g = (warp - 4) >> 2;            // accumulator buffer handled by this warpgroup
+        const int e = (warp - 4) >> 2;            // epilogue warpgroup
+        const int g = C::EPI_SPLIT > 1 ? e & 1 : e;   // accumulator buffer handled by this warpgroup
+        const int qh = C::EPI_SPLIT > 1 ? e >> 1 : 0;   // which QPW queries of each item it sums
         const int quarter = warp & 3;             // TMEM lane quarter this warp may access
         const int row = quarter * 32 + lane;      // key row inside the tile
         const uint32_t t_lane = tmem + ((uint32_t)(quarter * 32) << 16);
-        float th[C::QPI];   // FILTER: the thresholds of this warpgroup's queries (h == g)
+        constexpr int QPW = C::QPW;
+        const int qw0 = qh * QPW;                 // this warpgroup's first query within an item
+        float th[QPW];      // FILTER: the thresholds of this warpgroup's queries (h == g)
 #pragma unroll
-        for (int qi = 0; qi < C::QPI; ++qi) {
-            const int q = g * C::QPI + qi;
+        for (int qi = 0; qi < QPW; ++qi) {
+            const int q = g * C::QPI + qw0 + qi;
             th[qi] = (MODE == FILTER && q < qcount) ? __ldg(sa.f_lo + (t0 + q - row_begin)) : 0.f;
         }
         for (int it = g; it < nitems; it += 2) {
@@ -277,31 +299,32 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             }
             if (misc[1] || !mbar_wait(acc_full(g), use & 1)) { misc[1] = 1; break; }
             tc_fence_after();
-            // The item's accumulator columns are read in 2 * QPI chunks of 32 (query qi, head
-            // half): the load of chunk k + 1 is in flight while chunk k is summed, and the
-            // buffer is released as soon as its last chunk has landed.
+            // This warpgroup's accumulator columns of the item are read in 2 * QPW chunks of 32
+            // (query qi, head half): the load of chunk k + 1 is in flight while chunk k is
+            // summed, and the buffer is released as soon as its last chunk has landed.
             // Sum over heads of w * ReLU(x) on packed fp32 FMAs: even heads in the low lane,
             // odd heads in the high lane (every lane rounds like a scalar fmaf).  FP8, whose
             // MMA leaves the epilogue less time, sums heads 0..31 and 32..63 in two
             // independent chains added at the end; bf16 keeps one chain in head order.
-            float res[C::QPI];
+            float res[QPW];
             uint32_t va[32], vb[32];
             uint64_t acc = 0, acc_hi = 0;
-            const uint32_t col0 = t_lane + (uint32_t)(g * C::N);
+            const uint32_t col0 = t_lane + (uint32_t)(g * C::N + qw0 * 64);
             tmem_ld32(col0, va);
             tmem_wait_ld();
             tmem_regs_ready(va);
 #pragma unroll
-            for (int k = 0; k < 2 * C::QPI; ++k) {
+            for (int k = 0; k < 2 * QPW; ++k) {
                 const int qi = k >> 1, half = k & 1;
                 uint32_t(&cur)[32] = half ? vb : va;
                 uint32_t(&nxt)[32] = half ? va : vb;
-                if (k + 1 < 2 * C::QPI) tmem_ld32(col0 + (uint32_t)((k + 1) * 32), nxt);
+                if (k + 1 < 2 * QPW) tmem_ld32(col0 + (uint32_t)((k + 1) * 32), nxt);
                 if (half == 0) {
                     acc = 0;
                     acc_hi = 0;
                 }
-                const uint64_t *wq2 = reinterpret_cast<const uint64_t *>(w_s + (h * C::QPI + qi) * 64 + half * 32);
+                const uint64_t *wq2 =
+                    reinterpret_cast<const uint64_t *>(w_s + (h * C::QPI + qw0 + qi) * 64 + half * 32);
                 uint64_t &dst = (FP8 && half) ? acc_hi : acc;
 #pragma unroll
                 for (int c = 0; c < 32; c += 2)
@@ -313,10 +336,10 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     unpack_f32x2(acc_hi, acc2, acc3);
                     res[qi] = FP8 ? (acc0 + acc1) + (acc2 + acc3) : acc0 + acc1;
                 }
-                if (k + 1 < 2 * C::QPI) {
+                if (k + 1 < 2 * QPW) {
                     tmem_wait_ld();
                     tmem_regs_ready(nxt);
-                    if (k + 2 == 2 * C::QPI) {   // the buffer's last chunk has landed
+                    if (k + 2 == 2 * QPW) {   // this warpgroup's last chunk of the buffer has landed
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive(acc_empty(g));
@@ -327,11 +350,11 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             if (MODE == FILTER) {
                 // each query is the same for the whole warp: the warp reserves its slots of
                 // the QPI rows with independent atomics (issued together), then stores
-                unsigned m[C::QPI];
-                int base[C::QPI];
+                unsigned m[QPW];
+                int base[QPW];
 #pragma unroll
-                for (int qi = 0; qi < C::QPI; ++qi) {
-                    const int q = h * C::QPI + qi;
+                for (int qi = 0; qi < QPW; ++qi) {
+                    const int q = h * C::QPI + qw0 + qi;
                     const bool valid = q < qcount && key <= pos0 + q && key < nkeys_total;
                     res[qi] = FP8 ? res[qi] * ks : res[qi];
                     m[qi] = __ballot_sync(0xffffffffu, valid && res[qi] >= th[qi]);
@@ -339,8 +362,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                     if (lane == 0 && m[qi] != 0u) base[qi] = atomicAdd(sa.cnt + (t0 + q - row_begin), __popc(m[qi]));
                 }
 #pragma unroll
-                for (int qi = 0; qi < C::QPI; ++qi) {
-                    const int t = t0 + h * C::QPI + qi;
+                for (int qi = 0; qi < QPW; ++qi) {
+                    const int t = t0 + h * C::QPI + qw0 + qi;
                     const int b = __shfl_sync(0xffffffffu, base[qi], 0);
                     const int slot = b + __popc(m[qi] & ((1u << lane) - 1u));
                     if (((m[qi] >> lane) & 1u) && slot < sa.cap)
@@ -348,8 +371,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 }
             } else {
 #pragma unroll
-                for (int qi = 0; qi < C::QPI; ++qi) {
-                    const int q = h * C::QPI + qi;
+                for (int qi = 0; qi < QPW; ++qi) {
+                    const int q = h * C::QPI + qw0 + qi;
                     if (q < qcount && key <= pos0 + q && key < nkeys_total) {
                         const int t = t0 + q;
                         const float v = FP8 ? res[qi] * ks : res[qi];
