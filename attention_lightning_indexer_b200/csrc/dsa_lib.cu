@@ -23,6 +23,8 @@ int g_debug_checks = 0;   // dsa_set_debug_checks
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
 dsa_status_t check_problem(const dsa_problem_t *p) {
     if (p == nullptr) return DSA_ERR_INVALID_ARG;
     if (p->batch < 1 || p->total_q < 0 || p->total_k < 0 || p->max_len_q < 0 || p->max_len_k < 0)
@@ -152,6 +154,9 @@ dsa_status_t set_smem_attrs() {
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(dsa::mla::sparse_mla_pair_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  dsa::mla::PairCfg::SMEM);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(dsa::mla::sparse_mla_pair_kernel<false, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, dsa::mla::PairCfg::SMEM);
     if (e == cudaSuccess) e = indexer_attr<8, false, dsa::indexer::SCORES>();
     if (e == cudaSuccess) e = indexer_attr<8, true, dsa::indexer::SCORES>();
     if (e == cudaSuccess) e = indexer_attr<8, false, dsa::indexer::SAMPLE>();
@@ -233,30 +238,79 @@ dsa_status_t topk_launch(const dsa_problem_t *p, const float *scores, int64_t ld
 
 // Sparse (gathered rows of idx) or dense (keys 0 .. pos(t), restricted to idx when idx is
 // given) attention of every query row.
+// CTA pairs the attention runs at once on one B200 (148 SMs, one CTA per SM), and the most
+// pairs one token's index row is split over.
+constexpr int MLA_PAIRS = 74;
+constexpr int MLA_MAX_SPLITS = 8;
+
+// Splits of each token's index row for the gathered attention: one pair per token when
+// the tokens alone fill the SMs (prefill, large decode batches); otherwise several pairs
+// per token, each over whole 256-slot blocks, merged by combine_splits_kernel.
+void mla_split_plan(const dsa_problem_t *p, int *nsplit, int *bps) {
+    const int T = p->total_q;
+    const int nb = (p->topk + dsa::mla::PairCfg::BLK - 1) / dsa::mla::PairCfg::BLK;   // blocks of a row
+    int sp = T > 0 ? MLA_PAIRS / T : 1;
+    sp = sp < nb ? sp : nb;
+    sp = sp < MLA_MAX_SPLITS ? sp : MLA_MAX_SPLITS;
+    if (sp < 2) {
+        *nsplit = 1;
+        *bps = 1 << 24;
+        return;
+    }
+    *bps = (nb + sp - 1) / sp;
+    *nsplit = (nb + *bps - 1) / *bps;   // no split left without blocks
+}
+
+// Bytes of the split partials (0 without splits).
+size_t mla_split_bytes(const dsa_problem_t *p) {
+    int ns, bps;
+    mla_split_plan(p, &ns, &bps);
+    if (ns < 2) return 0;
+    return align_up((size_t)p->total_q * (size_t)ns * 128 * 513 * sizeof(float), 256);
+}
+
 dsa_status_t mla_launch(const dsa_problem_t *p, const void *q, const void *kv, const int32_t *idx, void *out,
-                        float *lse, cudaStream_t stream, bool dense = false) {
+                        float *lse, cudaStream_t stream, bool dense = false, void *split_ws = nullptr) {
     if (p->total_q == 0) return DSA_OK;
     Problem P = to_dev(p);
+    dsa::mla::SplitArgs sp{1, 1 << 24, nullptr, nullptr};
+    if (!dense && split_ws != nullptr) {
+        mla_split_plan(p, &sp.nsplit, &sp.bps);
+        if (sp.nsplit > 1) {
+            sp.o_part = static_cast<float *>(split_ws);
+            sp.lse_part = sp.o_part + (size_t)p->total_q * (size_t)sp.nsplit * 128 * 512;
+        }
+    }
     CUtensorMap tq, to, tkv;
     // q: [T*128 rows, 576] read as 64-row boxes of 64 dims (each CTA of a pair loads its 64
-    // heads; the latent rows are gathered with cp.async); out: [T*128 rows, 512] written as
-    // 128 x 128 tiles
+    // heads; the latent rows are gathered by TMA, 4 rows per instruction); out: [T*128 rows,
+    // 512] written as 128 x 128 tiles
     if (!make_tmap_rows(&tq, q, false, 576, (uint64_t)p->total_q * 128, 64)) return DSA_ERR_CUDA;
     if (!make_tmap_plain_bf16(&to, out, 512, (uint64_t)p->total_q * 128, 128, 128)) return DSA_ERR_CUDA;
-    const unsigned grid = 2u * (unsigned)p->total_q;
+    const unsigned grid = 2u * (unsigned)p->total_q * (unsigned)sp.nsplit;
     const auto *kvb = reinterpret_cast<const __nv_bfloat16 *>(kv);
     auto *ob = reinterpret_cast<__nv_bfloat16 *>(out);
     if (dense) {
         // kv: [S rows, 576] read as 128-row boxes of 64 dims (contiguous keys)
         if (!make_tmap_rows(&tkv, kv, false, 576, (uint64_t)(p->total_k > 0 ? p->total_k : 1), 128)) return DSA_ERR_CUDA;
         dsa::mla::sparse_mla_pair_kernel<true><<<grid, dsa::mla::PairCfg::THREADS, dsa::mla::PairCfg::SMEM, stream>>>(
-            tq, to, tkv, P, kvb, idx, ob, lse);
+            tq, to, tkv, P, kvb, idx, ob, lse, sp);
     } else {
         // kv: [S rows, 576] gathered 4 rows x 64 dims at a time (one-row boxes)
         if (!make_tmap_rows(&tkv, kv, false, 576, (uint64_t)(p->total_k > 0 ? p->total_k : 1), 1)) return DSA_ERR_CUDA;
-        dsa::mla::sparse_mla_pair_kernel<false><<<grid, dsa::mla::PairCfg::THREADS, dsa::mla::PairCfg::SMEM, stream>>>(
-            tq, to, tkv, P, kvb, idx, ob, lse);
+        if (sp.nsplit > 1)
+            dsa::mla::sparse_mla_pair_kernel<false, true>
+                <<<grid, dsa::mla::PairCfg::THREADS, dsa::mla::PairCfg::SMEM, stream>>>(tq, to, tkv, P, kvb, idx, ob,
+                                                                                        lse, sp);
+        else
+            dsa::mla::sparse_mla_pair_kernel<false, false>
+                <<<grid, dsa::mla::PairCfg::THREADS, dsa::mla::PairCfg::SMEM, stream>>>(tq, to, tkv, P, kvb, idx, ob,
+                                                                                        lse, sp);
     }
+    dsa_status_t st = launch_status();
+    if (st != DSA_OK || sp.nsplit < 2) return st;
+    dsa::mla::combine_splits_kernel<<<(unsigned)p->total_q * 128u, 128, 0, stream>>>(sp.nsplit, sp.o_part,
+                                                                                   sp.lse_part, ob, lse);
     return launch_status();
 }
 
@@ -274,7 +328,6 @@ __global__ void bounded_wait_selftest_kernel(uint64_t limit_ns) {
     }
 }
 
-size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Key length up to which the fused forward runs the attention in the dense ("masked MHA")
 // form over the selected keys: on B200 its contiguous TMA tile loads beat the row gathers
@@ -458,7 +511,7 @@ size_t dsa_forward_workspace_size(const dsa_problem_t *p, int32_t chunk_q) {
     size_t chunk = (size_t)effective_chunk(p, chunk_q);
     size_t scores = align_up(chunk * (size_t)scores_ld(p) * sizeof(float), 256);
     size_t idx = align_up((size_t)(p->total_q > 0 ? p->total_q : 1) * (size_t)p->topk * sizeof(int32_t), 256);
-    return scores + idx;
+    return scores + idx + mla_split_bytes(p);
 }
 
 dsa_status_t dsa_forward(const dsa_problem_t *p, const void *q_idx, const void *q_scale, const void *k_idx,
@@ -501,7 +554,11 @@ dsa_status_t dsa_forward(const dsa_problem_t *p, const void *q_idx, const void *
         st = topk_launch(p, scores, ld, r0, rc, idx + (int64_t)r0 * p->topk, s);
         if (st != DSA_OK) return st;
     }
-    return mla_launch(p, q, kv, idx, out, lse, s, dense_for(p));
+    // the partials of a split attention follow the score rows and the indices
+    unsigned char *split_ws = static_cast<unsigned char *>(workspace) +
+                              align_up((size_t)chunk * (size_t)ld * sizeof(float), 256) +
+                              align_up((size_t)p->total_q * (size_t)p->topk * sizeof(int32_t), 256);
+    return mla_launch(p, q, kv, idx, out, lse, s, dense_for(p), split_ws);
 }
 
 size_t dsa_indexer_topk_streaming_workspace_size(const dsa_problem_t *p, int32_t chunk_q) {
@@ -660,7 +717,9 @@ extern "C" dsa_status_t dsa_forward_noalloc(const dsa_problem_t *p, const void *
         st = topk_launch(p, scores, ld, r0, rc, idx_out + (int64_t)r0 * p->topk, s);
         if (st != DSA_OK) return st;
     }
-    return mla_launch(p, q, kv, idx_out, out, lse, s, dense_for(p));
+    // the score rows are done: the scratch holds the partials of a split attention
+    return mla_launch(p, q, kv, idx_out, out, lse, s, dense_for(p),
+                      mla_split_bytes(p) <= NOALLOC_SCRATCH_BYTES ? static_cast<void *>(scores) : nullptr);
 }
 
 extern "C" size_t dsa_forward_noalloc_scratch_bytes(void) { return NOALLOC_SCRATCH_BYTES; }

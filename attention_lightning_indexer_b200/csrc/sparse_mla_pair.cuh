@@ -134,12 +134,25 @@ __device__ __forceinline__ float transpose_reduce32(float (&v)[32], int lane) {
     return v[0];
 }
 
-template <bool DENSE>
+// Split of each token's index row over several CTA pairs (sparse form only): pair c of a
+// token takes blocks [c * bps, (c + 1) * bps) of its 256-slot blocks and writes, instead of
+// out / lse, its normalised partial output in fp32 and the lse of its slots to
+// o_part [T * nsplit, 128, 512] / lse_part [T * nsplit, 128] (row t * nsplit + c);
+// combine_splits_kernel merges them.  The SPLIT = false instantiation (one pair per token)
+// writes out / lse directly.
+struct SplitArgs {
+    int nsplit;
+    int bps;
+    float *o_part;
+    float *lse_part;
+};
+
+template <bool DENSE, bool SPLIT = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
 sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_out,
                        const __grid_constant__ CUtensorMap tm_kv, Problem P,
                        const __nv_bfloat16 *__restrict__ kv, const int32_t *__restrict__ idx,
-                       __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
+                       __nv_bfloat16 *__restrict__ out, float *__restrict__ lse, SplitArgs sp) {
     using C = PairCfg;
     using namespace sm100;
     extern __shared__ __align__(1024) unsigned char smem[];
@@ -147,7 +160,12 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     const int cr = (int)cluster_ctarank();                   // 0: issues the MMAs
     const int peer = cr ^ 1;
     const int T = P.total_q;
-    const int t = T - 1 - (int)(blockIdx.x >> 1);           // heavier (later) tokens first
+    static_assert(!(DENSE && SPLIT), "the dense form is not split");
+    const int nsplit = SPLIT ? sp.nsplit : 1;
+    const int pair = (int)(blockIdx.x >> 1);
+    const int t = T - 1 - pair / nsplit;                    // heavier (later) tokens first
+    const int split = pair % nsplit;
+    constexpr bool partial = SPLIT;
     const int K = P.topk;
     const RowInfo ri = row_info(P, t);
     const bool rok = row_ok(P, ri);                          // same in both CTAs
@@ -257,7 +275,13 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     int last_slot = -1;
 #pragma unroll
     for (int i = 0; i < 8; ++i) last_slot = max(last_slot, reinterpret_cast<int *>(red)[i]);
-    const int nblocks = (misaligned || !rok) ? 0 : (last_slot + C::BLK) / C::BLK;   // 0 when no slot is visible
+    const int nblocks_row = (misaligned || !rok) ? 0 : (last_slot + C::BLK) / C::BLK;   // 0 when no slot is visible
+    const int bps = SPLIT ? sp.bps : nblocks_row;
+    const int b_begin = split * bps;                         // this pair's blocks of the row
+    const int nblocks = max(0, min(nblocks_row, b_begin + bps) - b_begin);
+    // this pair's part of the index row: slots from b_begin * BLK on, ks_left of them
+    const int32_t *irow_s = irow != nullptr ? irow + b_begin * C::BLK : nullptr;
+    const int ks_left = K - b_begin * C::BLK;
     __syncthreads();   // red is reused by the softmax warps
     const uint32_t peer_misc1 = mapa_shared(sbase + C::OFF_MISC + 4, (uint32_t)peer);
     auto abort_pair = [&]() {                                // stop both CTAs of the pair
@@ -308,14 +332,14 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 const int pp = p + m;
                 if (pp % C::NLOAD != lw) continue;
                 const int h = qk ? cr : ((m >> 1) & 1);
-                const int s0 = C::BLK * b + 128 * h + 4 * lane;   // this lane's 4 slots
+                const int s0 = C::BLK * b + 128 * h + 4 * lane;   // this lane's 4 slots (of the pair's part)
                 int e[4];
-                if ((K & 3) == 0 && s0 + 3 < K) {
-                    const int4 x = __ldg(reinterpret_cast<const int4 *>(irow + s0));
+                if ((K & 3) == 0 && s0 + 3 < ks_left) {
+                    const int4 x = __ldg(reinterpret_cast<const int4 *>(irow_s + s0));
                     e[0] = x.x; e[1] = x.y; e[2] = x.z; e[3] = x.w;
                 } else {
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) e[u] = s0 + u < K ? __ldg(irow + s0 + u) : -1;
+                    for (int u = 0; u < 4; ++u) e[u] = s0 + u < ks_left ? __ldg(irow_s + s0 + u) : -1;
                 }
 #pragma unroll
                 for (int u = 0; u < 4; ++u) e[u] = key_row(P, ri, pair_visible(e[u], ri) ? e[u] : 0);
@@ -427,7 +451,7 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         for (int j = 0; j < 64; ++j) l[j] = 0.f;
         bool ok = true;
         const int sown = 128 * cr + key;                     // slot of this thread's key within a block
-        int ent = !DENSE && nblocks > 0 && sown < K ? __ldg(irow + sown) : -1;
+        int ent = !DENSE && nblocks > 0 && sown < ks_left ? __ldg(irow_s + sown) : -1;
         for (int b = 0; b < nblocks; ++b) {
             bool vis;
             if (DENSE) {
@@ -436,7 +460,7 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             } else {
                 vis = pair_visible(ent, ri);
                 const int s = C::BLK * (b + 1) + sown;
-                ent = (b + 1 < nblocks && s < K) ? __ldg(irow + s) : -1;
+                ent = (b + 1 < nblocks && s < ks_left) ? __ldg(irow_s + s) : -1;
             }
             const bool fail = misc[1] != 0 || !mbar_wait_cluster(s_full(b & 1), (b >> 1) & 1);
             if (named_bar_or(1, 256, fail)) { ok = false; break; }
@@ -546,6 +570,7 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
 
         // ---- epilogue: row sums of the pair, lse, O^T / l transposed into out
         const int64_t obase = (int64_t)t * 128;
+        const int64_t pbase = ((int64_t)t * nsplit + split) * 128;   // partial rows (split mode)
         if (nblocks > 0 && ok) {
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
@@ -566,16 +591,33 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 const float l_tot = cr == 0 ? l_cta + xl[h] : xl[h] + l_cta;
                 const bool fine = okl && l_tot > 0.f;
                 fs[h] = fine ? 1.0f / l_tot : 0.f;
-                if ((h >> 6) == cr)
-                    lse[obase + h] = okl ? (l_tot > 0.f ? (mr[h] + log2f(l_tot)) * 0.6931471805599453f : -INFINITY) : NAN;
+                if ((h >> 6) == cr) {
+                    const float lv = okl ? (l_tot > 0.f ? (mr[h] + log2f(l_tot)) * 0.6931471805599453f : -INFINITY) : NAN;
+                    if (partial) sp.lse_part[pbase + h] = lv;
+                    else lse[obase + h] = lv;
+                }
             }
             const bool oko = mbar_wait_cluster(o_ready, 0);
             named_bar(1, 256);
             tc_fence_after();
             // O^T block i = h2: lanes = value dims 256 h2 + 128 cr + quarter*32 + lane, columns = heads
+            if (partial) {   // fp32 partial rows, written from registers (32 lanes: 128 bytes per head)
+                float *op = sp.o_part + pbase * 512 + 256 * h2 + 128 * cr + key;
+#pragma unroll 1
+                for (int ch = 0; ch < 4; ++ch) {
+                    uint32_t o[32];
+                    tmem_ld32(t_lane + C::TMEM_O + 128 * h2 + 32 * ch, o);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int h = 32 * ch + i;
+                        op[(int64_t)h * 512] = oko ? __uint_as_float(o[i]) * fs[h] : 0.f;
+                    }
+                }
+            }
             const uint32_t ostg = ring_s + (uint32_t)h2 * (128 * 256);
 #pragma unroll 1
-            for (int ch = 0; ch < 4; ++ch) {
+            for (int ch = 0; !partial && ch < 4; ++ch) {
                 uint32_t o[32];
                 tmem_ld32(t_lane + C::TMEM_O + 128 * h2 + 32 * ch, o);
                 tmem_wait_ld();
@@ -588,7 +630,7 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             }
             fence_proxy_async_smem();
             named_bar(1, 256);
-            if (st == 0) {
+            if (st == 0 && !partial) {
                 prefetch_tmap(&tm_out);
                 for (int i = 0; i < 2; ++i)
                     tma_store_2d(&tm_out, ring_s + (uint32_t)i * (128 * 256), 256 * i + 128 * cr, (int)obase);
@@ -600,9 +642,19 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             for (int e = st; e < 128 * 32; e += 256) {
                 const int h = e >> 5, part = e & 31;          // 32 x 16 bytes per head: the CTA's 2 x 128 dims
                 const int d0 = 256 * (part >> 4) + 128 * cr + 8 * (part & 15);
-                *reinterpret_cast<uint4 *>(out + (obase + h) * 512 + d0) = make_uint4(0, 0, 0, 0);
+                if (partial) {
+                    float4 *op = reinterpret_cast<float4 *>(sp.o_part + (pbase + h) * 512 + d0);
+                    op[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    op[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+                } else {
+                    *reinterpret_cast<uint4 *>(out + (obase + h) * 512 + d0) = make_uint4(0, 0, 0, 0);
+                }
             }
-            if (st < 128 && (st >> 6) == cr) lse[obase + st] = nblocks == 0 ? -INFINITY : NAN;
+            if (st < 128 && (st >> 6) == cr) {
+                const float lv = nblocks == 0 ? -INFINITY : NAN;
+                if (partial) sp.lse_part[pbase + st] = lv;
+                else lse[obase + st] = lv;
+            }
             if (st == 0) bulk_wait_all();
         }
     }
@@ -613,6 +665,41 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         tc_fence_after();
         tmem_dealloc_pair(tmem, 512);
     }
+}
+
+// Merges the nsplit partial results of each (token, head): lse = log sum_c exp(lse_c),
+// out = sum_c exp(lse_c - lse) o_c, rounded once to bf16.  Splits without a visible slot
+// (lse_c = -inf) weigh 0; a row without any gives out = 0, lse = -inf.  grid = T * 128
+// blocks of 128 threads (4 value dims each).
+__global__ void __launch_bounds__(128) combine_splits_kernel(int nsplit, const float *__restrict__ o_part,
+                                                            const float *__restrict__ lse_part,
+                                                            __nv_bfloat16 *__restrict__ out, float *__restrict__ lse) {
+    const int row = blockIdx.x;                              // t * 128 + h
+    const int t = row >> 7, h = row & 127;
+    float m = -INFINITY;
+    for (int c = 0; c < nsplit; ++c) m = fmaxf(m, lse_part[((int64_t)t * nsplit + c) * 128 + h]);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float wsum = 0.f;
+    if (m != -INFINITY) {
+        for (int c = 0; c < nsplit; ++c) {
+            const int64_t pr = ((int64_t)t * nsplit + c) * 128 + h;
+            const float lc = lse_part[pr];
+            const float wgt = lc == -INFINITY ? 0.f : expf(lc - m);
+            wsum += wgt;
+            const float4 v = reinterpret_cast<const float4 *>(o_part + pr * 512)[threadIdx.x];
+            acc.x = fmaf(wgt, v.x, acc.x);
+            acc.y = fmaf(wgt, v.y, acc.y);
+            acc.z = fmaf(wgt, v.z, acc.z);
+            acc.w = fmaf(wgt, v.w, acc.w);
+        }
+    }
+    const float inv = wsum > 0.f ? 1.0f / wsum : 0.f;
+    __nv_bfloat16 *o = out + (int64_t)row * 512 + 4 * threadIdx.x;
+    o[0] = __float2bfloat16_rn(acc.x * inv);
+    o[1] = __float2bfloat16_rn(acc.y * inv);
+    o[2] = __float2bfloat16_rn(acc.z * inv);
+    o[3] = __float2bfloat16_rn(acc.w * inv);
+    if (threadIdx.x == 0) lse[row] = m == -INFINITY ? -INFINITY : m + logf(wsum);
 }
 
 }  // namespace mla

@@ -383,6 +383,41 @@ def test_forward_decode_small_ragged():
     _check_forward_rows(inp, np.arange(6))
 
 
+# ------------------------------------- split attention (few tokens: several CTA pairs each)
+
+def test_forward_decode_batch_4_splits_each_row_over_8_pairs():
+    # 4 tokens, index_topk 2048: each row's 8 blocks of 256 slots go to 8 CTA pairs whose
+    # partial outputs are merged by their lse
+    inp = dsa_synth.make_decode(4, 5000, 20000, topk=2048, seed=61, device=DEV)
+    _, out, lse = _check_forward_rows(inp, np.arange(4))
+    # the unsplit kernel on the same indices agrees to rounding
+    p = dsa.problem_from_inputs(inp)
+    idx = torch.empty((4, 2048), dtype=torch.int32, device=DEV)
+    ws = torch.empty(dsa.dsa_forward_workspace_size(p, 0), dtype=torch.uint8, device=DEV)
+    o2 = torch.empty_like(out)
+    l2 = torch.empty_like(lse)
+    dsa.dsa_forward(p, inp["q_idx"], inp["k_idx"], inp["w"], inp["q"], inp["kv"], o2, l2, ws, idx_out=idx)
+    o1 = torch.empty_like(out)
+    l1 = torch.empty_like(lse)
+    dsa.dsa_sparse_mla_fwd(p, inp["q"], inp["kv"], idx, o1, l1)
+    assert torch.max(torch.abs(o1.float() - o2.float())).item() <= 2e-2
+    assert torch.max(torch.abs(l1 - l2)).item() <= 2e-3
+
+
+def test_forward_decode_split_with_empty_parts():
+    # contexts from 300 keys: a short row has fewer blocks than splits, so some of its parts
+    # hold no visible slot (lse -inf, weight 0 in the merge)
+    inp = dsa_synth.make_decode(6, 300, 9000, topk=2048, seed=62, device=DEV)
+    lens = (inp["cu_k"][1:] - inp["cu_k"][:-1]).cpu().numpy()
+    assert lens.min() < 7 * 256 and inp["max_len_k"] > 3584   # empty parts, and the gathered form
+    _check_forward_rows(inp, np.arange(6))
+
+
+def test_forward_decode_split_topk_512_three_queries_per_sequence():
+    inp = dsa_synth.make_decode(3, 4000, 12000, topk=512, seed=63, device=DEV, q_per_seq=3)
+    _check_forward_rows(inp, np.arange(9))
+
+
 # ------------------------------------------- full-size workloads, sampled rows
 
 def test_prefill_4k_full_size_sampled():
