@@ -337,6 +337,29 @@ def _decode_secondary(dsa, args, rank, dev, stream, flush, dist):
     res["us_per_step_paged_cache"] = _max_over_ranks(dist, sum(s.elapsed_time(e) for s, e in zip(starts, ends))) / n * 1e3
     dsa.dsa_check_device_errors()
     del pg
+    # a small batch (8 sequences, the same context range): too few tokens to fill the SMs,
+    # so the attention splits each index row over several CTA pairs and merges by lse
+    sb = dsa_synth.make_decode(8, 8192, 65536, topk=inp["topk"], seed=args.seed + 11, device=dev)
+    ps = dsa.problem_from_inputs(sb)
+    out_s = torch.empty((sb["total_q"], 128, 512), dtype=torch.bfloat16, device=dev)
+    lse_s = torch.empty((sb["total_q"], 128), dtype=torch.float32, device=dev)
+    ws_s = torch.empty(dsa.dsa_forward_workspace_size(ps, 0), dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        dsa.dsa_forward(ps, sb["q_idx"], sb["k_idx"], sb["w"], sb["q"], sb["kv"], out_s, lse_s, ws_s, stream=stream)
+    torch.cuda.synchronize(dev)
+    _barrier(dist)
+    for i in range(n):
+        flush.zero_()
+        starts[i].record(stream)
+        dsa.dsa_forward(ps, sb["q_idx"], sb["k_idx"], sb["w"], sb["q"], sb["kv"], out_s, lse_s, ws_s, stream=stream)
+        ends[i].record(stream)
+    torch.cuda.synchronize(dev)
+    _barrier(dist)
+    res["small_batch"] = {"batch": 8, "mean_context": float(sb["total_k"]) / 8, "gpu_launches_per_step": 4,
+                          "us_per_step": _max_over_ranks(dist, sum(s.elapsed_time(e) for s, e in zip(starts, ends)))
+                          / n * 1e3}
+    dsa.dsa_check_device_errors()
+    del sb, ws_s
     if rank == 0 and not args.no_breakdown:
         res["roofline"], res["kernels"] = _breakdown(dsa, p, inp, fa, 0, dev, stream, flush, decode=True)
     return res
