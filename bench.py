@@ -47,7 +47,7 @@ TRAFFIC = {
     # 499 MB written: q reads and out writes, both proportional to the query count; kv rows
     # come from L2), scaled x8 to the 32768-query launch of the 32K step (that prefill only:
     # at 128K the kv rows no longer fit in L2)
-    "sparse_mla": {"bytes_per_launch": 1.142312e9 * 8, "total_q": 32768, "src_sha": "fa50549e97859dac"},
+    "sparse_mla": {"bytes_per_launch": 1.141754e9 * 8, "total_q": 32768, "src_sha": "d9a63f4278d4b7f9"},
 }
 
 
