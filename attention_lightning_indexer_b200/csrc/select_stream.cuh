@@ -108,7 +108,7 @@ select_candidates_kernel(Problem P, const int *__restrict__ cnt, const uint2 *__
                          int row_begin, int32_t *__restrict__ idx, uint8_t *__restrict__ flag) {
     using C = StreamCfg;
     extern __shared__ __align__(16) unsigned char smem[];
-    const int r = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
+    const int r = blockIdx.x, tid = threadIdx.x;
     const int K = P.topk;
     int32_t *out = idx + (int64_t)r * K;
     const RowInfo ri = row_info(P, row_begin + r);
@@ -185,7 +185,6 @@ select_candidates_kernel(Problem P, const int *__restrict__ cnt, const uint2 *__
     __syncthreads();
     ordered_bits(gt, nw, out, wtot);
     ordered_bits(eq, nw, out + above, wtot);
-    (void)lane;
 }
 
 }  // namespace topk

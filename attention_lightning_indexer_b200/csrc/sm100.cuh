@@ -196,17 +196,6 @@ __device__ __forceinline__ void tmem_regs_ready(uint32_t (&r)[32]) {
 namespace dsa {
 namespace sm100 {
 
-// D[tmem] (+)= A[tmem] * B[smem desc]^T, kind::f16 (A read from tensor memory).
-__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                           uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
 // Instruction descriptor with B in MN-major order (bit 16), bf16 inputs, fp32 accumulator.
 __host__ __device__ constexpr uint32_t idesc_bf16_bmn(int M, int N) { return idesc_bf16(M, N) | (1u << 16); }
 
@@ -275,25 +264,11 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 namespace dsa {
 namespace sm100 {
 
-// 16-byte global -> shared copy through L2 only (LDGSTS), asynchronous.
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 // Orders shared-memory data written through the generic proxy (cp.async copies whose
 // completion this thread has observed on an mbarrier) before this thread's following
 // async-proxy operations (tensor-core operand reads).
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-// Arrives on the mbarrier once all of this thread's earlier cp.async copies have landed
-// (without raising the expected count: the barrier is initialised with one arrival per
-// signalling thread).
-__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 
 // Packed fp32 pairs (sm_100): two independent round-to-nearest fp32 FMAs in one instruction,
@@ -376,19 +351,7 @@ __device__ __forceinline__ void st_async_f32(uint32_t cluster_addr, float v, uin
                  : "memory");
 }
 
-// Bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned) from this CTA's
-// shared memory into a peer CTA's, completing the bytes on the peer's mbarrier.
-__device__ __forceinline__ void bulk_copy_s2peer(uint32_t dst_cluster, uint32_t src_cta, uint32_t bytes,
-                                                 uint32_t bar_cluster) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            dst_cluster),
-        "r"(src_cta), "r"(bytes), "r"(bar_cluster)
-        : "memory");
-}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// Waits until every committed bulk copy of this thread has finished reading its source.
-__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 // Waits until every committed bulk operation of this thread has completed.
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
@@ -399,10 +362,6 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, uint32_t sr
                  "r"(src), "r"(x), "r"(y)
                  : "memory");
 }
-
-// Generic-proxy writes (st.shared, cp.async) ordered before async-proxy accesses
-// (tensor-core operand reads, bulk copies) of shared memory.
-__device__ __forceinline__ void fence_proxy_async_all() { asm volatile("fence.proxy.async;" ::: "memory"); }
 
 // TMEM allocation for CTA pairs: one warp with the same warp index in both CTAs.
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
@@ -441,16 +400,6 @@ __device__ __forceinline__ void mma_commit_pair_both(uint32_t bar) {
 // Instruction descriptor, bf16 inputs, fp32 accumulator, A and B both MN-major.
 __host__ __device__ constexpr uint32_t idesc_bf16_mn_mn(int M, int N) {
     return idesc_bf16(M, N) | (1u << 15) | (1u << 16);
-}
-
-// 32 lanes x 32 bits, 16 consecutive columns.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
 }
 
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {

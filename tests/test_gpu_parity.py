@@ -78,7 +78,7 @@ def test_topk_adversarial_rows_take_every_path(pattern, rows):
     # Rows built so that the sampled fast path is exact (spike), or must give up (all
     # keys equal; all top keys clustered in one warp's range; two values) and the general
     # path decides.  Either way the result must equal the oracle's.  8 rows run with
-    # 512 threads per row (fewer rows than SMs), 200 rows with 256.
+    # 1024 threads per row (fewer rows than SMs), 200 rows with 256.
     L, k = 6000, 2048
     base = torch.arange(L, dtype=torch.float32)
     if pattern == "constant":
