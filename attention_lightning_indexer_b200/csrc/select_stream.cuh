@@ -23,7 +23,7 @@ namespace dsa {
 namespace topk {
 
 constexpr int STREAM_NT = 256;
-using StreamCfg = Cfg<STREAM_NT>;
+using StreamCfg = Cfg<STREAM_NT, 7168>;   // room for ~1.4 k candidates and long rows' samples
 constexpr int STREAM_CAP = StreamCfg::WARPS * StreamCfg::SEG;          // candidates a row may hold
 constexpr int STREAM_MAX_SAMPLES = 2 * StreamCfg::WARPS * StreamCfg::SEG;
 

@@ -6,7 +6,7 @@
 //
 // Scores map to order-preserving 32-bit keys (-0.0 folded onto +0.0), so comparing keys
 // as unsigned integers compares the floats as values.  One CTA per row: 256 threads when
-// there are many rows (several CTAs share an SM), 1024 when a launch has fewer rows than
+// there are many rows (four CTAs share an SM), 1024 when a launch has fewer rows than
 // SMs (decode), so a long row is not left to 8 warps.
 //
 // Fast path (one HBM read of the row):
@@ -39,11 +39,13 @@ constexpr int BINS = 2048;        // 11-bit digits
 constexpr int GROUPS = 32;        // group sums per histogram (one per lane of the bin search)
 constexpr unsigned FULL = 0xffffffffu;
 
-template <int NT>
+// NT threads; CAP candidate slots in all (about 1.2 k = 2.5 K are expected per row).  The
+// 256-thread shape keeps 4096, so that four CTAs share an SM (49.5 KB of shared memory each).
+template <int NT, int CAP = (NT >= 512 ? 7168 : 4096)>
 struct Cfg {
     static constexpr int THREADS = NT;
     static constexpr int WARPS = NT / 32;
-    static constexpr int SEG = 7168 / WARPS;                  // candidate slots per warp (fast path)
+    static constexpr int SEG = CAP / WARPS;                   // candidate slots per warp (fast path)
     static constexpr int CAND_CAP = WARPS * SEG * 2;          // general-path candidate indices (same bytes)
     // Dynamic shared memory layout.
     static constexpr int OFF_HIST = 0;                             // [2][BINS] u32
@@ -56,7 +58,7 @@ struct Cfg {
     // [3] overflow flag, then three per-warp arrays A = scal + 8, B = A + WARPS, C = B + WARPS
     static constexpr int NSCAL = 8 + 3 * WARPS;
     static constexpr int SMEM = OFF_SCAL + NSCAL * 4;
-    static_assert(7168 % WARPS == 0 && NT % 32 == 0, "whole warps, equal segments");
+    static_assert(CAP % WARPS == 0 && NT % 32 == 0, "whole warps, equal segments");
     static_assert(CAND_CAP * 4 == 2 * WARPS * SEG * 4, "general-path candidates reuse both segment arrays");
 };
 
@@ -573,7 +575,7 @@ __device__ void select_row_general(const float *src, int n, int K, unsigned char
 // grid = row_count CTAs of NT threads, dynamic shared memory Cfg<NT>::SMEM bytes.  With a
 // row_mask only the rows r with row_mask[r] != 0 are selected (the others are untouched).
 template <int NT>
-__global__ void __launch_bounds__(NT, NT >= 512 ? 1 : 3) topk_rows_kernel(Problem P, const float *__restrict__ scores, int64_t ld,
+__global__ void __launch_bounds__(NT, NT >= 512 ? 1 : 4) topk_rows_kernel(Problem P, const float *__restrict__ scores, int64_t ld,
                                                        int row_begin, int32_t *__restrict__ idx,
                                                        const uint8_t *__restrict__ row_mask) {
     using C = Cfg<NT>;
