@@ -8,8 +8,9 @@
 //   k_I[row]      = RoPE_half(LayerNorm(k_raw) * ln_w + ln_b)   pairs (i, i + 32), i < 32
 //   kv[row, :512] = k_raw_latent[:512] / rms * rms_w
 //   kv[row, 512:] = RoPE_interleaved(latent[512:])             pairs (512 + 2i, 513 + 2i)
-// with the angle pos * inv_freq[i] of pair i, evaluated in fp64 (positions reach 163,840).
-// One warp per token: HBM-bound (1.4 KB read, 1.4 KB written per token).
+// with the angle pos * inv_freq[i] of pair i, evaluated in fp64 (positions reach 163,840)
+// once per token and pair (lane i) and shared by both RoPEs through warp shuffles.
+// One warp per token: 1.4 KB read and 1.4 KB written per token.
 #pragma once
 
 #include "dsa_common.cuh"
@@ -43,6 +44,10 @@ cache_write_kernel(int n, const __nv_bfloat16 *__restrict__ k_raw, const __nv_bf
     if (t >= n) return;                                       // whole warp
     const int p = __ldg(pos + t);
     const int64_t row = __ldg(rows + t);
+    // the 32 rotation angles of this position, pair i by lane i (both RoPEs use the same
+    // frequencies); lanes read the ones they need by shuffles
+    float c_lane, s_lane;
+    rot_cs(p, __ldg(inv_freq + lane), c_lane, s_lane);
 
     // ---- indexer key: lane l holds dims 4l .. 4l+3
     float x[4];
@@ -63,18 +68,17 @@ cache_write_kernel(int n, const __nv_bfloat16 *__restrict__ k_raw, const __nv_bf
         x[j] = (x[j] - mean) * inv * __ldg(ln_w + d) + __ldg(ln_b + d);
     }
     // RoPE, non-interleaved: dims i (lanes 0-7) pair with i + 32 (lanes 8-15)
-    float partner[4];
+    float partner[4], ck[4], sk[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) partner[j] = __shfl_xor_sync(0xffffffffu, x[j], 8);
+    for (int j = 0; j < 4; ++j) {
+        partner[j] = __shfl_xor_sync(0xffffffffu, x[j], 8);
+        ck[j] = __shfl_sync(0xffffffffu, c_lane, 4 * (lane & 7) + j);   // pair i = 4 (lane & 7) + j
+        sk[j] = __shfl_sync(0xffffffffu, s_lane, 4 * (lane & 7) + j);
+    }
     if (lane < 16) {
         const bool lower = lane < 8;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int i = 4 * (lane & 7) + j;
-            float c, s;
-            rot_cs(p, __ldg(inv_freq + i), c, s);
-            x[j] = lower ? x[j] * c - partner[j] * s : x[j] * c + partner[j] * s;
-        }
+        for (int j = 0; j < 4; ++j) x[j] = lower ? x[j] * ck[j] - partner[j] * sk[j] : x[j] * ck[j] + partner[j] * sk[j];
     }
     {
         uint2 o;
@@ -116,6 +120,12 @@ cache_write_kernel(int n, const __nv_bfloat16 *__restrict__ k_raw, const __nv_bf
         }
         dst[lane + 32 * c2] = make_uint4(o4[0], o4[1], o4[2], o4[3]);
     }
+    float cl[4], sl[4];   // lanes 0-7: pairs i = 4 lane .. 4 lane + 3 of the latent's RoPE dims
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        cl[j] = __shfl_sync(0xffffffffu, c_lane, (4 * lane + j) & 31);
+        sl[j] = __shfl_sync(0xffffffffu, s_lane, (4 * lane + j) & 31);
+    }
     if (lane < 8) {   // RoPE, interleaved: pairs (512 + 2i, 513 + 2i), i = 4 lane .. 4 lane + 3
         const uint4 v = __ldg(src + 64 + lane);
         const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
@@ -124,9 +134,7 @@ cache_write_kernel(int n, const __nv_bfloat16 *__restrict__ k_raw, const __nv_bf
         for (int j = 0; j < 4; ++j) {
             const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162 *>(&w4[j]);
             const float u = __low2float(h), w = __high2float(h);
-            float c, s;
-            rot_cs(p, __ldg(inv_freq + 4 * lane + j), c, s);
-            __nv_bfloat162 r = __floats2bfloat162_rn(u * c - w * s, w * c + u * s);
+            __nv_bfloat162 r = __floats2bfloat162_rn(u * cl[j] - w * sl[j], w * cl[j] + u * sl[j]);
             o4[j] = *reinterpret_cast<uint32_t *>(&r);
         }
         dst[64 + lane] = make_uint4(o4[0], o4[1], o4[2], o4[3]);
