@@ -608,6 +608,12 @@ def test_forward_paged_decode_small():
     _forward_paged_vs_packed(inp, seed=54, rows=np.arange(6))
 
 
+def test_forward_paged_decode_batch_4_split_attention():
+    # 4 tokens: the attention splits each row over 8 CTA pairs and gathers through the table
+    inp = dsa_synth.make_decode(4, 5000, 20000, topk=2048, seed=56, device=DEV)
+    _forward_paged_vs_packed(inp, seed=57, rows=np.arange(4))
+
+
 def test_forward_paged_decode_b64_full_size():
     inp = dsa_synth.make_workload("decode_b64", seed=0, device=DEV)
     _forward_paged_vs_packed(inp, seed=55, rows=np.array([0, 17, 40, 63]))
