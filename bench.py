@@ -283,6 +283,16 @@ def run_ours(args, ws, rank, local, dist):
         print(json.dumps(res), flush=True)
 
 
+def _capture(step, dev):
+    """One call of step() captured as a CUDA graph (on a side stream, as capture needs)."""
+    torch.cuda.synchronize(dev)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step(torch.cuda.current_stream(dev))
+    torch.cuda.synchronize(dev)
+    return graph
+
+
 def _decode_secondary(dsa, args, rank, dev, stream, flush, dist):
     """The metric's second half: decode microseconds per step (64 sequences, one query
     each, contexts ~U[8192, 65536]), timed like the main step (events, L2 flushed between
@@ -295,9 +305,9 @@ def _decode_secondary(dsa, args, rank, dev, stream, flush, dist):
     lse = torch.empty((T, 128), dtype=torch.float32, device=dev)
     wsb = torch.empty(dsa.dsa_forward_workspace_size(p, 0), dtype=torch.uint8, device=dev)
 
-    def step():
+    def step(st=stream):
         dsa.dsa_forward(p, fa["q_idx"], fa["k_idx"], inp["w"], inp["q"], inp["kv"], out, lse, wsb, chunk_q=0,
-                        stream=stream)
+                        stream=st)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -305,38 +315,40 @@ def _decode_secondary(dsa, args, rank, dev, stream, flush, dist):
     n = max(args.steps, 10)
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
-    _barrier(dist)
-    for i in range(n):
-        flush.zero_()
-        starts[i].record(stream)
-        step()
-        ends[i].record(stream)
-    torch.cuda.synchronize(dev)
-    _barrier(dist)
-    total_ms = _max_over_ranks(dist, sum(s.elapsed_time(e) for s, e in zip(starts, ends)))
+
+    def timed(run):
+        _barrier(dist)
+        for i in range(n):
+            flush.zero_()
+            starts[i].record(stream)
+            run()
+            ends[i].record(stream)
+        torch.cuda.synchronize(dev)
+        _barrier(dist)
+        return _max_over_ranks(dist, sum(s.elapsed_time(e) for s, e in zip(starts, ends))) / n * 1e3
+
+    # A serving loop captures its decode step once and replays it: the step as a CUDA graph
+    # of its kernel launches, replayed on the bench stream (the eager time is reported too).
+    graph = _capture(step, dev)
+    us_graph = timed(graph.replay)
+    us_eager = timed(step)
     dsa.dsa_check_device_errors()
-    res = {"workload": "decode_b64", "us_per_step": total_ms / n * 1e3, "steps": n, "batch": inp["batch"],
-           "mean_context": float(inp["total_k"]) / inp["batch"], "gpu_launches_per_step": 3,
-           "higher_is_better": False}
+    res = {"workload": "decode_b64", "us_per_step": us_graph, "cuda_graph": True, "us_per_step_eager": us_eager,
+           "steps": n, "batch": inp["batch"], "mean_context": float(inp["total_k"]) / inp["batch"],
+           "gpu_launches_per_step": 3, "higher_is_better": False}
+    del graph
     # the same step with the key caches in shuffled 64-token pages (block table)
     pg = dsa_synth.to_paged(inp, page_size=64, seed=args.seed + 7)
     pp = dsa.problem_from_inputs(pg)
+    def step_paged(st=stream):
+        dsa.dsa_forward(pp, pg["q_idx"], pg["k_idx"], pg["w"], pg["q"], pg["kv"], out, lse, wsb, chunk_q=0, stream=st)
+
     for _ in range(3):
-        dsa.dsa_forward(pp, pg["q_idx"], pg["k_idx"], pg["w"], pg["q"], pg["kv"], out, lse, wsb, chunk_q=0,
-                        stream=stream)
-    torch.cuda.synchronize(dev)
-    _barrier(dist)
-    for i in range(n):
-        flush.zero_()
-        starts[i].record(stream)
-        dsa.dsa_forward(pp, pg["q_idx"], pg["k_idx"], pg["w"], pg["q"], pg["kv"], out, lse, wsb, chunk_q=0,
-                        stream=stream)
-        ends[i].record(stream)
-    torch.cuda.synchronize(dev)
-    _barrier(dist)
-    res["us_per_step_paged_cache"] = _max_over_ranks(dist, sum(s.elapsed_time(e) for s, e in zip(starts, ends))) / n * 1e3
+        step_paged()
+    graph = _capture(step_paged, dev)
+    res["us_per_step_paged_cache"] = timed(graph.replay)
     dsa.dsa_check_device_errors()
-    del pg
+    del graph, pg
     # a small batch (8 sequences, the same context range): too few tokens to fill the SMs,
     # so the attention splits each index row over several CTA pairs and merges by lse
     sb = dsa_synth.make_decode(8, 8192, 65536, topk=inp["topk"], seed=args.seed + 11, device=dev)
@@ -344,22 +356,16 @@ def _decode_secondary(dsa, args, rank, dev, stream, flush, dist):
     out_s = torch.empty((sb["total_q"], 128, 512), dtype=torch.bfloat16, device=dev)
     lse_s = torch.empty((sb["total_q"], 128), dtype=torch.float32, device=dev)
     ws_s = torch.empty(dsa.dsa_forward_workspace_size(ps, 0), dtype=torch.uint8, device=dev)
+    def step_small(st=stream):
+        dsa.dsa_forward(ps, sb["q_idx"], sb["k_idx"], sb["w"], sb["q"], sb["kv"], out_s, lse_s, ws_s, stream=st)
+
     for _ in range(3):
-        dsa.dsa_forward(ps, sb["q_idx"], sb["k_idx"], sb["w"], sb["q"], sb["kv"], out_s, lse_s, ws_s, stream=stream)
-    torch.cuda.synchronize(dev)
-    _barrier(dist)
-    for i in range(n):
-        flush.zero_()
-        starts[i].record(stream)
-        dsa.dsa_forward(ps, sb["q_idx"], sb["k_idx"], sb["w"], sb["q"], sb["kv"], out_s, lse_s, ws_s, stream=stream)
-        ends[i].record(stream)
-    torch.cuda.synchronize(dev)
-    _barrier(dist)
+        step_small()
+    graph = _capture(step_small, dev)
     res["small_batch"] = {"batch": 8, "mean_context": float(sb["total_k"]) / 8, "gpu_launches_per_step": 4,
-                          "us_per_step": _max_over_ranks(dist, sum(s.elapsed_time(e) for s, e in zip(starts, ends)))
-                          / n * 1e3}
+                          "cuda_graph": True, "us_per_step": timed(graph.replay)}
     dsa.dsa_check_device_errors()
-    del sb, ws_s
+    del graph, sb, ws_s
     if rank == 0 and not args.no_breakdown:
         res["roofline"], res["kernels"] = _breakdown(dsa, p, inp, fa, 0, dev, stream, flush, decode=True)
     return res
