@@ -338,6 +338,36 @@ constexpr int DENSE_KV_THRESHOLD = 3584;
 
 bool dense_for(const dsa_problem_t *p) { return p->block_table == nullptr && p->max_len_k <= DENSE_KV_THRESHOLD; }
 
+// The attention of the fused forward over its selected indices.  In one packed sequence the
+// first rows see at most topk keys, so their selection is every visible key in order: the
+// dense form over all causal keys computes them (the same MMAs on the same operands, so the
+// same output) without gathering, and the gathered form takes the remaining rows.
+dsa_status_t forward_attention(const dsa_problem_t *p, const void *q, const void *kv, const int32_t *idx, void *out,
+                               float *lse, cudaStream_t s, void *split_ws) {
+    if (dense_for(p)) return mla_launch(p, q, kv, idx, out, lse, s, true);
+    const int T = p->total_q;
+    int R = 0;   // rows with pos(t) + 1 <= topk
+    if (p->cu_q == nullptr && p->block_table == nullptr) {
+        const int64_t r = (int64_t)p->topk - ((int64_t)p->total_k - T);
+        R = r < 0 ? 0 : (r > T ? T : (int)r);
+    }
+    if (R == 0 || R == T) return mla_launch(p, q, kv, idx, out, lse, s, false, split_ws);
+    dsa_problem_t a = *p;   // rows 0 .. R-1 and the keys they see
+    a.total_q = R;
+    a.max_len_q = R;
+    a.total_k = p->total_k - T + R;
+    a.max_len_k = a.total_k;
+    dsa_status_t st = mla_launch(&a, q, kv, nullptr, out, lse, s, true);
+    if (st != DSA_OK) return st;
+    dsa_problem_t b = *p;   // rows R .. T-1 (the same keys: pos = total_k - (T - R) + local row)
+    b.total_q = T - R;
+    b.max_len_q = T - R;
+    const size_t qrow = 128u * 576u * 2u, orow = 128u * 512u * 2u;
+    return mla_launch(&b, static_cast<const unsigned char *>(q) + (size_t)R * qrow, kv, idx + (int64_t)R * p->topk,
+                      static_cast<unsigned char *>(out) + (size_t)R * orow, lse + (int64_t)R * 128, s, false,
+                      split_ws);
+}
+
 int64_t scores_ld(const dsa_problem_t *p) { return (int64_t)align_up((size_t)(p->max_len_k > 0 ? p->max_len_k : 1), 4); }
 
 int effective_chunk(const dsa_problem_t *p, int32_t chunk_q) {
@@ -558,7 +588,7 @@ dsa_status_t dsa_forward(const dsa_problem_t *p, const void *q_idx, const void *
     unsigned char *split_ws = static_cast<unsigned char *>(workspace) +
                               align_up((size_t)chunk * (size_t)ld * sizeof(float), 256) +
                               align_up((size_t)p->total_q * (size_t)p->topk * sizeof(int32_t), 256);
-    return mla_launch(p, q, kv, idx, out, lse, s, dense_for(p), split_ws);
+    return forward_attention(p, q, kv, idx, out, lse, s, split_ws);
 }
 
 size_t dsa_indexer_topk_streaming_workspace_size(const dsa_problem_t *p, int32_t chunk_q) {
@@ -718,8 +748,8 @@ extern "C" dsa_status_t dsa_forward_noalloc(const dsa_problem_t *p, const void *
         if (st != DSA_OK) return st;
     }
     // the score rows are done: the scratch holds the partials of a split attention
-    return mla_launch(p, q, kv, idx_out, out, lse, s, dense_for(p),
-                      mla_split_bytes(p) <= NOALLOC_SCRATCH_BYTES ? static_cast<void *>(scores) : nullptr);
+    return forward_attention(p, q, kv, idx_out, out, lse, s,
+                             mla_split_bytes(p) <= NOALLOC_SCRATCH_BYTES ? static_cast<void *>(scores) : nullptr);
 }
 
 extern "C" size_t dsa_forward_noalloc_scratch_bytes(void) { return NOALLOC_SCRATCH_BYTES; }

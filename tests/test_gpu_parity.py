@@ -426,6 +426,21 @@ def test_prefill_4k_full_size_sampled():
     _check_forward_rows(inp, rows, chunk=4096)
 
 
+def test_forward_first_rows_take_the_dense_form_bit_identically():
+    # one 5000-token sequence, index_topk 2048: rows 0..2047 see at most 2048 keys and
+    # select all of them, so dsa_forward runs them in the dense form and the rest gathered;
+    # the output equals the gathered form over the same indices bit for bit
+    L, k = 5000, 2048
+    inp = dsa_synth.make_prefill(L, topk=k, seed=34, device=DEV)
+    idx, out, lse = _run_forward(inp)
+    p = dsa.problem_from_inputs(inp)
+    out2 = torch.empty_like(out)
+    lse2 = torch.empty_like(lse)
+    dsa.dsa_sparse_mla_fwd(p, inp["q"], inp["kv"], idx, out2, lse2)
+    assert torch.equal(out, out2) and torch.equal(lse, lse2)
+    _check_forward_rows(inp, np.array([0, 1, 1000, 2046, 2047, 2048, 2049, 4999]))
+
+
 def test_prefill_3k_forward_takes_the_masked_dense_form():
     # topk < max_len_k <= the short-sequence threshold: dsa_forward runs the indexer and the
     # top-k, then the dense form restricted to the selected keys (its key blocks group the
