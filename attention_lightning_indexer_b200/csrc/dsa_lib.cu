@@ -269,6 +269,28 @@ size_t mla_split_bytes(const dsa_problem_t *p) {
     return align_up((size_t)p->total_q * (size_t)ns * 128 * 513 * sizeof(float), 256);
 }
 
+// CTA pairs of one attention instantiation that run at once on the current device (one
+// CTA per SM; asked of the occupancy calculator once per device, after the shared-memory
+// attribute is set).
+template <bool DENSE, bool SPLIT>
+int mla_resident_pairs() {
+    static int pairs[MAX_DEVICES] = {};
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return 0;
+    if (pairs[dev] > 0) return pairs[dev];
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(dsa::mla::PairCfg::THREADS, 1, 1);
+    cfg.dynamicSmemBytes = dsa::mla::PairCfg::SMEM;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, dsa::mla::sparse_mla_pair_kernel<DENSE, SPLIT>, &cfg) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return 0;
+    }
+    pairs[dev] = n;
+    return n;
+}
+
 dsa_status_t mla_launch(const dsa_problem_t *p, const void *q, const void *kv, const int32_t *idx, void *out,
                         float *lse, cudaStream_t stream, bool dense = false, void *split_ws = nullptr) {
     if (p->total_q == 0) return DSA_OK;
@@ -281,31 +303,31 @@ dsa_status_t mla_launch(const dsa_problem_t *p, const void *q, const void *kv, c
             sp.lse_part = sp.o_part + (size_t)p->total_q * (size_t)sp.nsplit * 128 * 512;
         }
     }
-    CUtensorMap tq, to, tkv;
+    CUtensorMap tq, tkv;
     // q: [T*128 rows, 576] read as 64-row boxes of 64 dims (each CTA of a pair loads its 64
-    // heads; the latent rows are gathered by TMA, 4 rows per instruction); out: [T*128 rows,
-    // 512] written as 128 x 128 tiles
+    // heads; the latent rows are gathered by TMA, 4 rows per instruction)
     if (!make_tmap_rows(&tq, q, false, 576, (uint64_t)p->total_q * 128, 64)) return DSA_ERR_CUDA;
-    if (!make_tmap_plain_bf16(&to, out, 512, (uint64_t)p->total_q * 128, 128, 128)) return DSA_ERR_CUDA;
-    const unsigned grid = 2u * (unsigned)p->total_q * (unsigned)sp.nsplit;
-    const auto *kvb = reinterpret_cast<const __nv_bfloat16 *>(kv);
+    // persistent pairs: no more than run at once, each taking units (token, split) in turn
+    const long long units = (long long)p->total_q * sp.nsplit;
+    const int resident = dense ? mla_resident_pairs<true, false>()
+                               : (sp.nsplit > 1 ? mla_resident_pairs<false, true>() : mla_resident_pairs<false, false>());
+    if (resident <= 0) return DSA_ERR_CUDA;
+    const unsigned grid = 2u * (unsigned)(units < resident ? units : resident);
     auto *ob = reinterpret_cast<__nv_bfloat16 *>(out);
     if (dense) {
         // kv: [S rows, 576] read as 128-row boxes of 64 dims (contiguous keys)
         if (!make_tmap_rows(&tkv, kv, false, 576, (uint64_t)(p->total_k > 0 ? p->total_k : 1), 128)) return DSA_ERR_CUDA;
         dsa::mla::sparse_mla_pair_kernel<true><<<grid, dsa::mla::PairCfg::THREADS, dsa::mla::PairCfg::SMEM, stream>>>(
-            tq, to, tkv, P, kvb, idx, ob, lse, sp);
+            tq, tkv, P, idx, ob, lse, sp);
     } else {
         // kv: [S rows, 576] gathered 4 rows x 64 dims at a time (one-row boxes)
         if (!make_tmap_rows(&tkv, kv, false, 576, (uint64_t)(p->total_k > 0 ? p->total_k : 1), 1)) return DSA_ERR_CUDA;
         if (sp.nsplit > 1)
             dsa::mla::sparse_mla_pair_kernel<false, true>
-                <<<grid, dsa::mla::PairCfg::THREADS, dsa::mla::PairCfg::SMEM, stream>>>(tq, to, tkv, P, kvb, idx, ob,
-                                                                                        lse, sp);
+                <<<grid, dsa::mla::PairCfg::THREADS, dsa::mla::PairCfg::SMEM, stream>>>(tq, tkv, P, idx, ob, lse, sp);
         else
             dsa::mla::sparse_mla_pair_kernel<false, false>
-                <<<grid, dsa::mla::PairCfg::THREADS, dsa::mla::PairCfg::SMEM, stream>>>(tq, to, tkv, P, kvb, idx, ob,
-                                                                                        lse, sp);
+                <<<grid, dsa::mla::PairCfg::THREADS, dsa::mla::PairCfg::SMEM, stream>>>(tq, tkv, P, idx, ob, lse, sp);
     }
     dsa_status_t st = launch_status();
     if (st != DSA_OK || sp.nsplit < 2) return st;

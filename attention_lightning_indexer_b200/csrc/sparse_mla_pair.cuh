@@ -80,10 +80,10 @@ struct PairCfg {
     static constexpr int OFF_MASK = OFF_FS + 128 * 4;          // dense mode: listed-key bitmask
     static constexpr int DENSE_MAX_KEYS = 16384;               // keys a masked dense row may have
     static constexpr int OFF_BAR = OFF_MASK + DENSE_MAX_KEYS / 8;
-    // (unused)[7] empty[7] pfull[7] q_full q_peer s_full[2] s_free[2] p_full (unused)
-    // pv_done o_ready xbar[2] lbar drain
-    static constexpr int NBARS = 3 * NSLOT + 2 + 2 + 2 + 2 + 2 + 2 + 1 + 1;
-    static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
+    // empty[7] pfull[7] q_full q_free s_full[2] s_free[2] p_full pv_done o_ready xbar[2]
+    // lbar drain unit_full[2] unit_free[2]
+    static constexpr int NBARS = 2 * NSLOT + 2 + 2 + 2 + 3 + 2 + 2 + 2 + 2;
+    static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;   // [0] TMEM base, [1] abort, [2..3] unit blocks
     static constexpr int SMEM = OFF_MISC + 16;
     static constexpr int THREADS = 512;
     static constexpr int SOFT0 = 8;                 // first softmax warp
@@ -93,7 +93,6 @@ struct PairCfg {
     static_assert(SMEM <= 232448, "shared memory budget");
     static_assert(NLOAD <= NSLOT, "ring waits need NLOAD <= NSLOT");
     static_assert(256 * REG_LOW + 256 * REG_HIGH <= 65536 / THREADS * THREADS, "register split");
-    static_assert(2 * 128 * 128 * 2 <= NSLOT * ATOM, "output staging fits in the ring");
 };
 
 __device__ __forceinline__ bool pair_visible(int e, const RowInfo &ri) { return e >= 0 && e <= ri.pos && e < ri.len_k; }
@@ -134,11 +133,11 @@ __device__ __forceinline__ float transpose_reduce32(float (&v)[32], int lane) {
     return v[0];
 }
 
-// Split of each token's index row over several CTA pairs (sparse form only): pair c of a
+// Split of each token's index row over several CTA pairs (sparse form only): split c of a
 // token takes blocks [c * bps, (c + 1) * bps) of its 256-slot blocks and writes, instead of
 // out / lse, its normalised partial output in fp32 and the lse of its slots to
 // o_part [T * nsplit, 128, 512] / lse_part [T * nsplit, 128] (row t * nsplit + c);
-// combine_splits_kernel merges them.  The SPLIT = false instantiation (one pair per token)
+// combine_splits_kernel merges them.  The SPLIT = false instantiation (one unit per token)
 // writes out / lse directly.
 struct SplitArgs {
     int nsplit;
@@ -147,12 +146,55 @@ struct SplitArgs {
     float *lse_part;
 };
 
+// Blocks of one unit (token row ri, split `split` of `bps` blocks): the 256-slot blocks up
+// to the last visible slot of the index row (every lane of the warp returns the same
+// count).  Dense form: keys 0 .. pos(t) are the slots.
+template <bool DENSE>
+__device__ __forceinline__ int pair_unit_blocks(const Problem &P, const RowInfo &ri, const int32_t *irow, int K,
+                                                int split, int bps, int lane) {
+    if (!row_ok(P, ri)) return 0;
+    int last = -1;
+    if (DENSE) {
+        last = min(ri.pos, ri.len_k - 1);
+    } else {
+        if ((K & 3) == 0) {
+            const int n4 = K >> 2;
+#pragma unroll 4
+            for (int i4 = lane; i4 < n4; i4 += 32) {
+                const int4 x = __ldg(reinterpret_cast<const int4 *>(irow) + i4);
+                if (pair_visible(x.x, ri)) last = 4 * i4;
+                if (pair_visible(x.y, ri)) last = 4 * i4 + 1;
+                if (pair_visible(x.z, ri)) last = 4 * i4 + 2;
+                if (pair_visible(x.w, ri)) last = 4 * i4 + 3;
+            }
+        } else {
+            for (int i = lane; i < K; i += 32)
+                if (pair_visible(__ldg(irow + i), ri)) last = i;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
+    }
+    const int nb_row = (last + PairCfg::BLK) / PairCfg::BLK;   // 0 when no slot is visible
+    const int b_begin = split * bps;
+    return max(0, min(nb_row, b_begin + bps) - b_begin);
+}
+
+// Persistent schedule.  The grid holds at most as many pairs as run at once; pair g takes
+// the units g, g + npairs, g + 2 npairs, ... (unit u = token T - 1 - u / nsplit, split
+// u % nsplit: later, heavier tokens first).  Ring positions, the S^T double buffer and
+// every per-block barrier keep counting across units, so the gathers and the first QKs of
+// the next unit run while the current one finishes its last PV and its epilogue.  Per
+// unit, loader warp 0 publishes the unit's block count (a two-entry table guarded by
+// unit_full / unit_free) and loads its q as soon as the previous unit's last QK has read
+// q_s (q_free).  PV_0 of a unit overwrites O^T only once the P^T of its block 0 is in
+// place, and the softmax warps write that P^T after their epilogue of the previous unit
+// has read O^T out of tensor memory (loads waited for, then a tcgen05 fence before the
+// arrivals), so O^T needs no barrier of its own.
 template <bool DENSE, bool SPLIT = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(512, 1)
-sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_out,
-                       const __grid_constant__ CUtensorMap tm_kv, Problem P,
-                       const __nv_bfloat16 *__restrict__ kv, const int32_t *__restrict__ idx,
-                       __nv_bfloat16 *__restrict__ out, float *__restrict__ lse, SplitArgs sp) {
+sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kv,
+                       Problem P, const int32_t *__restrict__ idx, __nv_bfloat16 *__restrict__ out,
+                       float *__restrict__ lse, SplitArgs sp) {
     using C = PairCfg;
     using namespace sm100;
     extern __shared__ __align__(1024) unsigned char smem[];
@@ -162,18 +204,16 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     const int T = P.total_q;
     static_assert(!(DENSE && SPLIT), "the dense form is not split");
     const int nsplit = SPLIT ? sp.nsplit : 1;
-    const int pair = (int)(blockIdx.x >> 1);
-    const int t = T - 1 - pair / nsplit;                    // heavier (later) tokens first
-    const int split = pair % nsplit;
+    const int bps = SPLIT ? sp.bps : (1 << 24);
+    const int units = T * nsplit;
+    const int npairs = (int)(gridDim.x >> 1);
+    const int pair0 = (int)(blockIdx.x >> 1);
     constexpr bool partial = SPLIT;
     const int K = P.topk;
-    const RowInfo ri = row_info(P, t);
-    const bool rok = row_ok(P, ri);                          // same in both CTAs
-    const int32_t *irow = idx != nullptr ? idx + (int64_t)t * K : nullptr;
     const bool masked = DENSE && idx != nullptr;
 
     const uint32_t sbase = smem_u32(smem);
-    const bool misaligned = (sbase & 1023u) != 0;           // uniform; checked below without an early exit
+    const bool misaligned = (sbase & 1023u) != 0;           // uniform; no unit runs then
     const uint32_t q_s = sbase + C::OFF_Q;
     const uint32_t p_s = sbase + C::OFF_P;
     const uint32_t ring_s = sbase + C::OFF_RING;
@@ -184,19 +224,22 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     float *fs = reinterpret_cast<float *>(smem + C::OFF_FS);
     uint32_t *maskw = reinterpret_cast<uint32_t *>(smem + C::OFF_MASK);
     const uint32_t bar0 = sbase + C::OFF_BAR;
-    auto empty = [&](int s) { return bar0 + 8u * (C::NSLOT + s); };
-    auto pfull = [&](int s) { return bar0 + 8u * (2 * C::NSLOT + s); };
-    const uint32_t q_full = bar0 + 8u * (3 * C::NSLOT);
-    const uint32_t q_peer = q_full + 8;
+    auto empty = [&](int s) { return bar0 + 8u * s; };
+    auto pfull = [&](int s) { return bar0 + 8u * (C::NSLOT + s); };
+    const uint32_t q_full = bar0 + 8u * (2 * C::NSLOT);      // even CTA: q of both CTAs landed
+    const uint32_t q_free = q_full + 8;                      // the unit's last QK has read q_s
     auto s_full = [&](int b) { return q_full + 16 + 8u * b; };
     auto s_free = [&](int b) { return q_full + 32 + 8u * b; };
     const uint32_t p_full = q_full + 48;                    // P^T of both CTAs written (even CTA)
-    const uint32_t pv_done = q_full + 64;
-    const uint32_t o_ready = q_full + 72;
-    auto xbar = [&](int b) { return q_full + 80 + 8u * b; };
-    const uint32_t lbar = q_full + 96;
-    const uint32_t drain = q_full + 104;
-    volatile uint32_t *misc = reinterpret_cast<volatile uint32_t *>(smem + C::OFF_MISC);  // [0] tmem, [1] abort
+    const uint32_t pv_done = q_full + 56;
+    const uint32_t o_ready = q_full + 64;
+    auto xbar = [&](int b) { return q_full + 72 + 8u * b; };
+    const uint32_t lbar = q_full + 88;
+    const uint32_t drain = q_full + 96;
+    auto unit_full = [&](int i) { return q_full + 104 + 8u * i; };
+    auto unit_free = [&](int i) { return q_full + 120 + 8u * i; };
+    volatile uint32_t *misc = reinterpret_cast<volatile uint32_t *>(smem + C::OFF_MISC);
+    volatile int *unit_nb = reinterpret_cast<volatile int *>(smem + C::OFF_MISC + 8);
 
     // ---- setup (every thread of both CTAs reaches the cluster barriers below)
     if (tid == 0 && !misaligned) {
@@ -204,12 +247,14 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             mbar_init(empty(s), 1);
             mbar_init(pfull(s), 1);       // the even CTA's expect-tx for both CTAs' bytes
         }
-        mbar_init(q_full, 1);
-        mbar_init(q_peer, 1);
+        mbar_init(q_full, 1);             // likewise
+        mbar_init(q_free, 1);
         for (int b = 0; b < 2; ++b) {
             mbar_init(s_full(b), 1);
             mbar_init(s_free(b), 16);     // 8 softmax warps of each CTA
             mbar_init(xbar(b), 1);
+            mbar_init(unit_full(b), 1);   // loader warp 0
+            mbar_init(unit_free(b), cr == 0 ? 2 : 1);   // the MMA thread (even CTA), the softmax warps
         }
         mbar_init(p_full, 16);            // 8 softmax warps of each CTA
         mbar_init(pv_done, 1);
@@ -218,53 +263,10 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         mbar_init(drain, 1);
         misc[1] = 0;
         fence_barrier_init();
-        // this CTA's 64 heads of q land while the index row is scanned
-        prefetch_tmap(&tm_q);
-        mbar_expect_tx(q_full, C::NATOM * C::QATOM);
-        for (int a = 0; a < C::NATOM; ++a) tma_load_2d(q_s + a * C::QATOM, &tm_q, q_full, 64 * a, t * 128 + 64 * cr);
     }
     if (tid == 0 && misaligned) {
         raise_error(ERR_SMEM_ALIGN);
         misc[1] = 1;
-    }
-    const char *kv_bytes = reinterpret_cast<const char *>(kv);
-    const int lw = warp;                                     // loader warps 0 .. NLOAD-1
-    const bool loader = warp < C::NLOAD;
-    if (DENSE && warp >= C::SOFT0) {
-        // last visible key; the bitmask of the listed keys (keys 0 .. last)
-        const int part = warp - C::SOFT0;
-        const int last = min(ri.pos, ri.len_k - 1);
-        if (masked && last >= 0) {
-            for (int i = part * 32 + lane; i <= (last >> 5); i += 256) maskw[i] = 0u;
-            named_bar(1, 256);
-            for (int i = part * 32 + lane; i < K; i += 256) {
-                const int e = __ldg(irow + i);
-                if (pair_visible(e, ri)) atomicOr(maskw + (e >> 5), 1u << (e & 31));
-            }
-        }
-        if (lane == 0) reinterpret_cast<int *>(red)[part] = last;
-        if (warp < C::SOFT0 + 4) mr[tid - 32 * C::SOFT0] = -INFINITY;   // reference maxima of the 128 heads
-    } else if (warp >= C::SOFT0) {   // last visible slot of the row (8 warps, interleaved int4 groups)
-        int last = -1;
-        const int part = warp - C::SOFT0;
-        if ((K & 3) == 0) {
-            const int n4 = K >> 2;
-#pragma unroll 2
-            for (int i4 = part * 32 + lane; i4 < n4; i4 += 256) {
-                const int4 x = __ldg(reinterpret_cast<const int4 *>(irow) + i4);
-                if (pair_visible(x.x, ri)) last = 4 * i4;
-                if (pair_visible(x.y, ri)) last = 4 * i4 + 1;
-                if (pair_visible(x.z, ri)) last = 4 * i4 + 2;
-                if (pair_visible(x.w, ri)) last = 4 * i4 + 3;
-            }
-        } else {
-            for (int i = part * 32 + lane; i < K; i += 256)
-                if (pair_visible(__ldg(irow + i), ri)) last = i;
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) last = max(last, __shfl_xor_sync(0xffffffffu, last, o));
-        if (lane == 0) reinterpret_cast<int *>(red)[part] = last;
-        if (warp < C::SOFT0 + 4) mr[tid - 32 * C::SOFT0] = -INFINITY;   // reference maxima of the 128 heads
     }
     cluster_sync();   // both CTAs running, their barriers initialised
     if (warp == 0) tmem_alloc_pair(sbase + C::OFF_MISC, 512);
@@ -272,152 +274,220 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = misc[0];
-    int last_slot = -1;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) last_slot = max(last_slot, reinterpret_cast<int *>(red)[i]);
-    const int nblocks_row = (misaligned || !rok) ? 0 : (last_slot + C::BLK) / C::BLK;   // 0 when no slot is visible
-    const int bps = SPLIT ? sp.bps : nblocks_row;
-    const int b_begin = split * bps;                         // this pair's blocks of the row
-    const int nblocks = max(0, min(nblocks_row, b_begin + bps) - b_begin);
-    // this pair's part of the index row: slots from b_begin * BLK on, ks_left of them
-    const int32_t *irow_s = irow != nullptr ? irow + b_begin * C::BLK : nullptr;
-    const int ks_left = K - b_begin * C::BLK;
-    __syncthreads();   // red is reused by the softmax warps
+    const bool run = !misaligned;
     const uint32_t peer_misc1 = mapa_shared(sbase + C::OFF_MISC + 4, (uint32_t)peer);
     auto abort_pair = [&]() {                                // stop both CTAs of the pair
         misc[1] = 1;
         st_cluster_u32(peer_misc1, 1u);
     };
+    const int lw = warp;                                     // loader warps 0 .. NLOAD-1
+    const bool loader = warp < C::NLOAD && (!DENSE || warp == 0);
 
     if (warp < C::SOFT0) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REG_LOW));
-    if (DENSE && loader) {
-        // ------------------------------------------------ TMA tile loads (one thread per CTA)
-        if (warp == 0 && lane == 0 && nblocks > 0) {
-            const uint32_t lead_pfull = mapa_shared(pfull(0), 0);
+    if (loader) {
+        // ------------------------------------------------ loads: q per unit, ring atoms
+        const uint32_t lead_pfull = mapa_shared(pfull(0), 0);
+        const uint32_t lead_q_full = mapa_shared(q_full, 0);
+        if (lw == 0 && lane == 0) {
+            prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_kv);
-            bool ok = true;
-            int p = 0;
+        }
+        bool ok = run;
+        int p = 0;                                           // ring position, counted across units
+        int nq = 0;                                          // units with blocks so far
+        for (int j = 0, u = pair0; ok && u < units; ++j, u += npairs) {
+            const int t = T - 1 - u / nsplit;
+            const int split = u % nsplit;
+            const RowInfo ri = row_info(P, t);
+            const int32_t *irow = idx != nullptr ? idx + (int64_t)t * K : nullptr;
+            const int nblocks = pair_unit_blocks<DENSE>(P, ri, irow, K, split, bps, lane);
+            if (lw == 0) {
+                bool okw = true;
+                if (lane == 0) {
+                    if (j >= 2) okw = mbar_wait(unit_free(j & 1), ((j >> 1) - 1) & 1);
+                    if (okw) {
+                        unit_nb[j & 1] = nblocks;
+                        mbar_arrive(unit_full(j & 1));
+                    }
+                    if (okw && nblocks > 0 && nq > 0) okw = mbar_wait(q_free, (nq - 1) & 1);
+                    if (okw && nblocks > 0) {
+                        if (cr == 0) mbar_expect_tx(q_full, 2 * C::NATOM * C::QATOM);   // both CTAs' q
+                        for (int a = 0; a < C::NATOM; ++a)
+                            tma_load_2d_pair(q_s + a * C::QATOM, &tm_q, lead_q_full, 64 * a, t * 128 + 64 * cr);
+                    }
+                }
+                if (!__shfl_sync(0xffffffffu, okw, 0)) {
+                    ok = false;
+                    break;
+                }
+            }
+            if (nblocks == 0) continue;
+            ++nq;
+            if (DENSE) {
+                // ---- TMA tile loads of contiguous keys (lane 0 of warp 0)
+                bool okd = true;
+                if (lane == 0) {
+                    for (int g = 0; okd && g < 2 * nblocks; ++g) {
+                        bool qk;
+                        int b;
+                        pair_group(g, nblocks, qk, b);
+                        const int natoms = qk ? C::NATOM : 8;
+                        for (int m = 0; m < natoms; ++m) {
+                            const int pp = p + m, slot = pp % C::NSLOT;
+                            if (pp >= C::NSLOT && !mbar_wait(empty(slot), ((pp / C::NSLOT) - 1) & 1)) {
+                                okd = false;
+                                break;
+                            }
+                            if (misc[1]) {
+                                okd = false;
+                                break;
+                            }
+                            const int h = qk ? cr : ((m >> 1) & 1);
+                            const int a = qk ? m : pv_value_atom(cr, p, m);
+                            if (cr == 0) mbar_expect_tx(pfull(slot), 2 * C::ATOM);   // both CTAs' tiles
+                            tma_load_2d_pair(ring_s + slot * C::ATOM, &tm_kv, lead_pfull + 8u * slot, 64 * a,
+                                             ri.kbase + C::BLK * b + 128 * h);
+                        }
+                        p += natoms;
+                    }
+                }
+                ok = __shfl_sync(0xffffffffu, okd, 0);
+                p = __shfl_sync(0xffffffffu, p, 0);
+            } else {
+                // ---- row gathers (TMA, 4 rows per lane; the loader warps take positions in turn)
+                const int b_begin = split * bps;
+                const int32_t *irow_s = irow + b_begin * C::BLK;
+                const int ks_left = K - b_begin * C::BLK;
+                for (int g = 0; ok && g < 2 * nblocks; ++g) {
+                    bool qk;
+                    int b;
+                    pair_group(g, nblocks, qk, b);
+                    const int natoms = qk ? C::NATOM : 8;
+                    for (int m = 0; m < natoms; ++m) {
+                        const int pp = p + m;
+                        if (pp % C::NLOAD != lw) continue;
+                        const int h = qk ? cr : ((m >> 1) & 1);
+                        const int s0 = C::BLK * b + 128 * h + 4 * lane;   // this lane's 4 slots (of the unit's part)
+                        int e[4];
+                        if ((K & 3) == 0 && s0 + 3 < ks_left) {
+                            const int4 x = __ldg(reinterpret_cast<const int4 *>(irow_s + s0));
+                            e[0] = x.x; e[1] = x.y; e[2] = x.z; e[3] = x.w;
+                        } else {
+#pragma unroll
+                            for (int v = 0; v < 4; ++v) e[v] = s0 + v < ks_left ? __ldg(irow_s + s0 + v) : -1;
+                        }
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) e[v] = key_row(P, ri, pair_visible(e[v], ri) ? e[v] : 0);
+                        const int a = qk ? m : pv_value_atom(cr, p, m);
+                        const int slot = pp % C::NSLOT;
+                        bool okw = true;
+                        if (lane == 0) {
+                            if (pp >= C::NSLOT) okw = mbar_wait(empty(slot), ((pp / C::NSLOT) - 1) & 1);
+                            if (okw && cr == 0) mbar_expect_tx(pfull(slot), 2 * C::ATOM);   // both CTAs' rows
+                        }
+                        if (!__shfl_sync(0xffffffffu, okw, 0) || misc[1]) {
+                            ok = false;
+                            break;
+                        }
+                        tma_gather4_pair(ring_s + slot * C::ATOM + 512 * lane, &tm_kv, lead_pfull + 8u * slot, 64 * a,
+                                         e[0], e[1], e[2], e[3]);
+                    }
+                    p += natoms;
+                }
+            }
+        }
+        if (!ok && lane == 0) abort_pair();
+        // the last q load has landed before the pair may exit (both CTAs' bytes complete on
+        // the even CTA's barrier; the cluster barrier at teardown holds the odd CTA)
+        if (lw == 0 && lane == 0 && cr == 0 && nq > 0) mbar_wait_cluster(q_full, (nq - 1) & 1);
+    } else if (warp == 7 && lane == 0 && cr == 0) {
+        // ------------------------------------------------ MMA issuer (even CTA)
+        const uint32_t idesc_qk = idesc_bf16(256, 128);
+        const uint32_t idesc_pv = idesc_bf16_mn_mn(256, 128);
+        bool ok = run;
+        bool issued = false;
+        int pos = 0;                                         // ring position, counted across units
+        int gb0 = 0;                                         // blocks of the earlier units
+        int nq = 0;                                          // units with blocks so far
+        for (int j = 0, u = pair0; ok && u < units; ++j, u += npairs) {
+            if (!mbar_wait(unit_full(j & 1), (j >> 1) & 1)) {
+                ok = false;
+                break;
+            }
+            const int nblocks = unit_nb[j & 1];
+            mbar_arrive(unit_free(j & 1));
+            if (nblocks == 0) continue;
+            if (!mbar_wait_cluster(q_full, nq & 1) || misc[1]) {
+                ok = false;
+                break;
+            }
             for (int g = 0; ok && g < 2 * nblocks; ++g) {
                 bool qk;
                 int b;
                 pair_group(g, nblocks, qk, b);
-                const int natoms = qk ? C::NATOM : 8;
-                for (int m = 0; m < natoms; ++m) {
-                    const int pp = p + m, slot = pp % C::NSLOT;
-                    if (pp >= C::NSLOT && !mbar_wait(empty(slot), ((pp / C::NSLOT) - 1) & 1)) { ok = false; break; }
-                    if (misc[1]) { ok = false; break; }
-                    const int h = qk ? cr : ((m >> 1) & 1);
-                    const int a = qk ? m : pv_value_atom(cr, p, m);
-                    if (cr == 0) mbar_expect_tx(pfull(slot), 2 * C::ATOM);   // both CTAs' tiles
-                    tma_load_2d_pair(ring_s + slot * C::ATOM, &tm_kv, lead_pfull + 8u * slot, 64 * a,
-                                     ri.kbase + C::BLK * b + 128 * h);
-                }
-                p += natoms;
-            }
-            if (!ok) abort_pair();
-        }
-    } else if (loader) {
-        // ------------------------------------------------ row gathers (TMA, 4 rows per lane)
-        bool ok = true;
-        int p = 0;
-        const uint32_t lead_pfull = mapa_shared(pfull(0), 0);
-        if (lw == 0 && lane == 0) prefetch_tmap(&tm_kv);
-        for (int g = 0; ok && g < 2 * nblocks; ++g) {
-            bool qk;
-            int b;
-            pair_group(g, nblocks, qk, b);
-            const int natoms = qk ? C::NATOM : 8;
-            for (int m = 0; m < natoms; ++m) {
-                const int pp = p + m;
-                if (pp % C::NLOAD != lw) continue;
-                const int h = qk ? cr : ((m >> 1) & 1);
-                const int s0 = C::BLK * b + 128 * h + 4 * lane;   // this lane's 4 slots (of the pair's part)
-                int e[4];
-                if ((K & 3) == 0 && s0 + 3 < ks_left) {
-                    const int4 x = __ldg(reinterpret_cast<const int4 *>(irow_s + s0));
-                    e[0] = x.x; e[1] = x.y; e[2] = x.z; e[3] = x.w;
-                } else {
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) e[u] = s0 + u < ks_left ? __ldg(irow_s + s0 + u) : -1;
-                }
-#pragma unroll
-                for (int u = 0; u < 4; ++u) e[u] = key_row(P, ri, pair_visible(e[u], ri) ? e[u] : 0);
-                const int a = qk ? m : pv_value_atom(cr, p, m);
-                const int slot = pp % C::NSLOT;
-                bool okw = true;
-                if (lane == 0) {
-                    if (pp >= C::NSLOT) okw = mbar_wait(empty(slot), ((pp / C::NSLOT) - 1) & 1);
-                    if (okw && cr == 0) mbar_expect_tx(pfull(slot), 2 * C::ATOM);   // both CTAs' rows
-                }
-                if (!__shfl_sync(0xffffffffu, okw, 0) || misc[1]) { ok = false; break; }
-                tma_gather4_pair(ring_s + slot * C::ATOM + 512 * lane, &tm_kv, lead_pfull + 8u * slot, 64 * a, e[0],
-                                 e[1], e[2], e[3]);
-            }
-            p += natoms;
-        }
-        if (!ok && lane == 0) abort_pair();
-    } else if (warp == 7 && lane == 0 && cr == 0 && nblocks > 0) {
-        // ------------------------------------------------ MMA issuer (even CTA)
-        const uint32_t idesc_qk = idesc_bf16(256, 128);
-        const uint32_t idesc_pv = idesc_bf16_mn_mn(256, 128);
-        bool ok = mbar_wait(q_full, 0) && mbar_wait_cluster(q_peer, 0);
-        bool issued = false;
-        int pos = 0;
-        for (int g = 0; ok && g < 2 * nblocks; ++g) {
-            bool qk;
-            int b;
-            pair_group(g, nblocks, qk, b);
-            if (qk) {                                        // QK_b -> S^T buffer b & 1
-                if (b >= 2 && !mbar_wait_cluster(s_free(b & 1), ((b >> 1) - 1) & 1)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t d = tmem + C::TMEM_S + 128 * (b & 1);
-                for (int a = 0; a < C::NATOM; ++a, ++pos) {
-                    const int slot = pos % C::NSLOT;
-                    const uint32_t par = (pos / C::NSLOT) & 1;
-                    if (!mbar_wait_cluster(pfull(slot), par) || misc[1]) {
+                const int gb = gb0 + b;
+                if (qk) {                                    // QK_b -> S^T buffer gb & 1
+                    if (gb >= 2 && !mbar_wait_cluster(s_free(gb & 1), ((gb >> 1) - 1) & 1)) {
                         ok = false;
                         break;
                     }
-                    const uint32_t sa = ring_s + slot * C::ATOM;
-#pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_f16_pair(d, desc_sw128(sa + kk * 32), desc_sw128(q_s + a * C::QATOM + kk * 32), idesc_qk,
-                                     (a > 0 || kk > 0) ? 1u : 0u);
-                    issued = true;
-                    mma_commit_pair_both(empty(slot));
-                }
-                if (!ok) break;
-                mma_commit_pair_both(s_full(b & 1));
-            } else {                                         // PV_b
-                if (!mbar_wait_cluster(p_full, b & 1)) { ok = false; break; }
-                tc_fence_after();
-                for (int i = 0; ok && i < 2; ++i) {
-                    const uint32_t d = tmem + C::TMEM_O + 128 * i;
-                    for (int h = 0; h < 2; ++h, pos += 2) {
-                        const int s0 = pos % C::NSLOT, s1 = (pos + 1) % C::NSLOT;
-                        const uint32_t par0 = (pos / C::NSLOT) & 1, par1 = ((pos + 1) / C::NSLOT) & 1;
-                        if (!mbar_wait_cluster(pfull(s0), par0) || !mbar_wait_cluster(pfull(s1), par1) || misc[1]) {
+                    tc_fence_after();
+                    const uint32_t d = tmem + C::TMEM_S + 128 * (gb & 1);
+                    for (int a = 0; a < C::NATOM; ++a, ++pos) {
+                        const int slot = pos % C::NSLOT;
+                        const uint32_t par = (pos / C::NSLOT) & 1;
+                        if (!mbar_wait_cluster(pfull(slot), par) || misc[1]) {
                             ok = false;
                             break;
                         }
-                        const int slo = s0 < s1 ? s0 : s1, shi = s0 < s1 ? s1 : s0;
-                        const uint32_t vb = ring_s + slo * C::ATOM;
-                        const uint32_t lbo = (uint32_t)(shi - slo) * C::ATOM;
+                        const uint32_t sa = ring_s + slot * C::ATOM;
 #pragma unroll
-                        for (int k8 = 0; k8 < 8; ++k8)
-                            mma_f16_pair(d, desc_sw128_mn(vb + k8 * 2048, lbo),
-                                         desc_sw128_mn(p_s + (8 * h + k8) * 2048, 16384), idesc_pv,
-                                         (b > 0 || h > 0 || k8 > 0) ? 1u : 0u);
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_f16_pair(d, desc_sw128(sa + kk * 32), desc_sw128(q_s + a * C::QATOM + kk * 32),
+                                         idesc_qk, (a > 0 || kk > 0) ? 1u : 0u);
                         issued = true;
-                        mma_commit_pair_both(empty(s0));
-                        mma_commit_pair_both(empty(s1));
+                        mma_commit_pair_both(empty(slot));
                     }
+                    if (!ok) break;
+                    if (b == nblocks - 1) mma_commit_pair_both(q_free);   // the unit's last read of q_s
+                    mma_commit_pair_both(s_full(gb & 1));
+                } else {                                     // PV_b
+                    if (!mbar_wait_cluster(p_full, gb & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    for (int i = 0; ok && i < 2; ++i) {
+                        const uint32_t d = tmem + C::TMEM_O + 128 * i;
+                        for (int h = 0; h < 2; ++h, pos += 2) {
+                            const int s0 = pos % C::NSLOT, s1 = (pos + 1) % C::NSLOT;
+                            const uint32_t par0 = (pos / C::NSLOT) & 1, par1 = ((pos + 1) / C::NSLOT) & 1;
+                            if (!mbar_wait_cluster(pfull(s0), par0) || !mbar_wait_cluster(pfull(s1), par1) ||
+                                misc[1]) {
+                                ok = false;
+                                break;
+                            }
+                            const int slo = s0 < s1 ? s0 : s1, shi = s0 < s1 ? s1 : s0;
+                            const uint32_t vb = ring_s + slo * C::ATOM;
+                            const uint32_t lbo = (uint32_t)(shi - slo) * C::ATOM;
+#pragma unroll
+                            for (int k8 = 0; k8 < 8; ++k8)
+                                mma_f16_pair(d, desc_sw128_mn(vb + k8 * 2048, lbo),
+                                             desc_sw128_mn(p_s + (8 * h + k8) * 2048, 16384), idesc_pv,
+                                             (b > 0 || h > 0 || k8 > 0) ? 1u : 0u);
+                            issued = true;
+                            mma_commit_pair_both(empty(s0));
+                            mma_commit_pair_both(empty(s1));
+                        }
+                    }
+                    if (!ok) break;
+                    mma_commit_pair_both(pv_done);
+                    if (b == nblocks - 1) mma_commit_pair_both(o_ready);
                 }
-                if (!ok) break;
-                mma_commit_pair_both(pv_done);
-                if (b == nblocks - 1) mma_commit_pair_both(o_ready);
             }
+            gb0 += nblocks;
+            ++nq;
         }
         if (!ok) {
             abort_pair();
@@ -426,12 +496,7 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 mbar_wait(drain, 0);
             }
         }
-    } else if (warp == 7 && lane == 0 && cr == 1 && nblocks > 0) {
-        // ------------------------------------------------ the odd CTA's q has landed
-        if (mbar_wait(q_full, 0)) mbar_arrive_cluster(mapa_shared(q_peer, 0));
-        else abort_pair();
     }
-    if (warp == 0 && lane == 0 && !misaligned) mbar_wait(q_full, 0);   // q landed before exit
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::REG_HIGH));
         // ------------------------------------------------ softmax + epilogue
@@ -446,216 +511,257 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         const uint32_t s_free_lead = mapa_shared(s_free(0), 0);
         const uint32_t p_full_lead = mapa_shared(p_full, 0);
         const uint32_t p_peer_s = mapa_shared(p_s, (uint32_t)peer);
-        float l[64];
-#pragma unroll
-        for (int j = 0; j < 64; ++j) l[j] = 0.f;
-        bool ok = true;
         const int sown = 128 * cr + key;                     // slot of this thread's key within a block
-        int ent = !DENSE && nblocks > 0 && sown < ks_left ? __ldg(irow_s + sown) : -1;
-        for (int b = 0; b < nblocks; ++b) {
-            bool vis;
-            if (DENSE) {
-                const int sk = C::BLK * b + sown;            // the key itself
-                vis = sk <= ri.pos && sk < ri.len_k && (!masked || ((maskw[sk >> 5] >> (sk & 31)) & 1u));
-            } else {
-                vis = pair_visible(ent, ri);
-                const int s = C::BLK * (b + 1) + sown;
-                ent = (b + 1 < nblocks && s < ks_left) ? __ldg(irow_s + s) : -1;
+        bool ok = run;
+        int gb0 = 0;                                         // blocks of the earlier units
+        int nq = 0;                                          // units with blocks so far
+        for (int j = 0, u = pair0; ok && u < units; ++j, u += npairs) {
+            const int t = T - 1 - u / nsplit;
+            const int split = u % nsplit;
+            const RowInfo ri = row_info(P, t);
+            const bool got = mbar_wait(unit_full(j & 1), (j >> 1) & 1);
+            const int nblocks = got ? unit_nb[j & 1] : 0;
+            if (named_bar_or(1, 256, !got || misc[1] != 0)) {
+                ok = false;
+                break;
             }
-            const bool fail = misc[1] != 0 || !mbar_wait_cluster(s_full(b & 1), (b >> 1) & 1);
-            if (named_bar_or(1, 256, fail)) { ok = false; break; }
-            tc_fence_after();
-            const uint32_t sb = t_lane + C::TMEM_S + 128 * (b & 1) + 64 * h2;
-            // ---- exact block maxima of this CTA's keys (per head), then of the pair
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                uint32_t sr[32];
-                float v[32];
-                tmem_ld32(sb + 32 * j, sr);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] = vis ? __uint_as_float(sr[i]) : -INFINITY;
-                red[quarter * 128 + 64 * h2 + 32 * j + lane] = transpose_reduce32<true>(v, lane);
-            }
-            named_bar(1, 256);
-            bool need = false;
-            if (st < 128) {
-                const int h = st;
-                const float m_cta = fmaxf(fmaxf(red[h], red[128 + h]), fmaxf(red[256 + h], red[384 + h]));
-                st_async_f32(xm_peer + 4u * (128 * (b & 1) + h), m_cta, xbar_peer + 8u * (b & 1));
-                if (st == 0) mbar_expect_tx(xbar(b & 1), 128 * 4);
-                const bool okx = mbar_wait_cluster(xbar(b & 1), (b >> 1) & 1);
-                const float m_blk = fmaxf(m_cta, okx ? xm[128 * (b & 1) + h] : m_cta) * sl2;
-                const float m_old = mr[h];
-                need = m_blk > m_old + C::TAU;
-                const float m_new = need ? m_blk : m_old;
-                fs[h] = (need && m_old != -INFINITY) ? exp2f(m_old - m_new) : 1.0f;
-                mr[h] = m_new;
-                if (!okx) misc[1] = 1;
-            }
-            // every exit decision below is taken through a barrier, so the 8 warps stay together
-            const bool any = named_bar_or(1, 256, need);
-            bool pv_waited = false;
-            if (any) {
-#pragma unroll
-                for (int j = 0; j < 64; ++j) l[j] *= fs[64 * h2 + j];
-                if (b > 0) {
-                    // O^T must hold PV_{b-1} before it is rescaled; PV_b cannot start before
-                    // this CTA's P^T arrives below
-                    const bool okp = mbar_wait_cluster(pv_done, (b - 1) & 1);
-                    pv_waited = true;
-                    tc_fence_after();
-                    if (__all_sync(0xffffffffu, okp)) {
-#pragma unroll 1
-                        for (int ch = 0; ch < 4; ++ch) {
-                            uint32_t o[32];
-                            const uint32_t oa = t_lane + C::TMEM_O + 128 * h2 + 32 * ch;
-                            tmem_ld32(oa, o);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * fs[32 * ch + i]);
-                            tmem_st32(oa, o);
-                        }
-                        tmem_wait_st();
-                    }
+            if (st == 0) mbar_arrive(unit_free(j & 1));
+            const int32_t *irow_s = idx != nullptr ? idx + (int64_t)t * K + split * bps * C::BLK : nullptr;
+            const int ks_left = K - split * bps * C::BLK;
+            if (masked && nblocks > 0) {
+                // bitmask of the listed keys (keys 0 .. last)
+                const int last = min(ri.pos, ri.len_k - 1);
+                for (int i = st; i <= (last >> 5); i += 256) maskw[i] = 0u;
+                named_bar(1, 256);
+                for (int i = st; i < K; i += 256) {
+                    const int e = __ldg(irow_s + i);
+                    if (pair_visible(e, ri)) atomicOr(maskw + (e >> 5), 1u << (e & 31));
                 }
+                named_bar(1, 256);
             }
-            // ---- P^T of this thread's key for its 64 heads (bf16 pairs)
-            uint32_t pk[32];
+            if (st < 128) mr[st] = -INFINITY;                // reference maxima of the 128 heads
+            float l[64];
 #pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                uint32_t sr[32];
-                tmem_ld32(sb + 32 * j, sr);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float2 m2 = reinterpret_cast<const float2 *>(mr)[32 * h2 + 16 * j + i];
-                    const float p0 = vis ? ex2_approx(fmaf(__uint_as_float(sr[2 * i]), sl2, -m2.x)) : 0.f;
-                    const float p1 = vis ? ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -m2.y)) : 0.f;
-                    l[32 * j + 2 * i] += p0;
-                    l[32 * j + 2 * i + 1] += p1;
-                    pk[16 * j + i] = pack_bf16x2(p0, p1);
-                }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(s_free_lead + 8u * (b & 1));   // S^T_b consumed
-            if (b > 0 && !pv_waited) {
-                // PV_{b-1} still reads the P^T buffer
-                const bool okp = mbar_wait_cluster(pv_done, (b - 1) & 1);
-                if (!okp) misc[1] = 1;
-            }
-            {
-                // row 128 cr + key of the P^T buffer of the CTA holding heads 64 h2 .. + 63
-                const uint32_t row = (uint32_t)(128 * cr + key);
-                if (h2 == cr) {
-                    const uint32_t base = p_s + row * 128;
-#pragma unroll
-                    for (int u = 0; u < 8; ++u)
-                        st_shared_v4(base + ((u ^ (row & 7)) << 4), pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-                    fence_proxy_async_smem();
+            for (int i = 0; i < 64; ++i) l[i] = 0.f;
+            int ent = !DENSE && nblocks > 0 && sown < ks_left ? __ldg(irow_s + sown) : -1;
+            for (int b = 0; b < nblocks; ++b) {
+                const int gb = gb0 + b;
+                bool vis;
+                if (DENSE) {
+                    const int sk = C::BLK * b + sown;        // the key itself
+                    vis = sk <= ri.pos && sk < ri.len_k && (!masked || ((maskw[sk >> 5] >> (sk & 31)) & 1u));
                 } else {
-                    const uint32_t base = p_peer_s + row * 128;
-#pragma unroll
-                    for (int u = 0; u < 8; ++u)
-                        st_cluster_v4(base + ((u ^ (row & 7)) << 4), pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-                    fence_proxy_async_cluster();
+                    vis = pair_visible(ent, ri);
+                    const int s = C::BLK * (b + 1) + sown;
+                    ent = (b + 1 < nblocks && s < ks_left) ? __ldg(irow_s + s) : -1;
                 }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(p_full_lead);   // this warp's 32 rows are in place
-            if (named_bar_or(1, 256, misc[1] != 0)) { ok = false; break; }
-        }
-        if (!ok && st == 0) abort_pair();
-
-        // ---- epilogue: row sums of the pair, lse, O^T / l transposed into out
-        const int64_t obase = (int64_t)t * 128;
-        const int64_t pbase = ((int64_t)t * nsplit + split) * 128;   // partial rows (split mode)
-        if (nblocks > 0 && ok) {
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                float v[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] = l[32 * j + i];
-                red[quarter * 128 + 64 * h2 + 32 * j + lane] = transpose_reduce32<false>(v, lane);
-            }
-            named_bar(1, 256);
-            if (st < 128) {
-                const int h = st;
-                const float l_cta = (red[h] + red[128 + h]) + (red[256 + h] + red[384 + h]);
-                st_async_f32(mapa_shared(sbase + C::OFF_XL + 4u * h, (uint32_t)peer), l_cta,
-                             mapa_shared(lbar, (uint32_t)peer));
-                if (st == 0) mbar_expect_tx(lbar, 128 * 4);
-                const bool okl = mbar_wait_cluster(lbar, 0);
-                // the two CTAs add the same two numbers in the same order
-                const float l_tot = cr == 0 ? l_cta + xl[h] : xl[h] + l_cta;
-                const bool fine = okl && l_tot > 0.f;
-                fs[h] = fine ? 1.0f / l_tot : 0.f;
-                if ((h >> 6) == cr) {
-                    const float lv = okl ? (l_tot > 0.f ? (mr[h] + log2f(l_tot)) * 0.6931471805599453f : -INFINITY) : NAN;
-                    if (partial) sp.lse_part[pbase + h] = lv;
-                    else lse[obase + h] = lv;
+                const bool fail = misc[1] != 0 || !mbar_wait_cluster(s_full(gb & 1), (gb >> 1) & 1);
+                if (named_bar_or(1, 256, fail)) {
+                    ok = false;
+                    break;
                 }
-            }
-            const bool oko = mbar_wait_cluster(o_ready, 0);
-            named_bar(1, 256);
-            tc_fence_after();
-            // O^T block i = h2: lanes = value dims 256 h2 + 128 cr + quarter*32 + lane, columns = heads
-            if (partial) {   // fp32 partial rows, written from registers (32 lanes: 128 bytes per head)
-                float *op = sp.o_part + pbase * 512 + 256 * h2 + 128 * cr + key;
-#pragma unroll 1
-                for (int ch = 0; ch < 4; ++ch) {
-                    uint32_t o[32];
-                    tmem_ld32(t_lane + C::TMEM_O + 128 * h2 + 32 * ch, o);
+                tc_fence_after();
+                const uint32_t sb = t_lane + C::TMEM_S + 128 * (gb & 1) + 64 * h2;
+                // ---- exact block maxima of this CTA's keys (per head), then of the pair
+#pragma unroll
+                for (int jj = 0; jj < 2; ++jj) {
+                    uint32_t sr[32];
+                    float v[32];
+                    tmem_ld32(sb + 32 * jj, sr);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int h = 32 * ch + i;
-                        op[(int64_t)h * 512] = oko ? __uint_as_float(o[i]) * fs[h] : 0.f;
+                    for (int i = 0; i < 32; ++i) v[i] = vis ? __uint_as_float(sr[i]) : -INFINITY;
+                    red[quarter * 128 + 64 * h2 + 32 * jj + lane] = transpose_reduce32<true>(v, lane);
+                }
+                named_bar(1, 256);
+                bool need = false;
+                if (st < 128) {
+                    const int h = st;
+                    const float m_cta = fmaxf(fmaxf(red[h], red[128 + h]), fmaxf(red[256 + h], red[384 + h]));
+                    st_async_f32(xm_peer + 4u * (128 * (gb & 1) + h), m_cta, xbar_peer + 8u * (gb & 1));
+                    if (st == 0) mbar_expect_tx(xbar(gb & 1), 128 * 4);
+                    const bool okx = mbar_wait_cluster(xbar(gb & 1), (gb >> 1) & 1);
+                    const float m_blk = fmaxf(m_cta, okx ? xm[128 * (gb & 1) + h] : m_cta) * sl2;
+                    const float m_old = mr[h];
+                    need = m_blk > m_old + C::TAU;
+                    const float m_new = need ? m_blk : m_old;
+                    fs[h] = (need && m_old != -INFINITY) ? exp2f(m_old - m_new) : 1.0f;
+                    mr[h] = m_new;
+                    if (!okx) misc[1] = 1;
+                }
+                // every exit decision below is taken through a barrier, so the 8 warps stay together
+                const bool any = named_bar_or(1, 256, need);
+                bool pv_waited = false;
+                if (any) {
+#pragma unroll
+                    for (int i = 0; i < 64; ++i) l[i] *= fs[64 * h2 + i];
+                    if (b > 0) {
+                        // O^T must hold PV_{b-1} before it is rescaled; PV_b cannot start before
+                        // this CTA's P^T arrives below
+                        const bool okp = mbar_wait_cluster(pv_done, (gb - 1) & 1);
+                        pv_waited = true;
+                        tc_fence_after();
+                        if (__all_sync(0xffffffffu, okp)) {
+#pragma unroll 1
+                            for (int ch = 0; ch < 4; ++ch) {
+                                uint32_t o[32];
+                                const uint32_t oa = t_lane + C::TMEM_O + 128 * h2 + 32 * ch;
+                                tmem_ld32(oa, o);
+                                tmem_wait_ld();
+#pragma unroll
+                                for (int i = 0; i < 32; ++i)
+                                    o[i] = __float_as_uint(__uint_as_float(o[i]) * fs[32 * ch + i]);
+                                tmem_st32(oa, o);
+                            }
+                            tmem_wait_st();
+                        }
                     }
                 }
-            }
-            const uint32_t ostg = ring_s + (uint32_t)h2 * (128 * 256);
-#pragma unroll 1
-            for (int ch = 0; !partial && ch < 4; ++ch) {
-                uint32_t o[32];
-                tmem_ld32(t_lane + C::TMEM_O + 128 * h2 + 32 * ch, o);
-                tmem_wait_ld();
+                // ---- P^T of this thread's key for its 64 heads (bf16 pairs)
+                uint32_t pk[32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int h = 32 * ch + i;
-                    const float val = oko ? __uint_as_float(o[i]) * fs[h] : 0.f;
-                    st_shared_u16(ostg + h * 256 + key * 2, __bfloat16_as_ushort(__float2bfloat16_rn(val)));
+                for (int jj = 0; jj < 2; ++jj) {
+                    uint32_t sr[32];
+                    tmem_ld32(sb + 32 * jj, sr);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float2 m2 = reinterpret_cast<const float2 *>(mr)[32 * h2 + 16 * jj + i];
+                        const float p0 = vis ? ex2_approx(fmaf(__uint_as_float(sr[2 * i]), sl2, -m2.x)) : 0.f;
+                        const float p1 = vis ? ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), sl2, -m2.y)) : 0.f;
+                        l[32 * jj + 2 * i] += p0;
+                        l[32 * jj + 2 * i + 1] += p1;
+                        pk[16 * jj + i] = pack_bf16x2(p0, p1);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(s_free_lead + 8u * (gb & 1));   // S^T consumed
+                if (b > 0 && !pv_waited) {
+                    // PV_{b-1} still reads the P^T buffer (block 0's predecessor, the previous
+                    // unit's last PV, completed before that unit's epilogue)
+                    const bool okp = mbar_wait_cluster(pv_done, (gb - 1) & 1);
+                    if (!okp) misc[1] = 1;
+                }
+                {
+                    // row 128 cr + key of the P^T buffer of the CTA holding heads 64 h2 .. + 63
+                    const uint32_t row = (uint32_t)(128 * cr + key);
+                    if (h2 == cr) {
+                        const uint32_t base = p_s + row * 128;
+#pragma unroll
+                        for (int v = 0; v < 8; ++v)
+                            st_shared_v4(base + ((v ^ (row & 7)) << 4), pk[4 * v], pk[4 * v + 1], pk[4 * v + 2],
+                                         pk[4 * v + 3]);
+                        fence_proxy_async_smem();
+                    } else {
+                        const uint32_t base = p_peer_s + row * 128;
+#pragma unroll
+                        for (int v = 0; v < 8; ++v)
+                            st_cluster_v4(base + ((v ^ (row & 7)) << 4), pk[4 * v], pk[4 * v + 1], pk[4 * v + 2],
+                                          pk[4 * v + 3]);
+                        fence_proxy_async_cluster();
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(p_full_lead);   // this warp's 32 rows are in place
+                if (named_bar_or(1, 256, misc[1] != 0)) {
+                    ok = false;
+                    break;
                 }
             }
-            fence_proxy_async_smem();
-            named_bar(1, 256);
-            if (st == 0 && !partial) {
-                prefetch_tmap(&tm_out);
-                for (int i = 0; i < 2; ++i)
-                    tma_store_2d(&tm_out, ring_s + (uint32_t)i * (128 * 256), 256 * i + 128 * cr, (int)obase);
-                bulk_commit();
-                bulk_wait_all();
-            }
-        } else {
-            // no visible slot (or an aborted pipeline): out = 0, lse = -inf (NaN if aborted)
-            for (int e = st; e < 128 * 32; e += 256) {
-                const int h = e >> 5, part = e & 31;          // 32 x 16 bytes per head: the CTA's 2 x 128 dims
-                const int d0 = 256 * (part >> 4) + 128 * cr + 8 * (part & 15);
-                if (partial) {
-                    float4 *op = reinterpret_cast<float4 *>(sp.o_part + (pbase + h) * 512 + d0);
-                    op[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-                    op[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (!ok && st == 0) abort_pair();
+
+            // ---- epilogue: row sums of the pair, lse, O^T / l transposed into out
+            const int64_t obase = (int64_t)t * 128;
+            const int64_t pbase = ((int64_t)t * nsplit + split) * 128;   // partial rows (split mode)
+            if (nblocks > 0 && ok) {
+#pragma unroll
+                for (int jj = 0; jj < 2; ++jj) {
+                    float v[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = l[32 * jj + i];
+                    red[quarter * 128 + 64 * h2 + 32 * jj + lane] = transpose_reduce32<false>(v, lane);
+                }
+                named_bar(1, 256);
+                if (st < 128) {
+                    const int h = st;
+                    const float l_cta = (red[h] + red[128 + h]) + (red[256 + h] + red[384 + h]);
+                    st_async_f32(mapa_shared(sbase + C::OFF_XL + 4u * h, (uint32_t)peer), l_cta,
+                                 mapa_shared(lbar, (uint32_t)peer));
+                    if (st == 0) mbar_expect_tx(lbar, 128 * 4);
+                    const bool okl = mbar_wait_cluster(lbar, nq & 1);
+                    // the two CTAs add the same two numbers in the same order
+                    const float l_tot = cr == 0 ? l_cta + xl[h] : xl[h] + l_cta;
+                    const bool fine = okl && l_tot > 0.f;
+                    fs[h] = fine ? 1.0f / l_tot : 0.f;
+                    if ((h >> 6) == cr) {
+                        const float lv =
+                            okl ? (l_tot > 0.f ? (mr[h] + log2f(l_tot)) * 0.6931471805599453f : -INFINITY) : NAN;
+                        if (partial) sp.lse_part[pbase + h] = lv;
+                        else lse[obase + h] = lv;
+                    }
+                }
+                const bool oko = mbar_wait_cluster(o_ready, nq & 1);
+                named_bar(1, 256);
+                tc_fence_after();
+                // O^T block i = h2: lanes = value dims 256 h2 + 128 cr + quarter*32 + lane, columns = heads
+                if (partial) {   // fp32 partial rows, written from registers (32 lanes: 128 bytes per head)
+                    float *op = sp.o_part + pbase * 512 + 256 * h2 + 128 * cr + key;
+#pragma unroll 1
+                    for (int ch = 0; ch < 4; ++ch) {
+                        uint32_t o[32];
+                        tmem_ld32(t_lane + C::TMEM_O + 128 * h2 + 32 * ch, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const int h = 32 * ch + i;
+                            op[(int64_t)h * 512] = oko ? __uint_as_float(o[i]) * fs[h] : 0.f;
+                        }
+                    }
                 } else {
-                    *reinterpret_cast<uint4 *>(out + (obase + h) * 512 + d0) = make_uint4(0, 0, 0, 0);
+                    // bf16 rows from registers: lanes 2m and 2m + 1 swap one value per head pair, so
+                    // each stores two adjacent dims of one head (64 contiguous bytes per head per warp)
+                    const bool odd = (lane & 1) != 0;
+                    __nv_bfloat16 *orow = out + obase * 512 + 256 * h2 + 128 * cr + 32 * quarter + (lane & ~1);
+#pragma unroll 1
+                    for (int ch = 0; ch < 4; ++ch) {
+                        uint32_t o[32];
+                        tmem_ld32(t_lane + C::TMEM_O + 128 * h2 + 32 * ch, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; i += 2) {
+                            const int h = 32 * ch + i;
+                            const float v0 = oko ? __uint_as_float(o[i]) * fs[h] : 0.f;
+                            const float v1 = oko ? __uint_as_float(o[i + 1]) * fs[h + 1] : 0.f;
+                            const float recv = __shfl_xor_sync(0xffffffffu, odd ? v0 : v1, 1);
+                            const uint32_t w = odd ? pack_bf16x2(recv, v1) : pack_bf16x2(v0, recv);
+                            *reinterpret_cast<uint32_t *>(orow + (int64_t)(h + (odd ? 1 : 0)) * 512) = w;
+                        }
+                    }
+                }
+                // O^T read out: ordered before this warp's next arrivals (s_free, p_full) by the
+                // tcgen05 fence that precedes them
+            } else {
+                // no visible slot (or an aborted pipeline): out = 0, lse = -inf (NaN if aborted)
+                for (int e = st; e < 128 * 32; e += 256) {
+                    const int h = e >> 5, part = e & 31;      // 32 x 16 bytes per head: the CTA's 2 x 128 dims
+                    const int d0 = 256 * (part >> 4) + 128 * cr + 8 * (part & 15);
+                    if (partial) {
+                        float4 *op = reinterpret_cast<float4 *>(sp.o_part + (pbase + h) * 512 + d0);
+                        op[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+                        op[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    } else {
+                        *reinterpret_cast<uint4 *>(out + (obase + h) * 512 + d0) = make_uint4(0, 0, 0, 0);
+                    }
+                }
+                if (st < 128 && (st >> 6) == cr) {
+                    const float lv = nblocks == 0 ? -INFINITY : NAN;
+                    if (partial) sp.lse_part[pbase + st] = lv;
+                    else lse[obase + st] = lv;
                 }
             }
-            if (st < 128 && (st >> 6) == cr) {
-                const float lv = nblocks == 0 ? -INFINITY : NAN;
-                if (partial) sp.lse_part[pbase + st] = lv;
-                else lse[obase + st] = lv;
-            }
-            if (st == 0) bulk_wait_all();
+            gb0 += nblocks;
+            if (nblocks > 0) ++nq;
         }
     }
     // ---- teardown: nothing of either CTA is in flight past this point
