@@ -355,30 +355,49 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 ok = __shfl_sync(0xffffffffu, okd, 0);
                 p = __shfl_sync(0xffffffffu, p, 0);
             } else {
-                // ---- row gathers (TMA, 4 rows per lane; the loader warps take positions in turn)
+                // ---- row gathers (TMA gather4: 4 rows per lane, one atom per warp and ring
+                // position; the loader warps take the positions in turn).  All atoms of a group
+                // gather the same rows, so each lane loads the index entries of the next group
+                // while the current one is issued.
                 const int b_begin = split * bps;
                 const int32_t *irow_s = irow + b_begin * C::BLK;
                 const int ks_left = K - b_begin * C::BLK;
+                auto entries = [&](int b, int h) {               // raw entries of this lane's 4 slots
+                    const int s0 = C::BLK * b + 128 * h + 4 * lane;
+                    int4 x;
+                    if ((K & 3) == 0 && s0 + 3 < ks_left) {
+                        x = __ldg(reinterpret_cast<const int4 *>(irow_s + s0));
+                    } else {
+                        x.x = s0 < ks_left ? __ldg(irow_s + s0) : -1;
+                        x.y = s0 + 1 < ks_left ? __ldg(irow_s + s0 + 1) : -1;
+                        x.z = s0 + 2 < ks_left ? __ldg(irow_s + s0 + 2) : -1;
+                        x.w = s0 + 3 < ks_left ? __ldg(irow_s + s0 + 3) : -1;
+                    }
+                    return x;
+                };
+                // group g needs key half cr of block b (QK_b, kept in e0) or both halves (PV_b)
+                int4 e0 = entries(0, cr), e1 = make_int4(-1, -1, -1, -1);
                 for (int g = 0; ok && g < 2 * nblocks; ++g) {
                     bool qk;
                     int b;
                     pair_group(g, nblocks, qk, b);
+                    int4 n0 = e0, n1 = e1;
+                    if (g + 1 < 2 * nblocks) {
+                        bool qk1;
+                        int b1;
+                        pair_group(g + 1, nblocks, qk1, b1);
+                        n0 = entries(b1, qk1 ? cr : 0);
+                        if (!qk1) n1 = entries(b1, 1);
+                    }
                     const int natoms = qk ? C::NATOM : 8;
                     for (int m = 0; m < natoms; ++m) {
                         const int pp = p + m;
                         if (pp % C::NLOAD != lw) continue;
-                        const int h = qk ? cr : ((m >> 1) & 1);
-                        const int s0 = C::BLK * b + 128 * h + 4 * lane;   // this lane's 4 slots (of the unit's part)
+                        const int4 x = (!qk && ((m >> 1) & 1)) ? e1 : e0;
+                        const int r[4] = {x.x, x.y, x.z, x.w};
                         int e[4];
-                        if ((K & 3) == 0 && s0 + 3 < ks_left) {
-                            const int4 x = __ldg(reinterpret_cast<const int4 *>(irow_s + s0));
-                            e[0] = x.x; e[1] = x.y; e[2] = x.z; e[3] = x.w;
-                        } else {
 #pragma unroll
-                            for (int v = 0; v < 4; ++v) e[v] = s0 + v < ks_left ? __ldg(irow_s + s0 + v) : -1;
-                        }
-#pragma unroll
-                        for (int v = 0; v < 4; ++v) e[v] = key_row(P, ri, pair_visible(e[v], ri) ? e[v] : 0);
+                        for (int v = 0; v < 4; ++v) e[v] = key_row(P, ri, pair_visible(r[v], ri) ? r[v] : 0);
                         const int a = qk ? m : pv_value_atom(cr, p, m);
                         const int slot = pp % C::NSLOT;
                         bool okw = true;
@@ -393,6 +412,8 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                         tma_gather4_pair(ring_s + slot * C::ATOM + 512 * lane, &tm_kv, lead_pfull + 8u * slot, 64 * a,
                                          e[0], e[1], e[2], e[3]);
                     }
+                    e0 = n0;
+                    e1 = n1;
                     p += natoms;
                 }
             }
