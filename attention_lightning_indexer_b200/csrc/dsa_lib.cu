@@ -97,22 +97,6 @@ bool make_tmap_rows(CUtensorMap *m, const void *base, bool fp8, uint64_t cols, u
     return r == CUDA_SUCCESS;
 }
 
-// 2-D row-major bf16 tensor map (`cols` x `rows`) with a `box_cols` x `box_rows` box and
-// no swizzle (TMA stores of row-major tiles staged in shared memory).
-bool make_tmap_plain_bf16(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint32_t box_cols,
-                          uint32_t box_rows) {
-    auto enc = tensor_map_encoder();
-    if (enc == nullptr) return false;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * 2};
-    cuuint32_t box[2] = {box_cols, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
 inline dsa_status_t launch_status() {
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;

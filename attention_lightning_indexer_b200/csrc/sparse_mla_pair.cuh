@@ -1,5 +1,6 @@
-// sparse_mla_pair.cuh -- attention over the selected latent rows (MLA in MQA mode) on a
-// pair of SMs: one 2-CTA cluster per query token, 2-SM tensor-core MMAs (cta_group::2).
+// sparse_mla_pair.cuh -- attention over the selected latent rows (MLA in MQA mode) on
+// pairs of SMs: persistent 2-CTA clusters that take query tokens in turn, 2-SM tensor-core
+// MMAs (cta_group::2).
 //
 // "DeepSeek-V3.2 tech report summary", §1 DSA: full attention only over the k selected
 // tokens; MLA-based implementation in MQA mode (every 576-d latent row is shared by all
@@ -49,11 +50,11 @@
 // atom with a 2-SM TMA tile load that completes on the even CTA's barrier.  With all
 // visible keys listed in order the two modes run the same MMAs on the same operands.
 //
-// Warp roles (16 warps per CTA): 0-6 gather (0 also issues the q TMA and allocates tensor
-// memory; in dense mode only warp 0 loads, one tile per atom), 7 issues the MMAs (even
-// CTA), 8-15 scan the index row, then run the softmax and the epilogue: warp w owns TMEM
-// lane quarter w % 4 and head half (w - 8) / 4.  The first two warpgroups give registers
-// to the last two (setmaxnreg).
+// Warp roles (16 warps per CTA): 0-6 gather and each scan a unit's index row for its block
+// count (0 also publishes the count, issues the q TMA and allocates tensor memory; in dense
+// mode only warp 0 loads, one tile per atom), 7 issues the MMAs (even CTA), 8-15 run the
+// softmax and the epilogue: warp w owns TMEM lane quarter w % 4 and head half (w - 8) / 4.
+// The first two warpgroups give registers to the last two (setmaxnreg).
 #pragma once
 
 #include "dsa_common.cuh"

@@ -43,11 +43,12 @@ FLOP_PER_PAIR_MLA = 128 * (576 + 512) * 2       # per (query, selected key) pair
 # sha256 of the source file it was captured from; reported only while the source is
 # unchanged.
 TRAFFIC = {
-    # ncu capture of the 4096-query prefill launch: 1.142 GB of DRAM traffic (643 MB read,
-    # 499 MB written: q reads and out writes, both proportional to the query count; kv rows
-    # come from L2), scaled x8 to the 32768-query launch of the 32K step (that prefill only:
-    # at 128K the kv rows no longer fit in L2)
-    "sparse_mla": {"bytes_per_launch": 1.141754e9 * 8, "total_q": 32768, "src_sha": "d9a63f4278d4b7f9"},
+    # ncu capture of the 4096-query prefill launch (persistent pairs): 1.143 GB of DRAM
+    # traffic (642 MB read, 501 MB written: q reads and out writes, both proportional to the
+    # query count; kv rows come from L2), scaled x8 to the 32768-query launch of the 32K step
+    # (that prefill only: at 128K the kv rows no longer fit in L2); the hash is of the source
+    # as captured plus comment-only edits
+    "sparse_mla": {"bytes_per_launch": 1.142902e9 * 8, "total_q": 32768, "src_sha": "730f3743a3d16970"},
 }
 
 
@@ -194,6 +195,22 @@ def _tokens(inp):
     return int(inp["total_q"])
 
 
+# Longest key sequence the library's forward attends in the dense (masked) form alone
+# (include/dsa.h, dsa_forward).
+DENSE_KV_THRESHOLD = 3584
+
+
+def _attention_launches(p) -> int:
+    """Attention launches of one dsa_forward call on a prefill without split partials: the
+    dense form alone for short key sequences; in one packed, unpaged sequence the rows whose
+    visible keys all fit in topk take the dense form and the rest the gathered form."""
+    if not p.block_table and p.max_len_k <= DENSE_KV_THRESHOLD:
+        return 1
+    T = p.total_q
+    R = min(max(p.topk - (p.total_k - T), 0), T) if not p.cu_q and not p.block_table else 0
+    return 2 if 0 < R < T else 1
+
+
 # ----------------------------------------------------------------- our arm
 
 def _forward_args(inp):
@@ -250,7 +267,7 @@ def run_ours(args, ws, rank, local, dist):
 
     tokens = _tokens(inp)
     n_chunks = (T + (chunk or T) - 1) // (chunk or T)
-    launches_per_step = 2 * n_chunks + 1
+    launches_per_step = 2 * n_chunks + _attention_launches(p)
     res = {
         "metric": METRIC,
         "value": ws * tokens * args.steps / (total_ms / 1e3),
