@@ -286,6 +286,33 @@ def test_sparse_mla_rows_without_valid_keys():
     assert torch.all(out[9] == 0) and torch.all(torch.isneginf(lse[9]))
 
 
+def test_sparse_mla_units_of_every_length_in_one_pair():
+    # 600 rows on at most 74 CTA pairs: each pair walks ~8 rows in turn, among them rows
+    # without a visible slot (all -1, or only future keys), rows whose only visible slot is
+    # the first or the last one (1 or 4 blocks), and rows with holes; the pipeline state
+    # carried from row to row must not leak into the next row's output
+    L, k = 600, 1000
+    inp = dsa_synth.make_prefill(L, topk=k, seed=21, device=DEV)
+    idx = _random_idx(inp, k, seed=21)
+    rng = np.random.default_rng(22)
+    rows = rng.permutation(np.arange(100, L))
+    empty, future, first, last, holes = np.split(rows[:250], 5)
+    idx[empty] = -1
+    for t in future:
+        idx[t] = t + 1 + rng.integers(0, L - t - 1, k) if t + 2 < L else -1   # keys after pos(t) = t
+    for t in first:
+        idx[t] = -1
+        idx[t, 0] = rng.integers(0, t + 1)
+    for t in last:
+        idx[t] = -1
+        idx[t, k - 1] = rng.integers(0, t + 1)
+    for t in holes:
+        idx[t, rng.choice(k, k // 2, replace=False)] = -1
+    out, lse = _check_mla(inp, idx)
+    for t in np.concatenate([empty, future]):
+        assert torch.all(out[int(t)] == 0) and torch.all(torch.isneginf(lse[int(t)]))
+
+
 def test_sparse_mla_topk_not_multiple_of_four_with_repeated_indices():
     # 130 slots: rows of idx are not 16-byte aligned (scalar index loads) and the second
     # block is partial; some rows list a visible key twice (it counts once per occurrence)
@@ -538,6 +565,28 @@ def test_dense_mla_masked_by_index_rows_equals_sparse_attention():
     lse = torch.empty((L, 128), dtype=torch.float32, device=DEV)
     dsa.dsa_dense_mla_fwd(p, inp["q"], inp["kv"], torch.from_numpy(idx_np).to(DEV), out, lse)
     _assert_mla_close(out, lse, *_oracle_mla(inp, idx_np))
+
+
+def test_dense_mla_masked_rows_without_listed_keys_among_others():
+    # 500 rows walked by at most 74 pairs; some index rows list no visible key (all -1, or
+    # only keys after pos(t)): those rows still run their blocks (the dense form's blocks come
+    # from pos(t)) and must come out as 0 / -inf, and the next row of the pair must not see
+    # their state
+    L, k = 500, 96
+    inp = dsa_synth.make_prefill(L, topk=k, seed=33, device=DEV)
+    idx_np = _random_idx(inp, k, seed=33)
+    rng = np.random.default_rng(34)
+    rows = rng.choice(np.arange(50, L - 2), 60, replace=False)
+    idx_np[rows[:30]] = -1
+    for t in rows[30:]:
+        idx_np[t] = t + 1 + rng.integers(0, L - t - 1, k)
+    p = dsa.problem_from_inputs(inp)
+    out = torch.empty((L, 128, 512), dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty((L, 128), dtype=torch.float32, device=DEV)
+    dsa.dsa_dense_mla_fwd(p, inp["q"], inp["kv"], torch.from_numpy(idx_np).to(DEV), out, lse)
+    _assert_mla_close(out, lse, *_oracle_mla(inp, idx_np))
+    for t in rows:
+        assert torch.all(out[int(t)] == 0) and torch.all(torch.isneginf(lse[int(t)]))
 
 
 def test_dense_mla_ragged_decode_masked():
