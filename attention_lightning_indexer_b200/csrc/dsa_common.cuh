@@ -64,6 +64,33 @@ __device__ __forceinline__ RowInfo row_info(const Problem &P, int t) {
     return r;
 }
 
+// row_info for a whole warp (all 32 lanes converged, the same t): a 32-way search over
+// cu_q.  The sequence of t is the last b with cu_q[b] <= t (cu_q[0] = 0 <= t keeps lane 0's
+// candidate true), found in ceil(log32(batch)) rounds of parallel loads instead of a binary
+// search's log2(batch) dependent ones; the same answer as row_info.
+__device__ __forceinline__ RowInfo row_info_warp(const Problem &P, int t) {
+    if (P.cu_q == nullptr) return row_info(P, t);
+    const int lane = threadIdx.x & 31;
+    int lo = 0, hi = P.batch;                                // the answer lies in [lo, hi)
+    while (hi - lo > 1) {
+        const int stride = (hi - lo + 31) >> 5;
+        const int b = lo + lane * stride;
+        const bool le = b < hi && __ldg(P.cu_q + b) <= t;
+        const unsigned m = __ballot_sync(0xffffffffu, le);
+        const int j = m != 0u ? 31 - __clz(m) : 0;
+        lo += j * stride;
+        hi = min(hi, lo + stride);
+    }
+    const int q0 = __ldg(P.cu_q + lo), q1 = __ldg(P.cu_q + lo + 1);
+    const int k0 = __ldg(P.cu_k + lo), k1 = __ldg(P.cu_k + lo + 1);
+    RowInfo r;
+    r.seq = lo;
+    r.kbase = k0;
+    r.len_k = k1 - k0;
+    r.pos = (k1 - k0) - (q1 - q0) + (t - q0);
+    return r;
+}
+
 // Row of the key arrays (k_idx, k_scale, kv) that holds key position s of the row's
 // sequence: packed (kbase + s) or through the block table (pages of 64 keys).  A position
 // past the sequence's last page maps to the sequence's first page (only loaded, never used).

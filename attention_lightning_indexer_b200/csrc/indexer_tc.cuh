@@ -123,7 +123,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const int r = (int)blockIdx.x / nsplit, split = (int)blockIdx.x % nsplit;
         t0 = row_begin + r;
         qcount = 1;
-        const RowInfo ri = row_info(P, t0);
+        const RowInfo ri = row_info_warp(P, t0);
         rk = ri;
         kbase = ri.kbase;
         pos0 = ri.pos;

@@ -300,7 +300,7 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         for (int j = 0, u = pair0; ok && u < units; ++j, u += npairs) {
             const int t = T - 1 - u / nsplit;
             const int split = u % nsplit;
-            const RowInfo ri = row_info(P, t);
+            const RowInfo ri = row_info_warp(P, t);
             const int32_t *irow = idx != nullptr ? idx + (int64_t)t * K : nullptr;
             const int nblocks = pair_unit_blocks<DENSE>(P, ri, irow, K, split, bps, lane);
             if (lw == 0) {
@@ -540,7 +540,7 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         for (int j = 0, u = pair0; ok && u < units; ++j, u += npairs) {
             const int t = T - 1 - u / nsplit;
             const int split = u % nsplit;
-            const RowInfo ri = row_info(P, t);
+            const RowInfo ri = row_info_warp(P, t);
             const bool got = mbar_wait(unit_full(j & 1), (j >> 1) & 1);
             const int nblocks = got ? unit_nb[j & 1] : 0;
             if (named_bar_or(1, 256, !got || misc[1] != 0)) {

@@ -584,7 +584,7 @@ __global__ void __launch_bounds__(NT, NT >= 512 ? 1 : 4) topk_rows_kernel(Proble
     if (row_mask != nullptr && row_mask[r] == 0) return;
     const int K = P.topk;
     int32_t *out = idx + (int64_t)r * K;
-    const RowInfo ri = row_info(P, row_begin + r);
+    const RowInfo ri = row_info_warp(P, row_begin + r);
     const int n = row_ok(P, ri) ? visible_keys(ri) : 0;
     if (n <= K) {   // select every visible key
         for (int j = threadIdx.x; j < K; j += NT) out[j] = j < n ? j : -1;
