@@ -227,9 +227,10 @@ dsa_status_t topk_launch(const dsa_problem_t *p, const float *scores, int64_t ld
 constexpr int MLA_PAIRS = 74;
 constexpr int MLA_MAX_SPLITS = 8;
 
-// Splits of each token's index row for the gathered attention: one pair per token when
-// the tokens alone fill the SMs (prefill, large decode batches); otherwise several pairs
-// per token, each over whole 256-slot blocks, merged by combine_splits_kernel.
+// Splits of each token's index row for the gathered attention: one unit per token when
+// the tokens alone fill the SMs (prefill, large decode batches); otherwise several units
+// (splits) per token, each over whole 256-slot blocks, each on its own CTA pair, merged by
+// combine_splits_kernel.
 void mla_split_plan(const dsa_problem_t *p, int *nsplit, int *bps) {
     const int T = p->total_q;
     const int nb = (p->topk + dsa::mla::PairCfg::BLK - 1) / dsa::mla::PairCfg::BLK;   // blocks of a row
