@@ -84,8 +84,11 @@ struct PairCfg {
     // empty[7] pfull[7] q_full q_free s_full[2] s_free[2] p_full pv_done o_ready xbar[2]
     // lbar drain unit_full[2] unit_free[2]
     static constexpr int NBARS = 2 * NSLOT + 2 + 2 + 2 + 3 + 2 + 2 + 2 + 2;
-    static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;   // [0] TMEM base, [1] abort, [2..3] unit blocks
-    static constexpr int SMEM = OFF_MISC + 16;
+    // [0] TMEM base, [1] abort, [2..3] unit blocks, [4] the peer CTA's abort flag at teardown
+    static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
+    // even CTA: [2][NSLOT] int, the last ring position each CTA issued into each slot
+    static constexpr int OFF_LASTPOS = OFF_MISC + 32;
+    static constexpr int SMEM = OFF_LASTPOS + 2 * NSLOT * 4;
     static constexpr int THREADS = 512;
     static constexpr int SOFT0 = 8;                 // first softmax warp
     static constexpr int REG_LOW = 88, REG_HIGH = 168;   // 256 x 88 + 256 x 168 = 512 x 128
@@ -263,6 +266,8 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         mbar_init(lbar, 1);
         mbar_init(drain, 1);
         misc[1] = 0;
+        misc[4] = 0;
+        for (int i = 0; i < 2 * C::NSLOT; ++i) reinterpret_cast<int *>(smem + C::OFF_LASTPOS)[i] = -1;
         fence_barrier_init();
     }
     if (tid == 0 && misaligned) {
@@ -297,6 +302,7 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         bool ok = run;
         int p = 0;                                           // ring position, counted across units
         int nq = 0;                                          // units with blocks so far
+        int last_issued = -1;                                // the last ring position this warp issued
         for (int j = 0, u = pair0; ok && u < units; ++j, u += npairs) {
             const int t = T - 1 - u / nsplit;
             const int split = u % nsplit;
@@ -349,6 +355,7 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                             if (cr == 0) mbar_expect_tx(pfull(slot), 2 * C::ATOM);   // both CTAs' tiles
                             tma_load_2d_pair(ring_s + slot * C::ATOM, &tm_kv, lead_pfull + 8u * slot, 64 * a,
                                              ri.kbase + C::BLK * b + 128 * h);
+                            last_issued = pp;
                         }
                         p += natoms;
                     }
@@ -412,6 +419,7 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                         }
                         tma_gather4_pair(ring_s + slot * C::ATOM + 512 * lane, &tm_kv, lead_pfull + 8u * slot, 64 * a,
                                          e[0], e[1], e[2], e[3]);
+                        last_issued = pp;
                     }
                     e0 = n0;
                     e1 = n1;
@@ -420,6 +428,21 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             }
         }
         if (!ok && lane == 0) abort_pair();
+        // the last position this warp issued into each of its slots, recorded in the even CTA
+        // for the drain after an abort (gathered form: warp lw owns slot lw; dense form: warp 0
+        // issued every position up to last_issued in order)
+        static_assert(C::NLOAD == C::NSLOT, "one ring slot per gathering warp");
+        if (lane == 0) {
+            const uint32_t rec = mapa_shared(sbase + C::OFF_LASTPOS + 4u * (uint32_t)(cr * C::NSLOT), 0);
+            if (DENSE) {
+                for (int sl = 0; sl < C::NSLOT; ++sl) {
+                    const int v = last_issued >= sl ? last_issued - (last_issued - sl) % C::NSLOT : -1;
+                    st_cluster_u32(rec + 4u * sl, (uint32_t)v);
+                }
+            } else {
+                st_cluster_u32(rec + 4u * lw, (uint32_t)last_issued);
+            }
+        }
         // the last q load has landed before the pair may exit (both CTAs' bytes complete on
         // the even CTA's barrier; the cluster barrier at teardown holds the odd CTA)
         if (lw == 0 && lane == 0 && cr == 0 && nq > 0) mbar_wait_cluster(q_full, (nq - 1) & 1);
@@ -786,9 +809,24 @@ sparse_mla_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
             if (nblocks > 0) ++nq;
         }
     }
-    // ---- teardown: nothing of either CTA is in flight past this point
+    // ---- teardown: nothing of either CTA is in flight past this point.  After an abort
+    // (either CTA's flag, so both take the same branch) the even CTA first waits, bounded,
+    // until the last position either CTA issued into each slot has landed.  Each CTA hands
+    // its final flag to the peer before the cluster barrier: past that barrier the peer may
+    // already have exited, so nothing reads the peer's shared memory there.
     tc_fence_before();
+    __syncthreads();                                         // this CTA's roles are done
+    if (tid == 0) st_cluster_u32(mapa_shared(sbase + C::OFF_MISC + 16, (uint32_t)peer), misc[1]);
     cluster_sync();
+    const bool aborted = misc[1] != 0u || misc[4] != 0u;     // the same in both CTAs
+    if (aborted) {
+        if (cr == 0 && run && tid < C::NSLOT) {
+            const int *lp = reinterpret_cast<const int *>(smem + C::OFF_LASTPOS);
+            const int pmax = max(lp[tid], lp[C::NSLOT + tid]);
+            if (pmax >= 0) mbar_wait_cluster(pfull(tid), (uint32_t)(pmax / C::NSLOT) & 1u);
+        }
+        cluster_sync();
+    }
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc_pair(tmem, 512);
