@@ -43,12 +43,11 @@ FLOP_PER_PAIR_MLA = 128 * (576 + 512) * 2       # per (query, selected key) pair
 # sha256 of the source file it was captured from; reported only while the source is
 # unchanged.
 TRAFFIC = {
-    # ncu capture of the 4096-query prefill launch (persistent pairs): 1.143 GB of DRAM
-    # traffic (642 MB read, 501 MB written: q reads and out writes, both proportional to the
+    # ncu capture of the 4096-query prefill launch (persistent pairs): 1.141 GB of DRAM
+    # traffic (642 MB read, 499 MB written: q reads and out writes, both proportional to the
     # query count; kv rows come from L2), scaled x8 to the 32768-query launch of the 32K step
-    # (that prefill only: at 128K the kv rows no longer fit in L2); the hash is of the source
-    # as captured plus comment-only edits
-    "sparse_mla": {"bytes_per_launch": 1.142902e9 * 8, "total_q": 32768, "src_sha": "730f3743a3d16970"},
+    # (that prefill only: at 128K the kv rows no longer fit in L2)
+    "sparse_mla": {"bytes_per_launch": 1.140993e9 * 8, "total_q": 32768, "src_sha": "ad33592d1748a857"},
 }
 
 
