@@ -194,6 +194,14 @@ def _tokens(inp):
     return int(inp["total_q"])
 
 
+def _config(args, inp, chunk, ws):
+    """The workload's `config`, the same for both arms (how each arm runs it is stated in its
+    own keys: `cpu_baseline.sample` for the reference arm)."""
+    return {"workload": args.workload, "global_batch": ws * inp["batch"], "seq_len": int(inp["max_len_k"]),
+            "topk": inp["topk"], "chunk_q": chunk, "parallelism": f"replicas x{ws}",
+            "l2": "flushed between timed steps (2 x 126 MB write) and inputs > L2"}
+
+
 # Longest key sequence the library's forward attends in the dense (masked) form alone
 # (include/dsa.h, dsa_forward).
 DENSE_KV_THRESHOLD = 3584
@@ -280,9 +288,7 @@ def run_ours(args, ws, rank, local, dist):
         "vs_baseline": None,
         "dtype": "bf16" if "q_idx8" not in inp else "e4m3 indexer + bf16 attention",
         "data": "synthetic (seeded; shapes and distributions of the workload recipe)",
-        "config": {"workload": args.workload, "global_batch": ws * inp["batch"], "seq_len": int(inp["max_len_k"]),
-                   "topk": inp["topk"], "chunk_q": chunk, "parallelism": f"replicas x{ws}",
-                   "l2": "flushed between timed steps (2 x 126 MB write) and inputs > L2"},
+        "config": _config(args, inp, chunk, ws),
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
     }
@@ -660,8 +666,7 @@ def run_reference(args, ws, rank, local):
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded; same recipe)",
-        "config": {"workload": args.workload, "global_batch": inp["batch"], "seq_len": int(inp["max_len_k"]),
-                   "topk": inp["topk"], "chunk_q": wl.chunk, "parallelism": "host cores (rank 0 only)"},
+        "config": _config(args, inp, args.chunk if args.chunk is not None else wl.chunk, ws),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
                          "cpu_model": _cpu_model(),
                          "sample": f"{per_step} uniformly drawn query rows per step of the same workload, fp64"},
