@@ -91,3 +91,27 @@ def test_metric_and_flop_constants_match_the_problem_shapes():
     assert bench.FLOP_PER_PAIR_MLA == 128 * (576 + 512) * 2
     assert "32K prefill" in bench.METRIC and "decode" in bench.METRIC
     assert np.isclose(bench.L2_BYTES, 126 * 2 ** 20)
+
+
+def test_attention_launch_count_follows_the_forward_forms():
+    # the forward's attention: the dense form alone up to the short-sequence threshold; in
+    # one packed sequence the rows that see at most topk keys take the dense form and the
+    # rest the gathered form (two launches); ragged or paged problems take one launch
+    import attention_lightning_indexer_b200 as dsa
+    assert bench._attention_launches(dsa.make_problem(1, 2048, 2048, 2048, 2048, 2048)) == 1
+    assert bench._attention_launches(dsa.make_problem(1, 3584, 3584, 3584, 3584, 2048)) == 1
+    assert bench._attention_launches(dsa.make_problem(1, 32768, 32768, 32768, 32768, 2048)) == 2
+    # every row sees more than topk keys: gathered only
+    assert bench._attention_launches(dsa.make_problem(1, 512, 40000, 512, 40000, 2048)) == 1
+    # every row sees at most topk keys (but the sequence is longer than the threshold)
+    assert bench._attention_launches(dsa.make_problem(1, 4000, 4000, 4000, 4000, 8192)) == 1
+
+
+def test_workload_config_names_the_workload_and_its_launch_shape():
+    # one helper builds the config of both arms (ours and --impl reference)
+    import argparse
+    args = argparse.Namespace(workload="prefill_32k")
+    cfg = bench._config(args, {"batch": 1, "max_len_k": 32768, "topk": 2048}, 8192, 2)
+    assert (cfg["workload"], cfg["global_batch"], cfg["seq_len"], cfg["topk"], cfg["chunk_q"]) == \
+        ("prefill_32k", 2, 32768, 2048, 8192)
+    assert cfg["parallelism"] == "replicas x2" and "l2" in cfg
