@@ -380,6 +380,22 @@ def _check_forward_rows(inp, rows, chunk=0):
     return idx, out, lse
 
 
+def test_forward_ragged_batch_of_70_with_sequences_without_queries():
+    # 70 sequences: more than one warp's worth of candidates, so each kernel's search over
+    # cu_q takes two rounds; 0 to 6 queries per sequence, the first, last and the ones around
+    # the warp boundary without any
+    inp = dsa_synth.make_decode(70, 300, 3000, topk=256, seed=41, device=DEV, q_per_seq=6)
+    rng = np.random.default_rng(41)
+    qc = rng.integers(0, 7, 70)
+    qc[[0, 5, 31, 32, 33, 69]] = 0
+    T = int(qc.sum())
+    for name in ("q_idx", "w", "q"):
+        inp[name] = inp[name][:T].contiguous()
+    inp["cu_q"] = torch.from_numpy(np.concatenate([[0], np.cumsum(qc)]).astype(np.int32)).to(DEV)
+    inp["total_q"], inp["max_len_q"] = T, int(qc.max())
+    _check_forward_rows(inp, np.arange(T))
+
+
 def test_forward_pr_reference_config_all_rows():
     inp = dsa_synth.make_workload("pr_ref_256", seed=0, device=DEV)
     _check_forward_rows(inp, np.arange(256))
