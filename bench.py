@@ -394,7 +394,9 @@ def _decode_secondary(dsa, args, rank, dev, stream, flush, dist):
 
 
 def _breakdown(dsa, p, inp, fa, chunk, dev, stream, flush, reps=2, decode=False):
-    """Average device time of each kernel of the step, timed with CUDA events on the launch stream."""
+    """Average device time of each kernel of the step: each call is captured once as a CUDA
+    graph (its host-side argument set-up happens at capture) and replayed between CUDA events
+    on the bench stream, L2 flushed before each replay."""
     T = inp["total_q"]
     chunk = chunk or T
     ld = dsa.scores_ld(inp["max_len_k"])
@@ -405,27 +407,30 @@ def _breakdown(dsa, p, inp, fa, chunk, dev, stream, flush, reps=2, decode=False)
     t_idx = t_topk = t_mla = 0.0
     n_idx = n_topk = n_mla = 0
 
-    def timed(fn):
+    def timed(call):
+        graph = _capture(call, dev)
         flush.zero_()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        fn()
-        b.record(stream)
+        with torch.cuda.stream(stream):
+            a.record(stream)
+            graph.replay()
+            b.record(stream)
         b.synchronize()
+        del graph
         return a.elapsed_time(b)
 
     for _ in range(reps):
         for r0 in range(0, T, chunk):
             rc = min(chunk, T - r0)
-            t_idx += timed(lambda: dsa.dsa_indexer_scores(p, fa["q_idx"], fa["k_idx"], inp["w"], scores, row_begin=r0,
-                                                          row_count=rc, q_scale=fa["q_scale"], k_scale=fa["k_scale"],
-                                                          stream=stream))
-            t_topk += timed(lambda: dsa.dsa_topk(p, scores, idx[r0:r0 + rc], row_begin=r0, row_count=rc,
-                                                 stream=stream))
+            t_idx += timed(lambda st: dsa.dsa_indexer_scores(p, fa["q_idx"], fa["k_idx"], inp["w"], scores,
+                                                             row_begin=r0, row_count=rc, q_scale=fa["q_scale"],
+                                                             k_scale=fa["k_scale"], stream=st))
+            t_topk += timed(lambda st: dsa.dsa_topk(p, scores, idx[r0:r0 + rc], row_begin=r0, row_count=rc,
+                                                    stream=st))
             n_idx += 1
             n_topk += 1
-        t_mla += timed(lambda: dsa.dsa_sparse_mla_fwd(p, inp["q"], inp["kv"], idx, out, lse, stream=stream))
+        t_mla += timed(lambda st: dsa.dsa_sparse_mla_fwd(p, inp["q"], inp["kv"], idx, out, lse, stream=st))
         n_mla += 1
     idx_pairs, mla_pairs, topk_bytes = _pairs(inp)
     pk = _peaks()

@@ -267,11 +267,14 @@ def _dense_causal_sdpa(q, kv, scale, d_v):
     kt = torch.from_numpy(kv)[None, None].expand(1, q.shape[1], -1, -1)
     vt = torch.from_numpy(kv[:, :d_v].copy())[None, None].expand(1, q.shape[1], -1, -1)
     o = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=True, scale=scale)
-    z = torch.einsum("bhld,bhsd->bhls", qt, kt) * scale
+    # lse from numpy's own einsum loops (no BLAS): torch's first fp64 CPU einsum in a process
+    # was seen to land 1e-9 away from later calls on the same inputs
+    z = np.einsum("lhd,sd->hls", q, kv, optimize=False) * scale
     L = q.shape[0]
-    mask = torch.ones(L, L, dtype=torch.bool).tril()
-    lse = torch.logsumexp(z.masked_fill(~mask, -float("inf")), dim=-1)
-    return o[0].permute(1, 0, 2).numpy(), lse[0].permute(1, 0).numpy()
+    z = np.where(np.tril(np.ones((L, L), dtype=bool))[None], z, -np.inf)
+    m = z.max(axis=-1, keepdims=True)
+    lse = (m[..., 0] + np.log(np.exp(z - m).sum(axis=-1)))
+    return o[0].permute(1, 0, 2).numpy(), lse.T
 
 
 def test_sparse_mla_equals_dense_causal_attention_when_k_covers_all():
